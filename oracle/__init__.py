@@ -1,0 +1,156 @@
+"""fp64 CPU oracle for the Monarch product and its backward.
+
+TEST INFRASTRUCTURE ONLY: imported by ``tests/``, by ``__graft_entry__.smoke()``
+and by the CPU-baseline leg of ``bench.py``, never by the product package.
+It shares no code with the CUDA path; the two meet only through the seeded
+input generator (``block_diagonal_linear_b200.synthetic``), which holds no
+arithmetic of the method.
+
+The arithmetic lives in ``monarch_oracle.c`` (plain loops in ``double``);
+this module compiles it with gcc on first use and calls it through ctypes.
+Every function takes and returns float64 numpy arrays.
+
+Sources (web pages on Monarch matrices): the Monarch abstract (product of two
+block-diagonal matrices), the scatterbrain "Definition C.3" issue (M = L R up to
+permutations; R has b blocks, L has n/b), the MonarchLinear factor shapes
+(nblocks, out_blk, in_blk), the unofficial-implementation comment (permutation
+[x0, x2, x1, x3] for N=4, lattice view) and the workload descriptions
+(reshape, transpose, flatten). Every function is pinned by tests in
+``tests/test_oracle_pins.py``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "monarch_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lib = None
+
+
+class _Dims(ctypes.Structure):
+    _fields_ = [
+        ("rows", ctypes.c_int64),
+        ("nb1", ctypes.c_int),
+        ("in1", ctypes.c_int),
+        ("out1", ctypes.c_int),
+        ("nb2", ctypes.c_int),
+        ("in2", ctypes.c_int),
+        ("out2", ctypes.c_int),
+        ("out_transpose", ctypes.c_int),
+    ]
+
+
+def build(force: bool = False) -> str:
+    """Compile the C oracle into ``oracle/liboracle.so`` (gcc, -O2, pthreads)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + ".tmp%d" % os.getpid()
+        subprocess.check_call(
+            ["gcc", "-O2", "-std=c99", "-shared", "-fPIC", "-pthread", _SRC, "-o", tmp]
+        )
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(build())
+        dp = ctypes.POINTER(ctypes.c_double)
+        lib.mo_forward.argtypes = [ctypes.POINTER(_Dims), dp, dp, dp, dp, ctypes.c_int]
+        lib.mo_backward.argtypes = [ctypes.POINTER(_Dims), dp, dp, dp, dp, dp, dp, dp, ctypes.c_int]
+        lib.mo_materialise.argtypes = [ctypes.POINTER(_Dims), dp, dp, dp]
+        for f in (lib.mo_forward, lib.mo_backward, lib.mo_materialise):
+            f.restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def _dims(d: dict, rows: int) -> _Dims:
+    return _Dims(
+        int(rows), d["nb1"], d["in1"], d["out1"], d["nb2"], d["in2"], d["out2"],
+        int(d.get("out_transpose", 1)),
+    )
+
+
+def _p(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+
+def _f64(a) -> np.ndarray:
+    return np.ascontiguousarray(np.asarray(a, dtype=np.float64))
+
+
+def default_threads() -> int:
+    try:
+        return max(1, len(os.sched_getaffinity(0)))
+    except AttributeError:  # pragma: no cover
+        return max(1, os.cpu_count() or 1)
+
+
+def sizes(d: dict) -> tuple[int, int, int]:
+    """(n_in, n_mid, n_out) of a Monarch shape."""
+    return d["nb1"] * d["in1"], d["nb1"] * d["out1"], d["nb2"] * d["out2"]
+
+
+def forward(d: dict, X, R, L, nthreads: int | None = None) -> np.ndarray:
+    """Y = X M^T, row by row (steps a1..a5), in fp64."""
+    X, R, L = _f64(X), _f64(R), _f64(L)
+    n_in, _, n_out = sizes(d)
+    X2 = X.reshape(-1, n_in)
+    Y = np.zeros((X2.shape[0], n_out), dtype=np.float64)
+    rc = _load().mo_forward(
+        ctypes.byref(_dims(d, X2.shape[0])), _p(X2), _p(R), _p(L), _p(Y),
+        nthreads or default_threads(),
+    )
+    if rc != 0:
+        raise ValueError("oracle: bad Monarch dims %r" % (d,))
+    return Y
+
+
+def backward(d: dict, dY, X, R, L, nthreads: int | None = None):
+    """(dX, dR, dL) by the chain rule (steps a6..a10), Z recomputed, in fp64."""
+    dY, X, R, L = _f64(dY), _f64(X), _f64(R), _f64(L)
+    n_in, _, n_out = sizes(d)
+    X2 = X.reshape(-1, n_in)
+    dY2 = dY.reshape(-1, n_out)
+    dX = np.zeros_like(X2)
+    dR = np.zeros((d["nb1"], d["out1"], d["in1"]), dtype=np.float64)
+    dL = np.zeros((d["nb2"], d["out2"], d["in2"]), dtype=np.float64)
+    rc = _load().mo_backward(
+        ctypes.byref(_dims(d, X2.shape[0])), _p(dY2), _p(X2), _p(R), _p(L), _p(dX), _p(dR),
+        _p(dL), nthreads or default_threads(),
+    )
+    if rc != 0:
+        raise ValueError("oracle: bad Monarch dims %r" % (d,))
+    return dX, dR, dL
+
+
+def materialise(d: dict, R, L) -> np.ndarray:
+    """Dense M (n_out, n_in), Y = X M^T, from the closed form of the product."""
+    R, L = _f64(R), _f64(L)
+    n_in, _, n_out = sizes(d)
+    M = np.zeros((n_out, n_in), dtype=np.float64)
+    rc = _load().mo_materialise(ctypes.byref(_dims(d, 0)), _p(R), _p(L), _p(M))
+    if rc != 0:
+        raise ValueError("oracle: bad Monarch dims %r" % (d,))
+    return M
+
+
+def param_count(d: dict) -> int:
+    return d["nb1"] * d["out1"] * d["in1"] + d["nb2"] * d["out2"] * d["in2"]
+
+
+def normwise_rel_err(got, ref) -> float:
+    """||got - ref||_F / ||ref||_F in fp64 (0 when both are zero)."""
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    den = float(np.linalg.norm(ref.ravel()))
+    num = float(np.linalg.norm((got - ref).ravel()))
+    if den == 0.0:
+        return 0.0 if num == 0.0 else float("inf")
+    return num / den
