@@ -1,0 +1,421 @@
+"""Benchmark of the Monarch training step (forward + backward) on B200 GPUs.
+
+python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A step is one pass of the whole hot path over one batch: forward Y = X M^T
+(R stage, permutation, L stage, output permutation) and backward (dX, dR, dL).
+With N > 1 (launched by torchrun, one rank per GPU) every rank runs its own
+batch of the same size (weak scaling, rows sharded across ranks) and the weight
+gradients are summed over ranks with NCCL all-reduce, the one exchange step of
+data-parallel training.
+
+Inputs are seeded synthetic tensors with the workload's shapes and value
+distributions.  Timing: CUDA events on the launching stream around each pass;
+L2 is flushed (256 MiB write, untimed) before every timed pass; max over ranks.
+Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from block_diagonal_linear_b200 import synthetic  # noqa: E402
+
+DEFAULT_WORKLOAD = "n1024_bf16"
+METRIC = "Monarch fwd/bwd rows/s and TFLOP/s at 1 B200; achieved % of roofline per shape"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def describe(name: str, w: dict) -> str:
+    return ("%s: R %d blocks of %dx%d, L %d blocks of %dx%d, %d->%d, out_transpose=%d, "
+            "%d rows, %s" % (name, w["nb1"], w["out1"], w["in1"], w["nb2"], w["out2"], w["in2"],
+                             w["nb1"] * w["in1"], w["nb2"] * w["out2"], w["out_transpose"],
+                             w["rows"], w["dtype"]))
+
+
+def algorithmic(w: dict, rows: int) -> dict:
+    """Algorithmic flops and HBM bytes per pass: read inputs and factors once, write
+    outputs once (no intermediates, no recompute)."""
+    n_in, _, n_out = synthetic.sizes(w)
+    params = w["nb1"] * w["out1"] * w["in1"] + w["nb2"] * w["out2"] * w["in2"]
+    es = 2 if w["dtype"] == "bf16" else 4
+    return {
+        "fwd": {"flops": 2.0 * rows * params,
+                "bytes": float(es * (rows * n_in + params + rows * n_out))},
+        "bwd": {"flops": 4.0 * rows * params,
+                "bytes": float(es * (rows * n_out + 2 * rows * n_in + 2 * params))},
+        "params": params,
+    }
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        d = json.load(open(p))
+        return {k: float(d[k]) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")}, \
+            "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def source_hash(files) -> str:
+    h = hashlib.sha256()
+    for f in files:
+        h.update(open(os.path.join(ROOT, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic(kernel: str, srcs) -> float | None:
+    """DRAM bytes per launch from a committed ncu summary, if the kernel source is unchanged."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        d = json.load(open(p))[kernel]
+    except Exception:
+        return None
+    if d.get("source_sha") != source_hash(srcs):
+        return None
+    return float(d["dram_bytes_per_launch_full"])
+
+
+# --------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while the timed region runs."""
+
+    REASONS = {
+        "hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40, "sw_thermal_slowdown": 0x20,
+        "sw_power_cap": 0x4, "hw_power_brake_slowdown": 0x80,
+    }
+
+    def __init__(self, device_index: int):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        self.ok = False
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            props = torch.cuda.get_device_properties(device_index)
+            bus = "%08x:%02x:%02x.0" % (props.pci_domain_id, props.pci_bus_id, props.pci_device_id)
+            self.h = pynvml.nvmlDeviceGetHandleByPciBusId(bus.encode())
+            self.nv = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # pragma: no cover - depends on the box
+            self.err = repr(e)
+
+    def _sample(self):
+        self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+        mask = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+        for name, bit in self.REASONS.items():
+            if mask & bit:
+                self.reasons.add(name)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self._sample()
+            except Exception:
+                pass
+            time.sleep(0.005)
+
+    def __enter__(self):
+        if self.ok:
+            self._sample()
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+            self._sample()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [],
+                    "note": "NVML unavailable"}
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# --------------------------------------------------------------------------- oracle arm
+def oracle_rate(w: dict, seed: int = 0, budget_s: float = 8.0):
+    """Rows/s of the fp64 CPU oracle (forward + backward) on a bounded sample of the
+    workload, all host cores.  Test infrastructure, timed as the CPU baseline."""
+    import oracle
+    shape = synthetic.shape_of(w)
+    params = algorithmic(w, 1)["params"]
+    # size the sample so one fwd+bwd pass is about budget_s / 4 at ~0.5 GFLOP/s/core
+    cores = oracle.default_threads()
+    per_row = 6.0 * params
+    rows = int(max(cores, min(w["rows"], budget_s / 4 * 0.5e9 * cores / per_row)))
+    inp = synthetic.make_inputs(w, seed=seed, rows=rows)
+    X, R, L, dY = inp["X"].f64, inp["R"].f64, inp["L"].f64, inp["dY"].f64
+    done, t0 = 0, time.perf_counter()
+    while True:
+        oracle.forward(shape, X, R, L, nthreads=cores)
+        oracle.backward(shape, dY, X, R, L, nthreads=cores)
+        done += rows
+        if time.perf_counter() - t0 >= budget_s or done >= 64 * rows:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": done / dt, "unit": "rows/s", "cores": cores, "kind": "oracle",
+            "sample": "%d rows of %s (forward+backward, fp64, %d passes, %.1f s)"
+                      % (rows, w.get("name", "workload"), done // rows, dt),
+            "tflops": 6.0 * params * done / dt / 1e12}
+
+
+def run_reference(args, w, name):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+    shape = synthetic.shape_of(w)
+    params = algorithmic(w, 1)["params"]
+    cores = oracle.default_threads()
+    rows = int(max(cores, min(w["rows"], 1.0 * 0.5e9 * cores / (6.0 * params))))
+    inp = synthetic.make_inputs(w, seed=0, rows=rows)
+    X, R, L, dY = inp["X"].f64, inp["R"].f64, inp["L"].f64, inp["dY"].f64
+    for _ in range(args.warmup):
+        oracle.forward(shape, X, R, L)
+        oracle.backward(shape, dY, X, R, L)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.forward(shape, X, R, L)
+        oracle.backward(shape, dY, X, R, L)
+    dt = time.perf_counter() - t0
+    value = rows * args.steps / dt
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "rows/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * dt / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": describe(name, w), "rows_per_step": rows,
+                   "note": "fp64 CPU oracle on a bounded sample of the workload's rows"},
+        "cpu_baseline": {"value": value, "unit": "rows/s", "cores": cores, "kind": "oracle",
+                         "sample": "%d of %d rows per step" % (rows, w["rows"])},
+        "e2e": {"value": value, "unit": "rows/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+# --------------------------------------------------------------------------- GPU arm
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synthetic.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    name = args.workload
+    w = dict(synthetic.WORKLOADS[name], name=name)
+
+    if args.impl == "reference":
+        run_reference(args, w, name)
+        return
+
+    import torch
+    import torch.distributed as dist
+    import block_diagonal_linear_b200 as bdl
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit("--gpus %d but WORLD_SIZE=%d" % (args.gpus, world))
+    torch.cuda.set_device(local)
+    dev_ = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev_)
+
+    shape = synthetic.shape_of(w)
+    rows = w["rows"]  # per rank (weak scaling)
+    inp = synthetic.make_inputs(w, seed=1000 + rank)
+    def to_dev(t):
+        if t.dtype == "bf16":
+            return torch.from_numpy(t.bits.view(np.int16).copy()).view(torch.bfloat16).to(dev_)
+        return torch.from_numpy(np.ascontiguousarray(t.bits)).to(dev_)
+
+    X, R, L, dY = (to_dev(inp[k]) for k in ("X", "R", "L", "dY"))
+    n_in, _, n_out = synthetic.sizes(w)
+    Y = torch.empty((rows, n_out), dtype=X.dtype, device=dev_)
+    dX = torch.empty_like(X)
+    dR = torch.empty_like(R)
+    dL = torch.empty_like(L)
+    ws = torch.empty(max(bdl.bwd_workspace_bytes(shape, rows, w["dtype"]), 256), dtype=torch.uint8,
+                     device=dev_)
+    l2 = torch.cuda.get_device_properties(dev_).L2_cache_size
+    flush = torch.empty(max(2 * l2, 256 << 20), dtype=torch.uint8, device=dev_)
+    stream = torch.cuda.current_stream()
+
+    def allreduce_grads():
+        if world > 1:
+            dist.all_reduce(dR)
+            dist.all_reduce(dL)
+
+    def step(ev=None):
+        if ev is not None:
+            flush.zero_()
+            ev[0].record(stream)
+        bdl.fwd(X, R, L, shape, Y=Y)
+        if ev is not None:
+            ev[1].record(stream)
+            flush.zero_()
+            ev[2].record(stream)
+        bdl.bwd(dY, X, R, L, shape, dX=dX, dR=dR, dL=dL, workspace=ws)
+        allreduce_grads()
+        if ev is not None:
+            ev[3].record(stream)
+
+    for _ in range(args.warmup):
+        step([torch.cuda.Event(enable_timing=True) for _ in range(4)])
+    torch.cuda.synchronize()
+    if bdl.last_device_status() != 0:
+        raise SystemExit("device status not OK after warm-up")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    sampler = ClockSampler(local)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with sampler:
+        for k in range(args.steps):
+            step(evs[k])
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    fwd_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    bwd_ms = [e[2].elapsed_time(e[3]) for e in evs]
+    tot_ms = sum(fwd_ms) + sum(bwd_ms)
+    if world > 1:
+        t = torch.tensor([tot_ms, sum(fwd_ms), sum(bwd_ms)], dtype=torch.float64, device=dev_)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        tot_ms, fwd_sum, bwd_sum = t.tolist()
+    else:
+        fwd_sum, bwd_sum = sum(fwd_ms), sum(bwd_ms)
+    status = bdl.last_device_status()
+
+    # ---- end to end through the public API with host buffers (pinned), copies timed
+    Xh = torch.empty_like(X, device="cpu").pin_memory()
+    Xh.copy_(X)
+    dYh = torch.empty_like(dY, device="cpu").pin_memory()
+    dYh.copy_(dY)
+    outs_h = [torch.empty_like(t, device="cpu").pin_memory() for t in (Y, dX, dR, dL)]
+    Xe, dYe = torch.empty_like(X), torch.empty_like(dY)
+    n_e2e = max(3, min(args.steps, 50))
+
+    def e2e_step():
+        Xe.copy_(Xh, non_blocking=True)
+        dYe.copy_(dYh, non_blocking=True)
+        bdl.fwd(Xe, R, L, shape, Y=Y)
+        bdl.bwd(dYe, Xe, R, L, shape, dX=dX, dR=dR, dL=dL, workspace=ws)
+        allreduce_grads()
+        for h, d_ in zip(outs_h, (Y, dX, dR, dL)):
+            h.copy_(d_, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(n_e2e):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev_)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = t.item()
+    h2d = X.numel() * X.element_size() + dY.numel() * dY.element_size()
+    d2h = sum(t.numel() * t.element_size() for t in (Y, dX, dR, dL))
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+
+    peaks, peak_src = load_peaks()
+    alg = algorithmic(w, rows)
+    K = args.steps
+    fwd_avg_s = fwd_sum / K / 1e3
+    bwd_avg_s = bwd_sum / K / 1e3
+    hbm = peaks["hbm_gbs"] * 1e9
+    tpk = peaks["bf16_tflops"] * 1e12
+    passes = {}
+    for pname, t_s in (("fwd", fwd_avg_s), ("bwd", bwd_avg_s)):
+        a = alg[pname]
+        t_roof = max(a["bytes"] / hbm, a["flops"] / tpk)
+        passes[pname] = {
+            "ms": t_s * 1e3, "rows_per_s": rows / t_s, "tflops": a["flops"] / t_s / 1e12,
+            "gbs": a["bytes"] / t_s / 1e9, "roofline_ms": t_roof * 1e3,
+            "roofline_frac": t_roof / t_s,
+            "bound": "hbm" if a["bytes"] / hbm >= a["flops"] / tpk else "tensor",
+        }
+    fwd_tc = bdl.fwd_path(shape, w["dtype"]) == 1
+    launches_per_step = 1 + 3
+    dom = "fwd" if fwd_avg_s >= bwd_avg_s else "bwd"
+    a = alg[dom]
+    t_dom = fwd_avg_s if dom == "fwd" else bwd_avg_s
+    bound = passes[dom]["bound"]
+    kname = ("tc_fwd_kernel" if fwd_tc else "gen_fwd_kernel") if dom == "fwd" else "monarch_bwd"
+    srcs = ["block_diagonal_linear_b200/csrc/tc_fwd.cu", "block_diagonal_linear_b200/csrc/ptx.cuh"]
+    if bound == "hbm":
+        roof = {"bound": "hbm", "achieved": a["bytes"] / t_dom / 1e9, "peak": peaks["hbm_gbs"],
+                "unit": "GB/s"}
+    else:
+        roof = {"bound": "tensor", "achieved": a["flops"] / t_dom / 1e12,
+                "peak": peaks["bf16_tflops"], "unit": "TFLOP/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["traffic"] = measured_traffic(kname, srcs) if dom == "fwd" and fwd_tc else None
+    roof["kernel"] = kname + (" (pass of 3 kernels)" if dom == "bwd" else "")
+    roof["algorithmic_bytes_per_launch"] = a["bytes"]
+    roof["peak_source"] = peak_src
+
+    value = world * rows * K / (tot_ms / 1e3)
+    out = {
+        "metric": METRIC, "value": value, "unit": "rows/s", "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": tot_ms / K, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": w["dtype"], "data": "synthetic",
+        "config": {"workload": describe(name, w), "rows_per_gpu": rows,
+                   "step": "forward + backward (dX, dR, dL)" +
+                           (" + NCCL all-reduce of dR, dL" if world > 1 else ""),
+                   "l2": "flushed before every timed pass (%d MiB write, untimed)"
+                         % (flush.numel() >> 20),
+                   "parallelism": "dp%d" % world},
+        "tflops": (alg["fwd"]["flops"] + alg["bwd"]["flops"]) * world * K / (tot_ms / 1e3) / 1e12,
+        "passes": passes,
+        "roofline": roof,
+        "e2e": {"value": world * rows * n_e2e / (e2e_ms / 1e3), "unit": "rows/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": n_e2e},
+        "gpu_launches": launches_per_step * K,
+        "clocks": sampler.summary(),
+        "device_status": status,
+    }
+    if not args.no_cpu_baseline and world == 1:
+        out["cpu_baseline"] = oracle_rate(w)
+    print(json.dumps(out), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,225 @@
+"""B200 (sm_100a) Monarch linear map: Python binding of libmonarch.so.
+
+This module only marshals arguments: every step of the forward and backward
+runs in the CUDA kernels behind the C ABI declared in ``include/monarch.h``.
+PyTorch provides device memory and the current CUDA stream.  There is no CPU
+fallback: if the library or a GPU is missing, calls raise.
+
+    Y = X M^T,   M = P_out L P R   (Monarch: products of two block-diagonal
+    matrices with a reshape-transpose permutation; scatterbrain issue thread,
+    Definition C.3 and the N=4 permutation example)
+
+Shapes use the MonarchLinear convention: R is (nb1, out1, in1), L is
+(nb2, out2, in2), X is (rows, nb1*in1), Y is (rows, nb2*out2).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libmonarch.so")
+
+MONARCH_F32 = 0
+MONARCH_BF16 = 1
+
+STATUS = {
+    0: "MONARCH_OK",
+    -1: "MONARCH_ERR_DIMS",
+    -2: "MONARCH_ERR_DTYPE",
+    -3: "MONARCH_ERR_ALIGN",
+    -4: "MONARCH_ERR_NULL",
+    -5: "MONARCH_ERR_WORKSPACE",
+    -6: "MONARCH_ERR_CUDA",
+    -7: "MONARCH_ERR_TIMEOUT",
+    -8: "MONARCH_ERR_UNSUPPORTED",
+}
+CODES = {v: k for k, v in STATUS.items()}
+
+EXPORTED = (
+    "monarch_validate", "monarch_fwd", "monarch_bwd", "monarch_bwd_workspace_bytes",
+    "monarch_materialise", "monarch_status_string", "monarch_last_device_status",
+    "monarch_debug_wait_timeout", "monarch_fwd_path", "monarch_bwd_path",
+)
+
+
+class MonarchDims(ctypes.Structure):
+    """Mirror of ``monarch_dims`` in include/monarch.h."""
+    _fields_ = [
+        ("rows", ctypes.c_int64),
+        ("nb1", ctypes.c_int32),
+        ("in1", ctypes.c_int32),
+        ("out1", ctypes.c_int32),
+        ("nb2", ctypes.c_int32),
+        ("in2", ctypes.c_int32),
+        ("out2", ctypes.c_int32),
+        ("out_transpose", ctypes.c_int32),
+        ("dtype", ctypes.c_int32),
+    ]
+
+
+class MonarchError(RuntimeError):
+    def __init__(self, fn: str, code: int):
+        self.code = code
+        super().__init__("%s failed: %s (%d)" % (fn, STATUS.get(code, "?"), code))
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libmonarch.so (built in-tree by ``block_diagonal_linear_b200.build``)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                "libmonarch.so is not built; run `python -m block_diagonal_linear_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, dp = ctypes.c_void_p, ctypes.POINTER(MonarchDims)
+        L.monarch_validate.argtypes = [dp]
+        L.monarch_fwd.argtypes = [vp, vp, vp, dp, vp, vp]
+        L.monarch_bwd.argtypes = [vp, vp, vp, vp, dp, vp, vp, vp, vp, ctypes.c_size_t, vp]
+        L.monarch_bwd_workspace_bytes.argtypes = [dp]
+        L.monarch_bwd_workspace_bytes.restype = ctypes.c_size_t
+        L.monarch_materialise.argtypes = [vp, vp, dp, vp, vp]
+        L.monarch_status_string.argtypes = [ctypes.c_int]
+        L.monarch_status_string.restype = ctypes.c_char_p
+        L.monarch_last_device_status.argtypes = [vp]
+        L.monarch_debug_wait_timeout.argtypes = [ctypes.c_uint64, vp]
+        L.monarch_fwd_path.argtypes = [dp]
+        L.monarch_bwd_path.argtypes = [dp]
+        for name in ("monarch_validate", "monarch_fwd", "monarch_bwd", "monarch_materialise",
+                     "monarch_last_device_status", "monarch_debug_wait_timeout",
+                     "monarch_fwd_path", "monarch_bwd_path"):
+            getattr(L, name).restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def make_dims(shape: dict, rows: int, dtype) -> MonarchDims:
+    """Build a ``monarch_dims`` from a shape dict (nb1, in1, out1, nb2, in2, out2,
+    out_transpose), a row count and a dtype ('bf16' / 'f32' / torch dtype / code)."""
+    return MonarchDims(
+        int(rows), int(shape["nb1"]), int(shape["in1"]), int(shape["out1"]), int(shape["nb2"]),
+        int(shape["in2"]), int(shape["out2"]), int(shape.get("out_transpose", 1)),
+        dtype_code(dtype),
+    )
+
+
+def dtype_code(dtype) -> int:
+    if isinstance(dtype, int):
+        return dtype
+    if isinstance(dtype, str):
+        return {"bf16": MONARCH_BF16, "f32": MONARCH_F32, "fp32": MONARCH_F32}[dtype]
+    import torch
+    return {torch.bfloat16: MONARCH_BF16, torch.float32: MONARCH_F32}[dtype]
+
+
+def _torch_dtype(code: int):
+    import torch
+    return torch.bfloat16 if code == MONARCH_BF16 else torch.float32
+
+
+def _check(fn: str, rc: int):
+    if rc != 0:
+        raise MonarchError(fn, rc)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    import torch
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _require_cuda(*ts):
+    for t in ts:
+        if t is not None and (not t.is_cuda or not t.is_contiguous()):
+            raise ValueError("Monarch kernels take contiguous CUDA tensors")
+
+
+def validate(shape: dict, rows: int = 0, dtype="bf16") -> int:
+    """Host-only shape check; returns the status code (0 = valid)."""
+    return lib().monarch_validate(ctypes.byref(make_dims(shape, rows, dtype)))
+
+
+def fwd_path(shape: dict, dtype="bf16") -> int:
+    """0 = generic FMA kernels, 1 = fused tcgen05 kernel (host-only query)."""
+    return lib().monarch_fwd_path(ctypes.byref(make_dims(shape, 1, dtype)))
+
+
+def bwd_path(shape: dict, dtype="bf16") -> int:
+    return lib().monarch_bwd_path(ctypes.byref(make_dims(shape, 1, dtype)))
+
+
+def bwd_workspace_bytes(shape: dict, rows: int, dtype="bf16") -> int:
+    return int(lib().monarch_bwd_workspace_bytes(ctypes.byref(make_dims(shape, rows, dtype))))
+
+
+def fwd(X, R, L, shape: dict, Y=None, stream=None):
+    """Y = X M^T on the GPU.  X: (rows, nb1*in1); returns Y (rows, nb2*out2)."""
+    import torch
+    code = dtype_code(X.dtype)
+    n_out = shape["nb2"] * shape["out2"]
+    rows = X.shape[0]
+    if Y is None:
+        Y = torch.empty((rows, n_out), dtype=X.dtype, device=X.device)
+    _require_cuda(X, R, L, Y)
+    d = make_dims(shape, rows, code)
+    _check("monarch_fwd", lib().monarch_fwd(_ptr(X), _ptr(R), _ptr(L), ctypes.byref(d), _ptr(Y),
+                                            _stream(stream)))
+    return Y
+
+
+def bwd(dY, X, R, L, shape: dict, dX=None, dR=None, dL=None, workspace=None, stream=None):
+    """(dX, dR, dL) of Y = X M^T for upstream gradient dY, on the GPU."""
+    import torch
+    code = dtype_code(X.dtype)
+    rows = X.shape[0]
+    if dX is None:
+        dX = torch.empty_like(X)
+    if dR is None:
+        dR = torch.empty_like(R)
+    if dL is None:
+        dL = torch.empty_like(L)
+    d = make_dims(shape, rows, code)
+    need = int(lib().monarch_bwd_workspace_bytes(ctypes.byref(d)))
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=X.device)
+    _require_cuda(dY, X, R, L, dX, dR, dL, workspace)
+    _check("monarch_bwd", lib().monarch_bwd(
+        _ptr(dY), _ptr(X), _ptr(R), _ptr(L), ctypes.byref(d), _ptr(dX), _ptr(dR), _ptr(dL),
+        _ptr(workspace), ctypes.c_size_t(workspace.numel() * workspace.element_size()),
+        _stream(stream)))
+    return dX, dR, dL
+
+
+def materialise(R, L, shape: dict, M=None, stream=None):
+    """Dense M (n_out, n_in) as float32 with Y = X M^T."""
+    import torch
+    code = dtype_code(R.dtype)
+    n_in = shape["nb1"] * shape["in1"]
+    n_out = shape["nb2"] * shape["out2"]
+    if M is None:
+        M = torch.empty((n_out, n_in), dtype=torch.float32, device=R.device)
+    _require_cuda(R, L, M)
+    d = make_dims(shape, 0, code)
+    _check("monarch_materialise", lib().monarch_materialise(_ptr(R), _ptr(L), ctypes.byref(d),
+                                                            _ptr(M), _stream(stream)))
+    return M
+
+
+def last_device_status(stream=None) -> int:
+    """Synchronise the stream and return/clear the device status word."""
+    return lib().monarch_last_device_status(_stream(stream))
+
+
+def debug_wait_timeout(timeout_ns: int, stream=None) -> int:
+    return lib().monarch_debug_wait_timeout(ctypes.c_uint64(int(timeout_ns)), _stream(stream))
+
+
+def status_string(code: int) -> str:
+    return lib().monarch_status_string(int(code)).decode()

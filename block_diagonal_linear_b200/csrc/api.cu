@@ -1,0 +1,168 @@
+// C ABI of libmonarch.so: argument checks, dispatch to the kernel families,
+// the device status word and the bounded-wait test hook.
+#include <stdint.h>
+
+#include <initializer_list>
+
+#include "common.cuh"
+#include "ptx.cuh"
+
+namespace monarch {
+
+// Device status word: kernels that give up a bounded wait store kStatusTimeout.
+__device__ int g_status;
+
+static int* status_ptr() {
+  int* p = nullptr;
+  if (cudaGetSymbolAddress((void**)&p, g_status) != cudaSuccess) return nullptr;
+  return p;
+}
+
+static bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+static int check_dims(const monarch_dims* d) {
+  if (d == nullptr) return MONARCH_ERR_NULL;
+  if (d->dtype != MONARCH_F32 && d->dtype != MONARCH_BF16) return MONARCH_ERR_DTYPE;
+  if (d->rows < 0 || d->nb1 <= 0 || d->in1 <= 0 || d->out1 <= 0 || d->nb2 <= 0 || d->in2 <= 0 ||
+      d->out2 <= 0)
+    return MONARCH_ERR_DIMS;
+  if ((int64_t)d->nb1 * d->out1 != (int64_t)d->nb2 * d->in2) return MONARCH_ERR_DIMS;
+  // every flattened size must stay well inside int64 and int32 grid limits
+  const int64_t lim = int64_t(1) << 40;
+  if ((int64_t)d->nb1 * d->in1 > lim || (int64_t)d->nb1 * d->out1 > lim ||
+      (int64_t)d->nb2 * d->out2 > lim)
+    return MONARCH_ERR_DIMS;
+  return MONARCH_OK;
+}
+
+static int check_ptrs(std::initializer_list<const void*> ps) {
+  for (const void* p : ps) {
+    if (p == nullptr) return MONARCH_ERR_NULL;
+    if (!aligned16(p)) return MONARCH_ERR_ALIGN;
+  }
+  return MONARCH_OK;
+}
+
+__global__ void debug_wait_kernel(uint64_t timeout_ns, int* status) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    ptx::mbar_init(&bar, 1);
+    ptx::fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    // nothing ever arrives on `bar`: the bounded wait must give up
+    if (!ptx::mbar_wait_bounded(&bar, 0, timeout_ns)) atomicExch(status, kStatusTimeout);
+  }
+  __syncthreads();
+}
+
+cudaError_t debug_wait_timeout(uint64_t timeout_ns, int* status, cudaStream_t st) {
+  debug_wait_kernel<<<1, 32, 0, st>>>(timeout_ns, status);
+  return cudaGetLastError();
+}
+
+static int fwd_path(const Shape& s, int dtype) {
+  return (dtype == MONARCH_BF16 && tc_fwd_supported(s)) ? 1 : 0;
+}
+
+}  // namespace monarch
+
+using namespace monarch;
+
+extern "C" {
+
+int monarch_validate(const monarch_dims* d) { return check_dims(d); }
+
+int monarch_fwd_path(const monarch_dims* d) {
+  if (check_dims(d) != MONARCH_OK) return -1;
+  return fwd_path(to_shape(*d), d->dtype);
+}
+
+int monarch_bwd_path(const monarch_dims* d) {
+  if (check_dims(d) != MONARCH_OK) return -1;
+  return 0;
+}
+
+int monarch_fwd(const void* X, const void* R, const void* L, const monarch_dims* d, void* Y,
+                void* stream) {
+  int rc = check_dims(d);
+  if (rc != MONARCH_OK) return rc;
+  if (d->rows == 0) return MONARCH_OK;
+  if ((rc = check_ptrs({X, R, L, Y})) != MONARCH_OK) return rc;
+  const Shape s = to_shape(*d);
+  cudaStream_t st = (cudaStream_t)stream;
+  cudaError_t e;
+  if (fwd_path(s, d->dtype) == 1) {
+    int* status = status_ptr();
+    if (status == nullptr) return MONARCH_ERR_CUDA;
+    e = tc_fwd(X, R, L, Y, s, status, st);
+  } else {
+    if (!generic_fwd_supported(s)) return MONARCH_ERR_UNSUPPORTED;
+    e = generic_fwd(X, R, L, Y, s, d->dtype, st);
+  }
+  return e == cudaSuccess ? MONARCH_OK : MONARCH_ERR_CUDA;
+}
+
+size_t monarch_bwd_workspace_bytes(const monarch_dims* d) {
+  if (check_dims(d) != MONARCH_OK) return 0;
+  return generic_bwd_workspace(to_shape(*d));
+}
+
+int monarch_bwd(const void* dY, const void* X, const void* R, const void* L, const monarch_dims* d,
+                void* dX, void* dR, void* dL, void* workspace, size_t workspace_bytes,
+                void* stream) {
+  int rc = check_dims(d);
+  if (rc != MONARCH_OK) return rc;
+  if ((rc = check_ptrs({R, L, dR, dL})) != MONARCH_OK) return rc;
+  if (d->rows > 0 && (rc = check_ptrs({dY, X, dX})) != MONARCH_OK) return rc;
+  const Shape s = to_shape(*d);
+  const size_t need = generic_bwd_workspace(s);
+  if (workspace == nullptr || workspace_bytes < need) return MONARCH_ERR_WORKSPACE;
+  if (((uintptr_t)workspace & 255u) != 0) return MONARCH_ERR_ALIGN;
+  if (!generic_bwd_supported(s)) return MONARCH_ERR_UNSUPPORTED;
+  cudaError_t e = generic_bwd(dY, X, R, L, dX, dR, dL, workspace, s, d->dtype, (cudaStream_t)stream);
+  return e == cudaSuccess ? MONARCH_OK : MONARCH_ERR_CUDA;
+}
+
+int monarch_materialise(const void* R, const void* L, const monarch_dims* d, void* M,
+                        void* stream) {
+  int rc = check_dims(d);
+  if (rc != MONARCH_OK) return rc;
+  if ((rc = check_ptrs({R, L, M})) != MONARCH_OK) return rc;
+  cudaError_t e = generic_materialise(R, L, (float*)M, to_shape(*d), d->dtype, (cudaStream_t)stream);
+  return e == cudaSuccess ? MONARCH_OK : MONARCH_ERR_CUDA;
+}
+
+const char* monarch_status_string(int status) {
+  switch (status) {
+    case MONARCH_OK: return "ok";
+    case MONARCH_ERR_DIMS: return "invalid Monarch dims";
+    case MONARCH_ERR_DTYPE: return "unsupported dtype";
+    case MONARCH_ERR_ALIGN: return "pointer not 16-byte aligned";
+    case MONARCH_ERR_NULL: return "null pointer";
+    case MONARCH_ERR_WORKSPACE: return "workspace missing or too small";
+    case MONARCH_ERR_CUDA: return "CUDA error";
+    case MONARCH_ERR_TIMEOUT: return "bounded device wait timed out";
+    case MONARCH_ERR_UNSUPPORTED: return "shape not supported by any kernel";
+    default: return "unknown status";
+  }
+}
+
+int monarch_last_device_status(void* stream) {
+  if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return MONARCH_ERR_CUDA;
+  int v = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&v, g_status, sizeof(int)) != cudaSuccess) return MONARCH_ERR_CUDA;
+  if (cudaMemcpyToSymbol(g_status, &zero, sizeof(int)) != cudaSuccess) return MONARCH_ERR_CUDA;
+  return v == kStatusTimeout ? MONARCH_ERR_TIMEOUT : MONARCH_OK;
+}
+
+int monarch_debug_wait_timeout(uint64_t timeout_ns, void* stream) {
+  int* status = status_ptr();
+  if (status == nullptr) return MONARCH_ERR_CUDA;
+  return debug_wait_timeout(timeout_ns, status, (cudaStream_t)stream) == cudaSuccess
+             ? MONARCH_OK
+             : MONARCH_ERR_CUDA;
+}
+
+}  // extern "C"

@@ -1,0 +1,69 @@
+// Shared definitions of the Monarch CUDA kernels (sm_100a).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/monarch.h"
+
+namespace monarch {
+
+// Shape passed by value to kernels.  Notation as in monarch.h.
+struct Shape {
+  int64_t rows;
+  int nb1, in1, out1;
+  int nb2, in2, out2;
+  int out_transpose;
+  __host__ __device__ int64_t n_in() const { return (int64_t)nb1 * in1; }
+  __host__ __device__ int64_t n_mid() const { return (int64_t)nb1 * out1; }
+  __host__ __device__ int64_t n_out() const { return (int64_t)nb2 * out2; }
+  __host__ __device__ int64_t n_R() const { return (int64_t)nb1 * out1 * in1; }
+  __host__ __device__ int64_t n_L() const { return (int64_t)nb2 * out2 * in2; }
+  // Column of v[j][o] in a row of Y (the output permutation).
+  __host__ __device__ int64_t out_index(int j, int o) const {
+    return out_transpose ? (int64_t)o * nb2 + j : (int64_t)j * out2 + o;
+  }
+};
+
+inline Shape to_shape(const monarch_dims& d) {
+  Shape s;
+  s.rows = d.rows;
+  s.nb1 = d.nb1; s.in1 = d.in1; s.out1 = d.out1;
+  s.nb2 = d.nb2; s.in2 = d.in2; s.out2 = d.out2;
+  s.out_transpose = d.out_transpose ? 1 : 0;
+  return s;
+}
+
+// Element load / store in fp32 for both storage types.
+__device__ __forceinline__ float ld_as_f32(const float* p) { return __ldg(p); }
+__device__ __forceinline__ float ld_as_f32(const __nv_bfloat16* p) {
+  return __bfloat162float(__ldg(p));
+}
+__device__ __forceinline__ void st_from_f32(float* p, float v) { *p = v; }
+__device__ __forceinline__ void st_from_f32(__nv_bfloat16* p, float v) {
+  *p = __float2bfloat16_rn(v);
+}
+
+// Device status word values (written by kernels, read by the host).
+constexpr int kStatusTimeout = 1;
+
+// ---- launchers implemented in the .cu files (all return cudaError_t) ----
+cudaError_t generic_fwd(const void* X, const void* R, const void* L, void* Y, const Shape& s,
+                        int dtype, cudaStream_t st);
+size_t generic_bwd_workspace(const Shape& s);
+cudaError_t generic_bwd(const void* dY, const void* X, const void* R, const void* L, void* dX,
+                        void* dR, void* dL, void* ws, const Shape& s, int dtype, cudaStream_t st);
+cudaError_t generic_materialise(const void* R, const void* L, float* M, const Shape& s, int dtype,
+                                cudaStream_t st);
+bool generic_fwd_supported(const Shape& s);
+bool generic_bwd_supported(const Shape& s);
+
+// tcgen05 fused forward for bf16 (returns cudaErrorNotSupported if the shape has no kernel).
+bool tc_fwd_supported(const Shape& s);
+cudaError_t tc_fwd(const void* X, const void* R, const void* L, void* Y, const Shape& s,
+                   int* status, cudaStream_t st);
+
+cudaError_t debug_wait_timeout(uint64_t timeout_ns, int* status, cudaStream_t st);
+
+}  // namespace monarch

@@ -1,0 +1,147 @@
+/*
+ * monarch.h -- C ABI of libmonarch.so, the B200 (sm_100a) Monarch linear map.
+ *
+ * The operation (Monarch: Expressive Structured Matrices for Efficient and
+ * Accurate Training, abstract; scatterbrain issue thread, "Definition C.3"):
+ * a Monarch matrix is a product of two block-diagonal matrices with a fixed
+ * reshape-transpose permutation between them,
+ *
+ *     Y = X * M^T,     M = P_out * L * P * R,
+ *
+ * applied to every row x of X (rows are independent):
+ *   u[k][p]      = sum_i R[k][p][i] * x[k*in1 + i]        (R: nb1 blocks of out1 x in1)
+ *   flat[p*nb1+k]= u[k][p]                                 (P: view (nb1,out1), transpose)
+ *   Z[j][q]      = flat[j*in2 + q]                         (regroup into nb2 blocks of in2)
+ *   v[j][o]      = sum_q L[j][o][q] * Z[j][q]              (L: nb2 blocks of out2 x in2)
+ *   y[o*nb2 + j] = v[j][o]   if out_transpose             (P_out: transpose and flatten)
+ *   y[j*out2 + o]= v[j][o]   otherwise                     (plain flatten)
+ * The permutation direction follows the worked N=4 example of the scatterbrain
+ * thread (x_new = [x0, x2, x1, x3]) and its lattice view: R contracts the rows
+ * of the (nb1 x in1) grid, L the columns.  Factor tensors use the nn.Linear
+ * weight convention of MonarchLinear's blkdiag1 / blkdiag2: (nblocks, out_blk,
+ * in_blk), row-major.
+ *
+ * Conventions for every entry point:
+ *   - Tensor pointers are DEVICE pointers owned by the caller, contiguous,
+ *     row-major, 16-byte aligned.  X is (rows, nb1*in1), Y and dY are
+ *     (rows, nb2*out2), R and dR are (nb1, out1, in1), L and dL are
+ *     (nb2, out2, in2).  All of X, R, L, Y, dY, dX, dR, dL have the element
+ *     type d->dtype (fp32 or bf16).  Accumulation is always fp32; bf16 results
+ *     are rounded to nearest-even.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Calls are
+ *     asynchronous on it; the library never synchronises the device except in
+ *     monarch_last_device_status().
+ *   - The library allocates no device memory.  monarch_bwd takes a caller-owned
+ *     workspace of at least monarch_bwd_workspace_bytes(d) bytes.
+ *   - Return value: MONARCH_OK (0) or a negative MONARCH_ERR_* code.  Nothing
+ *     aborts, throws or prints.  A failed call leaves its outputs unspecified.
+ *   - Kernel-side bounded waits that give up record MONARCH_ERR_TIMEOUT in a
+ *     device status word; read it with monarch_last_device_status().
+ */
+#ifndef MONARCH_H_
+#define MONARCH_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MONARCH_API __attribute__((visibility("default")))
+#else
+#define MONARCH_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MONARCH_F32 = 0,
+  MONARCH_BF16 = 1
+} monarch_dtype;
+
+enum {
+  MONARCH_OK = 0,
+  MONARCH_ERR_DIMS = -1,        /* non-positive sizes, rows < 0, or nb1*out1 != nb2*in2 */
+  MONARCH_ERR_DTYPE = -2,       /* dtype not in monarch_dtype */
+  MONARCH_ERR_ALIGN = -3,       /* a pointer is not 16-byte aligned */
+  MONARCH_ERR_NULL = -4,        /* a required pointer is NULL (rows > 0) */
+  MONARCH_ERR_WORKSPACE = -5,   /* workspace NULL or smaller than required */
+  MONARCH_ERR_CUDA = -6,        /* a CUDA runtime call or kernel launch failed */
+  MONARCH_ERR_TIMEOUT = -7,     /* a bounded device wait gave up (device status) */
+  MONARCH_ERR_UNSUPPORTED = -8  /* shape too large for any kernel of this build */
+};
+
+/* Shape of one Monarch map.  Scatterbrain thread, MonarchLinear __init__ and
+ * Definition C.3: R has nb1 blocks of (out1 x in1), L has nb2 blocks of
+ * (out2 x in2), and the middle width must agree: nb1*out1 == nb2*in2. */
+typedef struct {
+  int64_t rows;          /* rows of X (batch x tokens); 0 is a valid no-op      */
+  int32_t nb1, in1, out1;
+  int32_t nb2, in2, out2;
+  int32_t out_transpose; /* 1: y[o*nb2 + j] = v[j][o];  0: y[j*out2 + o]         */
+  int32_t dtype;         /* monarch_dtype of every tensor argument               */
+} monarch_dims;
+
+/* Host-only check of a shape: MONARCH_OK or MONARCH_ERR_DIMS / _DTYPE.  Needs
+ * no GPU. */
+MONARCH_API int monarch_validate(const monarch_dims* d);
+
+/* Forward, steps R -> P -> L -> P_out for every row:  Y = X * M^T.
+ * In:  X (rows, nb1*in1), R (nb1,out1,in1), L (nb2,out2,in2).
+ * Out: Y (rows, nb2*out2), overwritten.
+ * bf16 path: bf16 inputs, fp32 accumulation on the tensor cores, the middle
+ * vector rounded to bf16 on chip, Y rounded to bf16.  fp32 path: fp32 FMA. */
+MONARCH_API int monarch_fwd(const void* X, const void* R, const void* L, const monarch_dims* d, void* Y,
+                void* stream);
+
+/* Backward of Y = X * M^T for a loss with gradient dY (chain rule; the middle
+ * vector is recomputed from X rather than stored):
+ *   dV[j][o] = dY[idx(j,o)],  dL[j][o][q] = sum_rows dV[j][o] * Z[j][q],
+ *   dZ[j][q] = sum_o L[j][o][q] dV[j][o],  dU[k][p] = dZflat[p*nb1 + k],
+ *   dR[k][p][i] = sum_rows dU[k][p] * x[k*in1+i],  dX[k*in1+i] = sum_p R[k][p][i] dU[k][p].
+ * In:  dY (rows, n_out), X, R, L.   Out: dX (rows, n_in), dR, dL -- all
+ * overwritten (not accumulated).  Weight gradients are reduced over rows in a
+ * fixed order, so repeated calls give bitwise-identical results.
+ * workspace: device scratch of >= monarch_bwd_workspace_bytes(d) bytes, 256-byte
+ * aligned, owned by the caller, not read before it is written. */
+MONARCH_API int monarch_bwd(const void* dY, const void* X, const void* R, const void* L, const monarch_dims* d,
+                void* dX, void* dR, void* dL, void* workspace, size_t workspace_bytes,
+                void* stream);
+
+/* Workspace bytes monarch_bwd needs for this shape (0 if d is invalid). */
+MONARCH_API size_t monarch_bwd_workspace_bytes(const monarch_dims* d);
+
+/* Dense equivalent for checking (scatterbrain thread: applying the multiply to
+ * the identity "is essentially the full matrix"): writes M (n_out, n_in) as
+ * FLOAT32 regardless of d->dtype, with Y = X * M^T.  d->rows is ignored.
+ * Entry: M[idx(j,o)][k*in1+i] = sum over p with (p*nb1+k) div in2 == j of
+ *        L[j][o][(p*nb1+k) mod in2] * R[k][p][i]. */
+MONARCH_API int monarch_materialise(const void* R, const void* L, const monarch_dims* d, void* M,
+                        void* stream);
+
+/* Human-readable name of a status code (static string). */
+MONARCH_API const char* monarch_status_string(int status);
+
+/* Synchronises `stream`, then returns and clears the device status word of the
+ * current device: MONARCH_OK, MONARCH_ERR_TIMEOUT (a bounded wait inside a
+ * kernel gave up and that kernel skipped its remaining work), or
+ * MONARCH_ERR_CUDA if the synchronisation itself failed. */
+MONARCH_API int monarch_last_device_status(void* stream);
+
+/* Test hook for the bounded-wait machinery: launches one block that waits on
+ * an mbarrier nothing will ever arrive on, giving up after timeout_ns
+ * nanoseconds and recording MONARCH_ERR_TIMEOUT in the device status word.
+ * Returns the launch status; read the outcome with
+ * monarch_last_device_status(). */
+MONARCH_API int monarch_debug_wait_timeout(uint64_t timeout_ns, void* stream);
+
+/* Which kernel family monarch_fwd / monarch_bwd would run for this shape:
+ * 0 = generic FMA kernels, 1 = tcgen05 fused kernels.  Host-only. */
+MONARCH_API int monarch_fwd_path(const monarch_dims* d);
+MONARCH_API int monarch_bwd_path(const monarch_dims* d);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MONARCH_H_ */

@@ -1,0 +1,92 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports
+every symbol include/monarch.h declares, and rejects bad arguments before it
+touches the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import block_diagonal_linear_b200 as bdl
+from block_diagonal_linear_b200 import synthetic
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_symbols():
+    text = open(os.path.join(ROOT, "include", "monarch.h")).read()
+    return sorted(set(re.findall(r"MONARCH_API\s+[\w\s\*]+?\b(monarch_\w+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_symbol():
+    names = declared_symbols()
+    assert len(names) >= 8
+    lib = bdl.lib()
+    for n in names:
+        assert hasattr(lib, n), n
+    assert sorted(bdl.EXPORTED) == names
+
+
+def test_status_strings():
+    for code in bdl.STATUS:
+        assert bdl.status_string(code)
+    assert bdl.status_string(-7) == "bounded device wait timed out"
+
+
+@pytest.mark.parametrize("name", sorted(synthetic.WORKLOADS))
+def test_workloads_validate(name):
+    w = synthetic.WORKLOADS[name]
+    assert bdl.validate(synthetic.shape_of(w), w["rows"], w["dtype"]) == 0
+
+
+def test_bad_dims_rejected():
+    good = dict(nb1=4, in1=8, out1=8, nb2=4, in2=8, out2=8, out_transpose=1)
+    assert bdl.validate(good, 3, "f32") == 0
+    assert bdl.validate(dict(good, out1=6), 3, "f32") == bdl.CODES["MONARCH_ERR_DIMS"]
+    assert bdl.validate(dict(good, nb2=0), 3, "f32") == bdl.CODES["MONARCH_ERR_DIMS"]
+    assert bdl.validate(good, -1, "f32") == bdl.CODES["MONARCH_ERR_DIMS"]
+    assert bdl.validate(good, 3, 7) == bdl.CODES["MONARCH_ERR_DTYPE"]
+    # rows == 0 is a valid no-op shape
+    assert bdl.validate(good, 0, "bf16") == 0
+
+
+def test_fwd_argument_errors_before_device_work():
+    lib = bdl.lib()
+    shape = dict(nb1=4, in1=8, out1=8, nb2=4, in2=8, out2=8, out_transpose=1)
+    d = bdl.make_dims(shape, 5, "f32")
+    p = ctypes.c_void_p(4096)
+    assert lib.monarch_fwd(None, p, p, ctypes.byref(d), p, None) == bdl.CODES["MONARCH_ERR_NULL"]
+    assert lib.monarch_fwd(ctypes.c_void_p(4100), p, p, ctypes.byref(d), p, None) == \
+        bdl.CODES["MONARCH_ERR_ALIGN"]
+    bad = bdl.make_dims(dict(shape, in2=5), 5, "f32")
+    assert lib.monarch_fwd(p, p, p, ctypes.byref(bad), p, None) == bdl.CODES["MONARCH_ERR_DIMS"]
+    # rows == 0: nothing to do, even with null tensors
+    z = bdl.make_dims(shape, 0, "f32")
+    assert lib.monarch_fwd(None, p, p, ctypes.byref(z), None, None) == 0
+    assert lib.monarch_fwd(p, p, p, None, p, None) == bdl.CODES["MONARCH_ERR_NULL"]
+
+
+def test_bwd_workspace_checks_before_device_work():
+    lib = bdl.lib()
+    shape = synthetic.shape_of(synthetic.WORKLOADS["n1024_bf16"])
+    d = bdl.make_dims(shape, 1000, "bf16")
+    need = bdl.bwd_workspace_bytes(shape, 1000, "bf16")
+    assert need > 0
+    p = ctypes.c_void_p(4096)
+    rc = lib.monarch_bwd(p, p, p, p, ctypes.byref(d), p, p, p, p, ctypes.c_size_t(need - 1), None)
+    assert rc == bdl.CODES["MONARCH_ERR_WORKSPACE"]
+    rc = lib.monarch_bwd(p, p, p, p, ctypes.byref(d), p, p, p, None, ctypes.c_size_t(need), None)
+    assert rc == bdl.CODES["MONARCH_ERR_WORKSPACE"]
+    rc = lib.monarch_bwd(p, p, p, p, ctypes.byref(d), p, p, p, ctypes.c_void_p(4096 + 16),
+                         ctypes.c_size_t(need), None)
+    assert rc == bdl.CODES["MONARCH_ERR_ALIGN"]
+    assert bdl.bwd_workspace_bytes(dict(shape, out1=5), 10, "bf16") == 0
+
+
+def test_kernel_family_selection():
+    W = synthetic.WORKLOADS
+    for name in ("n1024_bf16", "r768x3072_bf16", "nblk4_1024x4096_bf16"):
+        assert bdl.fwd_path(synthetic.shape_of(W[name]), "bf16") == 1, name
+    assert bdl.fwd_path(synthetic.shape_of(W["n256_fp32"]), "f32") == 0
+    assert bdl.fwd_path(synthetic.shape_of(W["n256_fp32"]), "bf16") == 1
+    assert bdl.fwd_path(dict(nb1=3, in1=5, out1=4, nb2=2, in2=6, out2=7, out_transpose=1), "bf16") == 0
