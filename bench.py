@@ -220,6 +220,9 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synthetic.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end timing")
+    ap.add_argument("--pass", dest="only", default="step", choices=["step", "fwd", "bwd"],
+                    help="time the whole step (default) or one pass only")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     name = args.workload
@@ -270,17 +273,22 @@ def main():
             dist.all_reduce(dR)
             dist.all_reduce(dL)
 
+    do_fwd = args.only in ("step", "fwd")
+    do_bwd = args.only in ("step", "bwd")
+
     def step(ev=None):
         if ev is not None:
             flush.zero_()
             ev[0].record(stream)
-        bdl.fwd(X, R, L, shape, Y=Y)
+        if do_fwd:
+            bdl.fwd(X, R, L, shape, Y=Y)
         if ev is not None:
             ev[1].record(stream)
             flush.zero_()
             ev[2].record(stream)
-        bdl.bwd(dY, X, R, L, shape, dX=dX, dR=dR, dL=dL, workspace=ws)
-        allreduce_grads()
+        if do_bwd:
+            bdl.bwd(dY, X, R, L, shape, dX=dX, dR=dR, dL=dL, workspace=ws)
+            allreduce_grads()
         if ev is not None:
             ev[3].record(stream)
 
@@ -319,7 +327,7 @@ def main():
     dYh.copy_(dY)
     outs_h = [torch.empty_like(t, device="cpu").pin_memory() for t in (Y, dX, dR, dL)]
     Xe, dYe = torch.empty_like(X), torch.empty_like(dY)
-    n_e2e = max(3, min(args.steps, 50))
+    n_e2e = 0 if args.no_e2e or args.only != "step" else max(3, min(args.steps, 50))
 
     def e2e_step():
         Xe.copy_(Xh, non_blocking=True)
@@ -330,7 +338,7 @@ def main():
         for h, d_ in zip(outs_h, (Y, dX, dR, dL)):
             h.copy_(d_, non_blocking=True)
 
-    for _ in range(2):
+    for _ in range(2 if n_e2e else 0):
         e2e_step()
     torch.cuda.synchronize()
     if world > 1:
@@ -341,7 +349,7 @@ def main():
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1)
+    e2e_ms = e0.elapsed_time(e1) if n_e2e else 0.0
     if world > 1:
         t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev_)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
@@ -364,6 +372,8 @@ def main():
     tpk = peaks["bf16_tflops"] * 1e12
     passes = {}
     for pname, t_s in (("fwd", fwd_avg_s), ("bwd", bwd_avg_s)):
+        if (pname == "fwd" and not do_fwd) or (pname == "bwd" and not do_bwd):
+            continue
         a = alg[pname]
         t_roof = max(a["bytes"] / hbm, a["flops"] / tpk)
         passes[pname] = {
@@ -373,7 +383,7 @@ def main():
             "bound": "hbm" if a["bytes"] / hbm >= a["flops"] / tpk else "tensor",
         }
     fwd_tc = bdl.fwd_path(shape, w["dtype"]) == 1
-    launches_per_step = 1 + 3
+    launches_per_step = (1 if do_fwd else 0) + (3 if do_bwd else 0)
     dom = "fwd" if fwd_avg_s >= bwd_avg_s else "bwd"
     a = alg[dom]
     t_dom = fwd_avg_s if dom == "fwd" else bwd_avg_s
@@ -402,12 +412,13 @@ def main():
                            (" + NCCL all-reduce of dR, dL" if world > 1 else ""),
                    "l2": "flushed before every timed pass (%d MiB write, untimed)"
                          % (flush.numel() >> 20),
-                   "parallelism": "dp%d" % world},
+                   "parallelism": "dp%d" % world, "timed": args.only},
         "tflops": (alg["fwd"]["flops"] + alg["bwd"]["flops"]) * world * K / (tot_ms / 1e3) / 1e12,
         "passes": passes,
         "roofline": roof,
-        "e2e": {"value": world * rows * n_e2e / (e2e_ms / 1e3), "unit": "rows/s",
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": n_e2e},
+        "e2e": ({"value": world * rows * n_e2e / (e2e_ms / 1e3), "unit": "rows/s",
+                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": n_e2e}
+                if n_e2e else None),
         "gpu_launches": launches_per_step * K,
         "clocks": sampler.summary(),
         "device_status": status,

@@ -177,7 +177,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       ptx::tma_prefetch_desc(&tmX);
       ptx::tma_prefetch_desc(&tmR);
       ptx::tma_prefetch_desc(&tmL);
-      const uint64_t pol_stream = ptx::policy_evict_first();
+      const uint64_t pol_stream = ptx::policy_evict_normal();  // X is read by NGROUPS CTAs
       const uint64_t pol_keep = ptx::policy_evict_last();
       uint32_t it = 0;  // global stage counter
       bool ok = true;
