@@ -62,8 +62,12 @@ cudaError_t debug_wait_timeout(uint64_t timeout_ns, int* status, cudaStream_t st
   return cudaGetLastError();
 }
 
+// 0 = generic FMA kernels, 1 = tcgen05 group kernel, 2 = tcgen05 row-tile kernel.
 static int fwd_path(const Shape& s, int dtype) {
-  return (dtype == MONARCH_BF16 && tc_fwd_supported(s)) ? 1 : 0;
+  if (dtype != MONARCH_BF16) return 0;
+  if (tc_rows_supported(s)) return 2;
+  if (tc_fwd_supported(s)) return 1;
+  return 0;
 }
 
 }  // namespace monarch
@@ -93,10 +97,11 @@ int monarch_fwd(const void* X, const void* R, const void* L, const monarch_dims*
   const Shape s = to_shape(*d);
   cudaStream_t st = (cudaStream_t)stream;
   cudaError_t e;
-  if (fwd_path(s, d->dtype) == 1) {
+  const int path = fwd_path(s, d->dtype);
+  if (path != 0) {
     int* status = status_ptr();
     if (status == nullptr) return MONARCH_ERR_CUDA;
-    e = tc_fwd(X, R, L, Y, s, status, st);
+    e = path == 2 ? tc_rows_fwd(X, R, L, Y, s, status, st) : tc_fwd(X, R, L, Y, s, status, st);
   } else {
     if (!generic_fwd_supported(s)) return MONARCH_ERR_UNSUPPORTED;
     e = generic_fwd(X, R, L, Y, s, d->dtype, st);

@@ -64,6 +64,11 @@ bool tc_fwd_supported(const Shape& s);
 cudaError_t tc_fwd(const void* X, const void* R, const void* L, void* Y, const Shape& s,
                    int* status, cudaStream_t st);
 
+// tcgen05 fused forward with 64-row tiles and the whole middle vector on chip (small blocks).
+bool tc_rows_supported(const Shape& s);
+cudaError_t tc_rows_fwd(const void* X, const void* R, const void* L, void* Y, const Shape& s,
+                        int* status, cudaStream_t st);
+
 cudaError_t debug_wait_timeout(uint64_t timeout_ns, int* status, cudaStream_t st);
 
 }  // namespace monarch

@@ -22,18 +22,19 @@
 // Every mbarrier wait is bounded; on timeout the CTA records
 // kStatusTimeout, skips the rest of its work, waits for its own copies and
 // MMAs, frees TMEM and returns.
-#include <cuda.h>
-
-#include <initializer_list>
-
-#include "common.cuh"
-#include "ptx.cuh"
+#include "tc_common.cuh"
 
 namespace monarch {
 
-constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s per wait
 constexpr int kTcThreads = 192;
-constexpr int kSmemBudget = 227 * 1024 - 1024;   // dynamic smem incl. 1 KB alignment slack
+
+struct Bars {
+  uint64_t full[8], empty[8];
+  uint64_t acc_full[2], acc_empty[2];
+  uint64_t z_full, z_empty, mma_done;
+  uint32_t tmem_base;
+  int abort_flag;
+};
 
 template <int NB1_, int IN1_, int OUT1_, int NB2_, int IN2_, int OUT2_, int OT_, int G_>
 struct FwdCfg {
@@ -89,47 +90,6 @@ struct FwdCfg {
   static_assert(NSTAGE >= 2, "shared memory");
   static_assert(LPS >= 1, "L slice larger than a stage");
 };
-
-// ---------------------------------------------------------------- descriptors
-// tcgen05 shared-memory matrix descriptor, K-major, given swizzle code
-// (2 = 128B, 6 = 32B) and stride between 8-row groups (bytes).
-__device__ __forceinline__ uint64_t make_sdesc(uint32_t saddr, uint32_t sbo_bytes, uint32_t swz) {
-  uint64_t d = 0;
-  d |= (uint64_t)((saddr >> 4) & 0x3FFF);
-  d |= (uint64_t)1 << 16;                              // leading byte offset (unused, K-major swizzled)
-  d |= (uint64_t)((sbo_bytes >> 4) & 0x3FFF) << 32;    // stride byte offset
-  d |= (uint64_t)1 << 46;                              // descriptor version (sm_100)
-  d |= (uint64_t)swz << 61;                            // layout / swizzle type
-  return d;
-}
-
-// Instruction descriptor: kind::f16, A = B = bf16, D = fp32, both K-major.
-__host__ __device__ constexpr uint32_t make_idesc(int M, int N) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) |
-         ((uint32_t)(M >> 4) << 24);
-}
-
-struct Bars {
-  uint64_t full[8], empty[8];
-  uint64_t acc_full[2], acc_empty[2];
-  uint64_t z_full, z_empty, mma_done;
-  uint32_t tmem_base;
-  int abort_flag;
-};
-
-__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, Bars* b, int* status) {
-  if (ptx::mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = ptx::globaltimer_ns();
-  while (true) {
-    if (ptx::mbar_try_wait(bar, parity)) return true;
-    if (*(volatile int*)&b->abort_flag) return false;
-    if (ptx::globaltimer_ns() - t0 > kWaitLimitNs) {
-      *(volatile int*)&b->abort_flag = 1;
-      atomicExch(status, kStatusTimeout);
-      return false;
-    }
-  }
-}
 
 template <class C>
 __global__ void __launch_bounds__(kTcThreads, 1)
@@ -187,7 +147,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         for (int b = 0; b < C::NXB && ok; ++b, ++it) {
           const int st = it % C::NSTAGE;
           const uint32_t ph = (it / C::NSTAGE) & 1;
-          if (!wait_or_abort(&bars->empty[st], ph ^ 1, bars, status)) { ok = false; break; }
+          if (!wait_or_abort(&bars->empty[st], ph ^ 1, &bars->abort_flag, status)) { ok = false; break; }
           uint8_t* sbase = ring + st * C::STAGE_BYTES;
           int nk = 0;
           for (int t = 0; t < 4; ++t) nk += (b * 64 + t * 16 < C::N_IN) ? 1 : 0;
@@ -204,7 +164,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         for (int sp = 0; sp < C::NSTAGE2 && ok; ++sp, ++it) {
           const int st = it % C::NSTAGE;
           const uint32_t ph = (it / C::NSTAGE) & 1;
-          if (!wait_or_abort(&bars->empty[st], ph ^ 1, bars, status)) { ok = false; break; }
+          if (!wait_or_abort(&bars->empty[st], ph ^ 1, &bars->abort_flag, status)) { ok = false; break; }
           uint8_t* sbase = ring + st * C::STAGE_BYTES;
           const int p0 = sp * C::LPS;
           const int np = (C::NPIECE2 - p0) < C::LPS ? (C::NPIECE2 - p0) : C::LPS;
@@ -246,7 +206,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         int cur_box = -1;
         for (int r1 = 0; r1 < C::NR1 && ok; ++r1, ++rnd) {
           const int slot = rnd & 1;
-          if (!wait_or_abort(&bars->acc_empty[slot], ((rnd >> 1) & 1) ^ 1, bars, status)) { ok = false; break; }
+          if (!wait_or_abort(&bars->acc_empty[slot], ((rnd >> 1) & 1) ^ 1, &bars->abort_flag, status)) { ok = false; break; }
           ptx::tc_fence_after();
           for (int kk = 0; kk < C::KR && ok; ++kk) {
             const int k = r1 * C::KR + kk;
@@ -256,7 +216,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
               if (b != cur_box) {
                 if (cur_box >= 0) { ptx::mma_commit(&bars->empty[it % C::NSTAGE]); ++it; }
                 cur_box = b;
-                if (!wait_or_abort(&bars->full[it % C::NSTAGE], (it / C::NSTAGE) & 1, bars, status)) { ok = false; break; }
+                if (!wait_or_abort(&bars->full[it % C::NSTAGE], (it / C::NSTAGE) & 1, &bars->abort_flag, status)) { ok = false; break; }
                 ptx::tc_fence_after();
               }
               const uint32_t sb = ring_s + (it % C::NSTAGE) * C::STAGE_BYTES;
@@ -272,13 +232,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         ptx::mma_commit(&bars->empty[it % C::NSTAGE]);  // release the last X box
         ++it;
         // ---- wait for the permuted Z tile
-        if (!wait_or_abort(&bars->z_full, unit_n & 1, bars, status)) { ok = false; break; }
+        if (!wait_or_abort(&bars->z_full, unit_n & 1, &bars->abort_flag, status)) { ok = false; break; }
         ptx::tc_fence_after();
         // ---- L stage
         int piece = 0;
         for (int r2 = 0; r2 < C::NR2 && ok; ++r2, ++rnd) {
           const int slot = rnd & 1;
-          if (!wait_or_abort(&bars->acc_empty[slot], ((rnd >> 1) & 1) ^ 1, bars, status)) { ok = false; break; }
+          if (!wait_or_abort(&bars->acc_empty[slot], ((rnd >> 1) & 1) ^ 1, &bars->abort_flag, status)) { ok = false; break; }
           ptx::tc_fence_after();
           const int oc = r2 % C::NOC;
           for (int jj = 0; jj < C::JR && ok; ++jj) {
@@ -286,7 +246,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             for (int s = 0; s < C::KS2; ++s, ++piece) {
               if (piece % C::LPS == 0) {
                 if (piece > 0) { ptx::mma_commit(&bars->empty[it % C::NSTAGE]); ++it; }
-                if (!wait_or_abort(&bars->full[it % C::NSTAGE], (it / C::NSTAGE) & 1, bars, status)) { ok = false; break; }
+                if (!wait_or_abort(&bars->full[it % C::NSTAGE], (it / C::NSTAGE) & 1, &bars->abort_flag, status)) { ok = false; break; }
                 ptx::tc_fence_after();
               }
               const uint32_t sb = ring_s + (it % C::NSTAGE) * C::STAGE_BYTES;
@@ -322,8 +282,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       // ---- R-stage rounds -> permuted bf16 Z tile in shared memory
       for (int r1 = 0; r1 < C::NR1 && ok; ++r1, ++rnd) {
         const int slot = rnd & 1;
-        if (!wait_or_abort(&bars->acc_full[slot], (rnd >> 1) & 1, bars, status)) { ok = false; break; }
-        if (r1 == 0 && !wait_or_abort(&bars->z_empty, (unit_n & 1) ^ 1, bars, status)) { ok = false; break; }
+        if (!wait_or_abort(&bars->acc_full[slot], (rnd >> 1) & 1, &bars->abort_flag, status)) { ok = false; break; }
+        if (r1 == 0 && !wait_or_abort(&bars->z_empty, (unit_n & 1) ^ 1, &bars->abort_flag, status)) { ok = false; break; }
         ptx::tc_fence_after();
         const uint32_t tbase = tmem + lane_off + slot * C::SLOT;
 #pragma unroll 1
@@ -368,7 +328,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       // ---- L-stage rounds -> Y
       for (int r2 = 0; r2 < C::NR2 && ok; ++r2, ++rnd) {
         const int slot = rnd & 1;
-        if (!wait_or_abort(&bars->acc_full[slot], (rnd >> 1) & 1, bars, status)) { ok = false; break; }
+        if (!wait_or_abort(&bars->acc_full[slot], (rnd >> 1) & 1, &bars->abort_flag, status)) { ok = false; break; }
         ptx::tc_fence_after();
         const uint32_t tbase = tmem + lane_off + slot * C::SLOT;
         const int jb = group * C::G + (r2 / C::NOC) * C::JR;  // first global j of the round
@@ -452,50 +412,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   __syncthreads();
   ptx::tc_fence_after();
   if (warp == 1) ptx::tmem_dealloc(tmem, 512);
-}
-
-// ------------------------------------------------------------------ host side
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-static EncodeTiledFn get_encode() {
-  static EncodeTiledFn fn = nullptr;
-  if (fn == nullptr) {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = (EncodeTiledFn)p;
-  }
-  return fn;
-}
-
-// 2-D bf16 tensor map over a row-major (outer x inner) matrix.
-static bool make_map_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
-                        uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swz) {
-  EncodeTiledFn enc = get_encode();
-  if (enc == nullptr) return false;
-  cuuint64_t dims[2] = {inner, outer};
-  cuuint64_t strides[1] = {inner * 2};
-  cuuint32_t box[2] = {box_inner, box_outer};
-  cuuint32_t estr[2] = {1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
-             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-static int num_sms() {
-  static int n = 0;
-  if (n == 0) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    if (n <= 0) n = 148;
-  }
-  return n;
 }
 
 template <class C>
