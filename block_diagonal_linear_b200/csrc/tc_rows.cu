@@ -29,7 +29,7 @@ namespace monarch {
 constexpr int kRowsThreads = 448;  // 14 warps
 constexpr int kRowsDrainWarps = 8;
 constexpr int kRowsLoaderWarps = 4;
-constexpr int kLoaderLag = 6;      // commit groups a loader keeps in flight before signalling
+constexpr int kRowsLoaderThreads = kRowsLoaderWarps * 32;
 
 template <int NB1_, int IN1_, int OUT1_, int NB2_, int IN2_, int OUT2_, int OT_>
 struct RowsCfg {
@@ -74,7 +74,6 @@ struct RowsCfg {
   static_assert(NSTAGE >= 3, "shared memory");
   static_assert(LPS >= 1 && PPR % LPS == 0, "L slices per stage");
   static_assert(NXB == NR1 * BPR, "R-stage rounds align with X boxes");
-  static_assert(kLoaderLag + 2 <= NSTAGE, "loader lag must leave the MMA a free stage");
 };
 
 struct RowsBars {
@@ -110,7 +109,8 @@ __global__ void __launch_bounds__(kRowsThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::NSTAGE; ++i) {
-      ptx::mbar_init(&bars->full[i], 1 + kRowsLoaderWarps);
+      // producer arrive (+ X bytes) and one cp.async completion arrival per loader thread
+      ptx::mbar_init(&bars->full[i], 1 + kRowsLoaderThreads);
       ptx::mbar_init(&bars->empty[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
@@ -180,6 +180,7 @@ __global__ void __launch_bounds__(kRowsThreads, 1)
         for (int bb = 0; bb < C::BPR; ++bb, ++it) {
           const int st = it % C::NSTAGE;
           if (!warp_wait_or_abort(lane, &bars->full[st], (it / C::NSTAGE) & 1, abort_flag, status)) { ok = false; break; }
+          ptx::fence_proxy_async_smem();  // weight slices were written by cp.async (generic proxy)
           ptx::tc_fence_after();
           const uint64_t soff = (uint64_t)((st * C::STAGE_BYTES) >> 4);
 #pragma unroll
@@ -208,6 +209,7 @@ __global__ void __launch_bounds__(kRowsThreads, 1)
         for (int sp = 0; sp < C::SPR; ++sp, ++it) {
           const int st = it % C::NSTAGE;
           if (!warp_wait_or_abort(lane, &bars->full[st], (it / C::NSTAGE) & 1, abort_flag, status)) { ok = false; break; }
+          ptx::fence_proxy_async_smem();  // weight slices were written by cp.async (generic proxy)
           ptx::tc_fence_after();
           const uint64_t soff = (uint64_t)((st * C::STAGE_BYTES) >> 4);
 #pragma unroll
@@ -234,9 +236,11 @@ __global__ void __launch_bounds__(kRowsThreads, 1)
     // Each stage gets its weight slices (R slices of the X box's four K steps, or
     // LPS slices of L) as 16-byte cp.async chunks written in the 32B-swizzled
     // K-major layout: chunk c of row n of a slice lands at n*32 + ((c ^ ((n>>2)&1)) << 4).
+    // Every loader thread then arrives on the stage's full barrier when its own
+    // copies have landed (cp.async.mbarrier.arrive.noinc); the MMA warp fences the
+    // async proxy after observing the barrier.
     const int lt = (warp - 2 - kRowsDrainWarps) * 32 + lane;
     const uint32_t ring_s = ptx::smem_u32(ring);
-    constexpr int NLT = kRowsLoaderWarps * 32;
     uint32_t it = 0;
     bool ok = true;
     for (int64_t u = blockIdx.x; u < nunits && ok; u += gridDim.x) {
@@ -246,7 +250,7 @@ __global__ void __launch_bounds__(kRowsThreads, 1)
         const uint32_t sb = ring_s + st * C::STAGE_BYTES;
         if (sq < C::NXB) {
           const int b = sq;
-          for (int g = lt; g < 4 * C::OUT1 * 2; g += NLT) {
+          for (int g = lt; g < 4 * C::OUT1 * 2; g += kRowsLoaderThreads) {
             const int t = g / (C::OUT1 * 2), n = (g >> 1) % C::OUT1, c = g & 1;
             const int col = b * 64 + t * 16;
             const int k = col / C::IN1, s16 = col % C::IN1;
@@ -256,29 +260,17 @@ __global__ void __launch_bounds__(kRowsThreads, 1)
         } else {
           const int p0 = (sq - C::NXB) * C::LPS;
           const int np = (C::NPIECE2 - p0) < C::LPS ? (C::NPIECE2 - p0) : C::LPS;
-          for (int g = lt; g < np * C::OUT2 * 2; g += NLT) {
+          for (int g = lt; g < np * C::OUT2 * 2; g += kRowsLoaderThreads) {
             const int t = g / (C::OUT2 * 2), n = (g >> 1) % C::OUT2, c = g & 1;
             const int pi = p0 + t, j = pi / C::KS2, s16 = (pi % C::KS2) * 16;
             ptx::cp_async_16(sb + t * C::LPIECE + n * 32 + ((c ^ ((n >> 2) & 1)) << 4),
                              L + ((int64_t)j * C::OUT2 + n) * C::IN2 + s16 + c * 8);
           }
         }
-        ptx::cp_async_commit();
-        if (it >= (uint32_t)kLoaderLag) {
-          ptx::cp_async_wait<kLoaderLag>();
-          ptx::fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) ptx::mbar_arrive(&bars->full[(it - kLoaderLag) % C::NSTAGE]);
-        }
+        ptx::cp_async_mbar_arrive_noinc(&bars->full[st]);
       }
     }
-    // signal the stages still in flight
-    ptx::cp_async_wait<0>();
-    ptx::fence_proxy_async_smem();
-    __syncwarp();
-    if (lane == 0)
-      for (uint32_t k = (it > (uint32_t)kLoaderLag ? it - kLoaderLag : 0); k < it; ++k)
-        ptx::mbar_arrive(&bars->full[k % C::NSTAGE]);
+    ptx::cp_async_wait<0>();  // no copy may still target this CTA's shared memory at exit
   } else {
     // ================================================================ drain (8 warps)
     const int quad = warp & 3;              // TMEM lane quadrant of this warp
