@@ -390,7 +390,8 @@ def main():
         }
     fpath = bdl.fwd_path(shape, w["dtype"])
     fwd_tc = fpath >= 1
-    launches_per_step = (1 if do_fwd else 0) + (3 if do_bwd else 0)
+    bpath = bdl.bwd_path(shape, w["dtype"])
+    launches_per_step = (1 if do_fwd else 0) + ((6 if bpath == 1 else 3) if do_bwd else 0)
     dom = "fwd" if fwd_avg_s >= bwd_avg_s else "bwd"
     a = alg[dom]
     t_dom = fwd_avg_s if dom == "fwd" else bwd_avg_s
@@ -407,7 +408,7 @@ def main():
                 "peak": peaks["bf16_tflops"], "unit": "TFLOP/s"}
     roof["frac"] = roof["achieved"] / roof["peak"]
     roof["traffic"] = measured_traffic(kname, srcs) if dom == "fwd" and fwd_tc else None
-    roof["kernel"] = kname + (" (pass of 3 kernels)" if dom == "bwd" else "")
+    roof["kernel"] = kname + (" (pass of %d kernels)" % (6 if bpath == 1 else 3) if dom == "bwd" else "")
     roof["algorithmic_bytes_per_launch"] = a["bytes"]
     roof["peak_source"] = peak_src
 

@@ -83,9 +83,17 @@ int monarch_fwd_path(const monarch_dims* d) {
   return fwd_path(to_shape(*d), d->dtype);
 }
 
+static int bwd_path(const Shape& s, int dtype) {
+  return (dtype == MONARCH_BF16 && fast_bwd_supported(s)) ? 1 : 0;
+}
+
+static size_t bwd_workspace(const Shape& s, int dtype) {
+  return bwd_path(s, dtype) == 1 ? fast_bwd_workspace(s) : generic_bwd_workspace(s);
+}
+
 int monarch_bwd_path(const monarch_dims* d) {
   if (check_dims(d) != MONARCH_OK) return -1;
-  return 0;
+  return bwd_path(to_shape(*d), d->dtype);
 }
 
 int monarch_fwd(const void* X, const void* R, const void* L, const monarch_dims* d, void* Y,
@@ -111,7 +119,7 @@ int monarch_fwd(const void* X, const void* R, const void* L, const monarch_dims*
 
 size_t monarch_bwd_workspace_bytes(const monarch_dims* d) {
   if (check_dims(d) != MONARCH_OK) return 0;
-  return generic_bwd_workspace(to_shape(*d));
+  return bwd_workspace(to_shape(*d), d->dtype);
 }
 
 int monarch_bwd(const void* dY, const void* X, const void* R, const void* L, const monarch_dims* d,
@@ -122,11 +130,18 @@ int monarch_bwd(const void* dY, const void* X, const void* R, const void* L, con
   if ((rc = check_ptrs({R, L, dR, dL})) != MONARCH_OK) return rc;
   if (d->rows > 0 && (rc = check_ptrs({dY, X, dX})) != MONARCH_OK) return rc;
   const Shape s = to_shape(*d);
-  const size_t need = generic_bwd_workspace(s);
+  const size_t need = bwd_workspace(s, d->dtype);
   if (workspace == nullptr || workspace_bytes < need) return MONARCH_ERR_WORKSPACE;
   if (((uintptr_t)workspace & 255u) != 0) return MONARCH_ERR_ALIGN;
-  if (!generic_bwd_supported(s)) return MONARCH_ERR_UNSUPPORTED;
-  cudaError_t e = generic_bwd(dY, X, R, L, dX, dR, dL, workspace, s, d->dtype, (cudaStream_t)stream);
+  cudaError_t e;
+  if (bwd_path(s, d->dtype) == 1) {
+    int* status = status_ptr();
+    if (status == nullptr) return MONARCH_ERR_CUDA;
+    e = fast_bwd(dY, X, R, L, dX, dR, dL, workspace, s, status, (cudaStream_t)stream);
+  } else {
+    if (!generic_bwd_supported(s)) return MONARCH_ERR_UNSUPPORTED;
+    e = generic_bwd(dY, X, R, L, dX, dR, dL, workspace, s, d->dtype, (cudaStream_t)stream);
+  }
   return e == cudaSuccess ? MONARCH_OK : MONARCH_ERR_CUDA;
 }
 

@@ -69,6 +69,12 @@ bool tc_rows_supported(const Shape& s);
 cudaError_t tc_rows_fwd(const void* X, const void* R, const void* L, void* Y, const Shape& s,
                         int* status, cudaStream_t st);
 
+// Tensor-core backward of the square small-block shapes (bf16).
+bool fast_bwd_supported(const Shape& s);
+size_t fast_bwd_workspace(const Shape& s);
+cudaError_t fast_bwd(const void* dY, const void* X, const void* R, const void* L, void* dX, void* dR,
+                     void* dL, void* ws, const Shape& s, int* status, cudaStream_t st);
+
 cudaError_t debug_wait_timeout(uint64_t timeout_ns, int* status, cudaStream_t st);
 
 }  // namespace monarch

@@ -31,10 +31,13 @@ constexpr int kRowsDrainWarps = 8;
 constexpr int kRowsLoaderWarps = 4;
 constexpr int kRowsLoaderThreads = kRowsLoaderWarps * 32;
 
-template <int NB1_, int IN1_, int OUT1_, int NB2_, int IN2_, int OUT2_, int OT_>
+// MODE 0: Y only.  MODE 1: Y, and the middle tile (bf16, block-contiguous) is also
+// stored through tmZ.  MODE 2: R stage and permutation only; the middle tile is the
+// output (tmZ).
+template <int NB1_, int IN1_, int OUT1_, int NB2_, int IN2_, int OUT2_, int OT_, int MODE_ = 0>
 struct RowsCfg {
   static constexpr int NB1 = NB1_, IN1 = IN1_, OUT1 = OUT1_;
-  static constexpr int NB2 = NB2_, IN2 = IN2_, OUT2 = OUT2_, OT = OT_;
+  static constexpr int NB2 = NB2_, IN2 = IN2_, OUT2 = OUT2_, OT = OT_, MODE = MODE_;
   static constexpr int N_IN = NB1 * IN1, N_MID = NB1 * OUT1, N_OUT = NB2 * OUT2;
   static constexpr int BM = 64;
   static constexpr int KS1 = IN1 / 16, KS2 = IN2 / 16;
@@ -53,7 +56,7 @@ struct RowsCfg {
   static constexpr int LPS = LPS_MAX >= PPR ? PPR : (LPS_MAX >= PPR / 2 ? PPR / 2 : (LPS_MAX >= PPR / 4 ? PPR / 4 : (LPS_MAX >= PPR / 8 ? PPR / 8 : PPR / 16)));
   static constexpr int SPR = PPR / LPS;   // ring stages per L-stage round
   static constexpr int NPIECE2 = NB2 * KS2;
-  static constexpr int NSTAGE2 = NR2 * SPR;
+  static constexpr int NSTAGE2 = MODE == 2 ? 0 : NR2 * SPR;
   static constexpr int BPR = IN1 / 4;     // X boxes (64 columns) per R-stage round of 16 blocks
   static constexpr int ATOM_BYTES = BM * 128;  // 64 rows x 64 bf16 columns
   static constexpr int ZATOMS = N_MID / 64;
@@ -79,7 +82,7 @@ struct RowsCfg {
 struct RowsBars {
   uint64_t full[12], empty[12];
   uint64_t acc_full[2], acc_empty[2];
-  uint64_t z_full, zfree, staged, mma_done;
+  uint64_t z_full, zfree, staged, zsaved, mma_done;
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -95,6 +98,7 @@ __device__ __forceinline__ uint32_t atom_chunk_off(int r, int c) {
 template <class C>
 __global__ void __launch_bounds__(kRowsThreads, 1)
     tc_rows_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmY,
+                   const __grid_constant__ CUtensorMap tmZ,
                    const __nv_bfloat16* __restrict__ R, const __nv_bfloat16* __restrict__ L,
                    int64_t rows, int* status) {
   extern __shared__ uint8_t smem_raw[];
@@ -120,6 +124,7 @@ __global__ void __launch_bounds__(kRowsThreads, 1)
     ptx::mbar_init(&bars->z_full, kRowsDrainWarps);
     ptx::mbar_init(&bars->zfree, kRowsDrainWarps);
     ptx::mbar_init(&bars->staged, kRowsDrainWarps);
+    ptx::mbar_init(&bars->zsaved, 1);
     ptx::mbar_init(&bars->mma_done, 1);
     bars->abort_flag = 0;
     ptx::fence_mbar_init();
@@ -137,7 +142,8 @@ __global__ void __launch_bounds__(kRowsThreads, 1)
     // ================================================================ TMA producer (X)
     if (lane == 0) {
       ptx::tma_prefetch_desc(&tmX);
-      ptx::tma_prefetch_desc(&tmY);
+      if (C::MODE != 2) ptx::tma_prefetch_desc(&tmY);
+      if (C::MODE != 0) ptx::tma_prefetch_desc(&tmZ);
       const uint64_t pol_x = ptx::policy_evict_first();
       uint32_t it = 0;
       bool ok = true;
@@ -198,6 +204,7 @@ __global__ void __launch_bounds__(kRowsThreads, 1)
         ptx::mma_commit_elect(&bars->acc_full[slot]);
       }
       if (!ok) break;
+      if (C::MODE == 2) continue;  // no L stage
       if (!warp_wait_or_abort(lane, &bars->z_full, unit_n & 1, abort_flag, status)) { ok = false; break; }
       ptx::tc_fence_after();
       // ---- L stage: round r2 covers blocks [16 r2, 16 r2 + 16), SPR ring stages of LPS slices
@@ -322,12 +329,41 @@ __global__ void __launch_bounds__(kRowsThreads, 1)
       if (!ok) break;
       ptx::fence_proxy_async_smem();
       __syncwarp();
+      if (C::MODE == 2) {
+        // the middle tile is the output: hand it to the TMA store engine
+        if (lane == 0) ptx::mbar_arrive(&bars->staged);
+        if (leader) {
+          if (!wait_or_abort(&bars->staged, unit_n & 1, abort_flag, status)) {
+            ok = false;
+          } else {
+            const int row0 = (int)(u * C::BM);
+            for (int a = 0; a < C::ZATOMS; ++a) ptx::tma_store_2d(&tmZ, zbuf + a * C::ATOM_BYTES, a * 64, row0);
+            ptx::bulk_commit_group();
+          }
+        }
+        continue;
+      }
       if (lane == 0) ptx::mbar_arrive(&bars->z_full);
+      if (C::MODE == 1) {
+        // side output of the middle tile; it must be read out before the staging reuses it
+        if (lane == 0) ptx::mbar_arrive(&bars->staged);
+        if (leader) {
+          // `staged` completes twice per unit in this mode: phase 2n (middle tile), 2n+1 (Y)
+          if (wait_or_abort(&bars->staged, 0u, abort_flag, status)) {
+            const int row0 = (int)(u * C::BM);
+            for (int a = 0; a < C::ZATOMS; ++a) ptx::tma_store_2d(&tmZ, zbuf + a * C::ATOM_BYTES, a * 64, row0);
+            ptx::bulk_commit_group();
+            ptx::bulk_wait_read_all();
+          }
+          ptx::mbar_arrive(&bars->zsaved);
+        }
+      }
       // ---- L-stage rounds: wait for all of them (Z is then dead), stage the output rows
       const uint32_t rnd0 = rnd;
       for (int r2 = 0; r2 < C::NR2 && ok; ++r2)
         if (!wait_or_abort(&bars->acc_full[(rnd0 + r2) & 1], ((rnd0 + r2) >> 1) & 1, abort_flag, status)) ok = false;
       if (!ok) break;
+      if (C::MODE == 1 && !wait_or_abort(&bars->zsaved, unit_n & 1, abort_flag, status)) { ok = false; break; }
       ptx::tc_fence_after();
       for (int r2 = 0; r2 < C::NR2; ++r2, ++rnd) {
         const uint32_t tb = tmem + lane_off + (rnd & 1) * C::SLOT;
@@ -370,7 +406,7 @@ __global__ void __launch_bounds__(kRowsThreads, 1)
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(&bars->staged);
       if (leader) {
-        if (!wait_or_abort(&bars->staged, unit_n & 1, abort_flag, status)) {
+        if (!wait_or_abort(&bars->staged, C::MODE == 1 ? 1u : (unit_n & 1), abort_flag, status)) {
           ok = false;
         } else {
           const int row0 = (int)(u * C::BM);
@@ -388,27 +424,45 @@ __global__ void __launch_bounds__(kRowsThreads, 1)
   if (warp == 1) ptx::tmem_dealloc(tmem, C::TMEM_COLS);
 }
 
+// Run one row-tile kernel.  X: (rows, N_IN) input; W1 (nb1, out1, in1) and W2
+// (nb2, out2, in2) the stage weights in the forward layout; Y (rows, N_OUT) output
+// (MODE 0/1); Zout (rows, N_MID) middle tile (MODE 1/2).
 template <class C>
-static cudaError_t launch_rows(const void* X, const void* R, const void* L, void* Y, const Shape& s,
-                               int* status, cudaStream_t st) {
-  if (s.rows == 0) return cudaSuccess;
-  CUtensorMap mX, mY;
-  if (!make_map_2d(&mX, X, C::N_IN, (uint64_t)s.rows, 64, C::BM, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_map_2d(&mY, Y, C::N_OUT, (uint64_t)s.rows, 64, C::BM, CU_TENSOR_MAP_SWIZZLE_128B))
+static cudaError_t launch_rows(const void* X, const void* W1, const void* W2, void* Y, void* Zout,
+                               int64_t rows, int* status, cudaStream_t st) {
+  if (rows == 0) return cudaSuccess;
+  CUtensorMap mX, mY, mZ;
+  if (!make_map_2d(&mX, X, C::N_IN, (uint64_t)rows, 64, C::BM, CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  mY = mX;
+  mZ = mX;
+  if (C::MODE != 2 &&
+      !make_map_2d(&mY, Y, C::N_OUT, (uint64_t)rows, 64, C::BM, CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  if (C::MODE != 0 &&
+      !make_map_2d(&mZ, Zout, C::N_MID, (uint64_t)rows, 64, C::BM, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(tc_rows_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        C::SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  const int64_t nunits = (s.rows + C::BM - 1) / C::BM;
+  const int64_t nunits = (rows + C::BM - 1) / C::BM;
   int64_t grid = num_sms();
   if (grid > nunits) grid = nunits;
   tc_rows_kernel<C><<<(unsigned)grid, kRowsThreads, C::SMEM_BYTES, st>>>(
-      mX, mY, (const __nv_bfloat16*)R, (const __nv_bfloat16*)L, s.rows, status);
+      mX, mY, mZ, (const __nv_bfloat16*)W1, (const __nv_bfloat16*)W2, rows, status);
   return cudaGetLastError();
 }
 
 using RowsSq16 = RowsCfg<16, 16, 16, 16, 16, 16, 1>;  // n = 256 = 16^2
 using RowsSq32 = RowsCfg<32, 32, 32, 32, 32, 32, 1>;  // n = 1024 = 32^2
+// Backward of the square shapes (in2 == nb1, out1 == nb2): the dual map
+// dU = P^-1 (L^T-stage(dV)), dX = R^T-stage(dU) is a row-tile map with the
+// transposed factors and no output transpose; MODE 1 also stores dU.
+using RowsSq16Bwd = RowsCfg<16, 16, 16, 16, 16, 16, 0, 1>;
+using RowsSq32Bwd = RowsCfg<32, 32, 32, 32, 32, 32, 0, 1>;
+// R stage and permutation only (Z = P R x), for the weight gradient of L.
+using RowsSq16Z = RowsCfg<16, 16, 16, 16, 16, 16, 1, 2>;
+using RowsSq32Z = RowsCfg<32, 32, 32, 32, 32, 32, 1, 2>;
 
 template <class C>
 static bool rows_shape_is(const Shape& s) {
@@ -422,8 +476,24 @@ bool tc_rows_supported(const Shape& s) {
 
 cudaError_t tc_rows_fwd(const void* X, const void* R, const void* L, void* Y, const Shape& s,
                         int* status, cudaStream_t st) {
-  if (rows_shape_is<RowsSq16>(s)) return launch_rows<RowsSq16>(X, R, L, Y, s, status, st);
-  if (rows_shape_is<RowsSq32>(s)) return launch_rows<RowsSq32>(X, R, L, Y, s, status, st);
+  if (rows_shape_is<RowsSq16>(s)) return launch_rows<RowsSq16>(X, R, L, Y, nullptr, s.rows, status, st);
+  if (rows_shape_is<RowsSq32>(s)) return launch_rows<RowsSq32>(X, R, L, Y, nullptr, s.rows, status, st);
+  return cudaErrorNotSupported;
+}
+
+// Z = P R x for every row (block-contiguous middle vector, bf16).
+cudaError_t tc_rows_middle(const void* X, const void* R, void* Z, const Shape& s, int* status,
+                           cudaStream_t st) {
+  if (rows_shape_is<RowsSq16>(s)) return launch_rows<RowsSq16Z>(X, R, nullptr, nullptr, Z, s.rows, status, st);
+  if (rows_shape_is<RowsSq32>(s)) return launch_rows<RowsSq32Z>(X, R, nullptr, nullptr, Z, s.rows, status, st);
+  return cudaErrorNotSupported;
+}
+
+// dX and dU from the block-contiguous dV with the transposed factors Lt, Rt.
+cudaError_t tc_rows_dual(const void* dV, const void* Lt, const void* Rt, void* dX, void* dU,
+                         const Shape& s, int* status, cudaStream_t st) {
+  if (rows_shape_is<RowsSq16>(s)) return launch_rows<RowsSq16Bwd>(dV, Lt, Rt, dX, dU, s.rows, status, st);
+  if (rows_shape_is<RowsSq32>(s)) return launch_rows<RowsSq32Bwd>(dV, Lt, Rt, dX, dU, s.rows, status, st);
   return cudaErrorNotSupported;
 }
 
