@@ -33,13 +33,14 @@ STATUS = {
     -6: "MONARCH_ERR_CUDA",
     -7: "MONARCH_ERR_TIMEOUT",
     -8: "MONARCH_ERR_UNSUPPORTED",
+    -9: "MONARCH_ERR_SCRATCH",
 }
 CODES = {v: k for k, v in STATUS.items()}
 
 EXPORTED = (
     "monarch_validate", "monarch_fwd", "monarch_bwd", "monarch_bwd_workspace_bytes",
     "monarch_materialise", "monarch_status_string", "monarch_last_device_status",
-    "monarch_debug_wait_timeout", "monarch_fwd_path", "monarch_bwd_path",
+    "monarch_debug_wait_timeout", "monarch_fwd_path", "monarch_bwd_path", "monarch_bwd_noalloc",
 )
 
 
@@ -86,11 +87,12 @@ def lib() -> ctypes.CDLL:
         L.monarch_status_string.restype = ctypes.c_char_p
         L.monarch_last_device_status.argtypes = [vp]
         L.monarch_debug_wait_timeout.argtypes = [ctypes.c_uint64, vp]
+        L.monarch_bwd_noalloc.argtypes = [vp, vp, vp, vp, dp, vp, vp, vp, vp]
         L.monarch_fwd_path.argtypes = [dp]
         L.monarch_bwd_path.argtypes = [dp]
         for name in ("monarch_validate", "monarch_fwd", "monarch_bwd", "monarch_materialise",
                      "monarch_last_device_status", "monarch_debug_wait_timeout",
-                     "monarch_fwd_path", "monarch_bwd_path"):
+                     "monarch_fwd_path", "monarch_bwd_path", "monarch_bwd_noalloc"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -193,6 +195,27 @@ def bwd(dY, X, R, L, shape: dict, dX=None, dR=None, dL=None, workspace=None, str
     _check("monarch_bwd", lib().monarch_bwd(
         _ptr(dY), _ptr(X), _ptr(R), _ptr(L), ctypes.byref(d), _ptr(dX), _ptr(dR), _ptr(dL),
         _ptr(workspace), ctypes.c_size_t(workspace.numel() * workspace.element_size()),
+        _stream(stream)))
+    return dX, dR, dL
+
+
+def bwd_noalloc(dY, X, R, L, shape: dict, dX=None, dR=None, dL=None, stream=None):
+    """Backward without a workspace argument, for callers that cannot allocate device
+    memory: the library's own fixed 32 MiB device scratch is used instead (problems
+    needing more raise MonarchError with MONARCH_ERR_SCRATCH).  Calls that overlap on
+    the GPU share that scratch and must not run concurrently."""
+    import torch
+    code = dtype_code(X.dtype)
+    if dX is None:
+        dX = torch.empty_like(X)
+    if dR is None:
+        dR = torch.empty_like(R)
+    if dL is None:
+        dL = torch.empty_like(L)
+    _require_cuda(dY, X, R, L, dX, dR, dL)
+    d = make_dims(shape, X.shape[0], code)
+    _check("monarch_bwd_noalloc", lib().monarch_bwd_noalloc(
+        _ptr(dY), _ptr(X), _ptr(R), _ptr(L), ctypes.byref(d), _ptr(dX), _ptr(dR), _ptr(dL),
         _stream(stream)))
     return dX, dR, dL
 

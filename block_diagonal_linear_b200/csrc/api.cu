@@ -165,6 +165,7 @@ const char* monarch_status_string(int status) {
     case MONARCH_ERR_CUDA: return "CUDA error";
     case MONARCH_ERR_TIMEOUT: return "bounded device wait timed out";
     case MONARCH_ERR_UNSUPPORTED: return "shape not supported by any kernel";
+    case MONARCH_ERR_SCRATCH: return "problem larger than the fixed scratch of monarch_bwd_noalloc";
     default: return "unknown status";
   }
 }

@@ -68,7 +68,8 @@ enum {
   MONARCH_ERR_WORKSPACE = -5,   /* workspace NULL or smaller than required */
   MONARCH_ERR_CUDA = -6,        /* a CUDA runtime call or kernel launch failed */
   MONARCH_ERR_TIMEOUT = -7,     /* a bounded device wait gave up (device status) */
-  MONARCH_ERR_UNSUPPORTED = -8  /* shape too large for any kernel of this build */
+  MONARCH_ERR_UNSUPPORTED = -8, /* shape too large for any kernel of this build */
+  MONARCH_ERR_SCRATCH = -9      /* monarch_bwd_noalloc: problem needs more than its fixed scratch */
 };
 
 /* Shape of one Monarch map.  Scatterbrain thread, MonarchLinear __init__ and
@@ -107,6 +108,31 @@ MONARCH_API int monarch_fwd(const void* X, const void* R, const void* L, const m
 MONARCH_API int monarch_bwd(const void* dY, const void* X, const void* R, const void* L, const monarch_dims* d,
                 void* dX, void* dR, void* dL, void* workspace, size_t workspace_bytes,
                 void* stream);
+
+/* Same as monarch_bwd, for callers that cannot allocate device memory.
+ * The pages describe no such entry point; it exists for integration.  Some callers
+ * have no way to provide the workspace monarch_bwd wants: code that only receives
+ * tensors from a host framework, processes whose device memory pool is fixed in
+ * advance, or code that must not call the CUDA allocator at that point.  This
+ * entry point runs the same kernels but takes its scratch from a 32 MiB array that
+ * is part of the library's device code; it calls no cudaMalloc, cudaFree or other
+ * allocating routine.
+ *   - Limit: problems whose monarch_bwd_workspace_bytes(d) exceeds 32 MiB are
+ *     rejected with MONARCH_ERR_SCRATCH before any device work (for the n = 1024
+ *     bf16 shape that is about 2000 rows; larger batches must use monarch_bwd).
+ *   - Every GPU that loads the library holds the 32 MiB array until the process
+ *     exits.
+ *   - The first call made with a given device current looks up the array's device
+ *     address (cudaGetSymbolAddress) and caches it; make that first call before
+ *     any stream capture.
+ *   - All calls share the one array and it keeps the previous call's contents
+ *     (nothing in it needs to start at zero).  Calls whose execution overlaps on
+ *     the GPU (different streams, or several host threads on one device) race on
+ *     it and give wrong results; serialise them.
+ * Arguments, layouts and results are those of monarch_bwd. */
+MONARCH_API int monarch_bwd_noalloc(const void* dY, const void* X, const void* R, const void* L,
+                                    const monarch_dims* d, void* dX, void* dR, void* dL,
+                                    void* stream);
 
 /* Workspace bytes monarch_bwd needs for this shape (0 if d is invalid). */
 MONARCH_API size_t monarch_bwd_workspace_bytes(const monarch_dims* d);
