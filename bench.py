@@ -268,10 +268,11 @@ def main():
     flush = torch.empty(max(2 * l2, 256 << 20), dtype=torch.uint8, device=dev_)
     stream = torch.cuda.current_stream()
 
+    from block_diagonal_linear_b200 import dp
+
     def allreduce_grads():
         if world > 1:
-            dist.all_reduce(dR)
-            dist.all_reduce(dL)
+            dp.allreduce_weight_grads(dR, dL)
 
     do_fwd = args.only in ("step", "fwd")
     do_bwd = args.only in ("step", "bwd")
@@ -392,7 +393,11 @@ def main():
     fwd_tc = fpath >= 1
     bpath = bdl.bwd_path(shape, w["dtype"])
     launches_per_step = (1 if do_fwd else 0) + ((6 if bpath == 1 else 3) if do_bwd else 0)
-    dom = "fwd" if fwd_avg_s >= bwd_avg_s else "bwd"
+    # Roofline object: the forward kernel (one launch per forward pass, so the pass time
+    # measured by the events is that kernel's launch duration).  The row-tile kernel
+    # family is also the largest share of the step in the ncu launch list.  When only
+    # the backward is timed, the backward pass (several launches) is reported instead.
+    dom = "fwd" if do_fwd else "bwd"
     a = alg[dom]
     t_dom = fwd_avg_s if dom == "fwd" else bwd_avg_s
     bound = passes[dom]["bound"]

@@ -40,41 +40,40 @@ __global__ void transpose_factors_kernel(const __nv_bfloat16* __restrict__ R,
   }
 }
 
-// dV[r][j*out2 + o] = dY[r][o*nb2 + j]: per row an (out2 x nb2) -> (nb2 x out2) transpose
-// through shared memory, 8 rows per step; global reads and writes are 16-byte and coalesced.
-constexpr int kGatherRows = 8;
-__global__ void __launch_bounds__(256) gather_dv_kernel(const __nv_bfloat16* __restrict__ dY,
-                                                        __nv_bfloat16* __restrict__ dV, Shape s) {
-  extern __shared__ __align__(16) uint16_t sh[];
+// dV[r][j*out2 + o] = dY[r][o*nb2 + j]: per row an (out2 x nb2) -> (nb2 x out2)
+// transpose.  One warp per row: the row is read with 16-byte coalesced loads, staged in
+// shared memory with an odd word pitch (nb2 + 2 elements, so the column reads of the
+// transpose hit 32 different banks), and written back with 16-byte coalesced stores.
+constexpr int kGatherWarps = 8;
+__global__ void __launch_bounds__(kGatherWarps * 32)
+    gather_dv_kernel(const __nv_bfloat16* __restrict__ dY, __nv_bfloat16* __restrict__ dV, Shape s) {
+  extern __shared__ __align__(16) uint32_t shw[];
   const int n = (int)s.n_out(), nb2 = s.nb2, out2 = s.out2;
-  const int pitch = n + 8;  // elements per staged row (keeps 16-byte alignment)
-  const int chunks = n / 8;
-  for (int64_t r0 = (int64_t)blockIdx.x * kGatherRows; r0 < s.rows; r0 += (int64_t)gridDim.x * kGatherRows) {
-    const int nr = (int)min((int64_t)kGatherRows, s.rows - r0);
-    for (int c = threadIdx.x; c < nr * chunks; c += blockDim.x) {
-      const int rr = c / chunks, cc = c % chunks;
-      *(uint4*)(sh + rr * pitch + cc * 8) = *(const uint4*)(dY + (r0 + rr) * n + cc * 8);
+  const int pitch = nb2 + 2;          // elements per staged grid row (o)
+  const int wpitch = pitch / 2;       // 32-bit words per staged grid row
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  uint32_t* buf = shw + warp * (out2 * wpitch);
+  const uint16_t* hb = (const uint16_t*)buf;
+  for (int64_t r = (int64_t)blockIdx.x * kGatherWarps + warp; r < s.rows;
+       r += (int64_t)gridDim.x * kGatherWarps) {
+    const __nv_bfloat16* src = dY + r * n;
+    for (int c = lane; c < n / 8; c += 32) {  // chunk c: o = (8c) / nb2, j0 = (8c) % nb2
+      const uint4 v = *(const uint4*)(src + c * 8);
+      const int o = (c * 8) / nb2, j0 = (c * 8) % nb2;
+      uint32_t* d = buf + o * wpitch + j0 / 2;
+      d[0] = v.x; d[1] = v.y; d[2] = v.z; d[3] = v.w;
     }
-    __syncthreads();
-    for (int c = threadIdx.x; c < nr * chunks; c += blockDim.x) {
-      const int rr = c / chunks, cc = c % chunks;  // output chunk: columns [cc*8, cc*8+8)
+    __syncwarp();
+    __nv_bfloat16* dst = dV + r * n;
+    for (int c = lane; c < n / 8; c += 32) {  // output chunk: j = (8c) / out2, o0 = (8c) % out2
+      const int j = (c * 8) / out2, o0 = (c * 8) % out2;
       uint32_t w[4];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        uint32_t lo, hi;
-        {
-          const int col = cc * 8 + 2 * e, j = col / out2, o = col % out2;
-          lo = sh[rr * pitch + o * nb2 + j];
-        }
-        {
-          const int col = cc * 8 + 2 * e + 1, j = col / out2, o = col % out2;
-          hi = sh[rr * pitch + o * nb2 + j];
-        }
-        w[e] = lo | (hi << 16);
-      }
-      *(uint4*)(dV + (r0 + rr) * n + cc * 8) = make_uint4(w[0], w[1], w[2], w[3]);
+      for (int e = 0; e < 4; ++e)
+        w[e] = (uint32_t)hb[(o0 + 2 * e) * pitch + j] | ((uint32_t)hb[(o0 + 2 * e + 1) * pitch + j] << 16);
+      *(uint4*)(dst + c * 8) = make_uint4(w[0], w[1], w[2], w[3]);
     }
-    __syncthreads();
+    __syncwarp();
   }
 }
 
@@ -273,8 +272,8 @@ cudaError_t fast_bwd(const void* dY, const void* X, const void* R, const void* L
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   const int nsplit = wg_nsplit(s);
   if (s.rows > 0) {
-    const size_t gsm = (size_t)kGatherRows * (size_t)(s.n_out() + 8) * 2;
-    gather_dv_kernel<<<296, 256, gsm, st>>>((const __nv_bfloat16*)dY, dV, s);
+    const size_t gsm = (size_t)kGatherWarps * (size_t)s.out2 * (size_t)(s.nb2 + 2) * 2;
+    gather_dv_kernel<<<2 * 148, kGatherWarps * 32, gsm, st>>>((const __nv_bfloat16*)dY, dV, s);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if ((e = tc_rows_middle(X, R, Z, s, status, st)) != cudaSuccess) return e;
     if ((e = tc_rows_dual(dV, Lt, Rt, dX, dU, s, status, st)) != cudaSuccess) return e;
