@@ -401,9 +401,9 @@ def main():
     a = alg[dom]
     t_dom = fwd_avg_s if dom == "fwd" else bwd_avg_s
     bound = passes[dom]["bound"]
-    kname = ({2: "tc_rows_kernel", 1: "tc_fwd_kernel"}.get(fpath, "gen_fwd_kernel")
+    kname = ({2: "tc_rows_kernel", 3: "tc_wide_kernel", 1: "tc_fwd_kernel"}.get(fpath, "gen_fwd_kernel")
              if dom == "fwd" else "monarch_bwd")
-    srcs = ["block_diagonal_linear_b200/csrc/%s.cu" % {2: "tc_rows", 1: "tc_fwd"}.get(fpath, "generic"),
+    srcs = ["block_diagonal_linear_b200/csrc/%s.cu" % {2: "tc_rows", 3: "tc_wide", 1: "tc_fwd"}.get(fpath, "generic"),
             "block_diagonal_linear_b200/csrc/ptx.cuh", "block_diagonal_linear_b200/csrc/tc_common.cuh"]
     if bound == "hbm":
         roof = {"bound": "hbm", "achieved": a["bytes"] / t_dom / 1e9, "peak": peaks["hbm_gbs"],

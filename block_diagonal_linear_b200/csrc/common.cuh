@@ -69,6 +69,11 @@ bool tc_rows_supported(const Shape& s);
 cudaError_t tc_rows_fwd(const void* X, const void* R, const void* L, void* Y, const Shape& s,
                         int* status, cudaStream_t st);
 
+// tcgen05 fused forward for transposed outputs wider than the middle vector (768 -> 3072).
+bool tc_wide_supported(const Shape& s);
+cudaError_t tc_wide_fwd(const void* X, const void* R, const void* L, void* Y, const Shape& s,
+                        int* status, cudaStream_t st);
+
 // Tensor-core backward of the square small-block shapes (bf16).
 bool fast_bwd_supported(const Shape& s);
 size_t fast_bwd_workspace(const Shape& s);

@@ -164,7 +164,9 @@ MONARCH_API int monarch_debug_wait_timeout(uint64_t timeout_ns, void* stream);
 /* Which kernel family monarch_fwd / monarch_bwd would run for this shape:
  * 0 = generic FMA kernels, 1 = tcgen05 fused kernel over (128-row tile, block
  * group) units, 2 = tcgen05 fused kernel over 64-row tiles with the whole middle
- * vector on chip.  For the backward: 0 = generic FMA kernels, 1 = tensor-core
+ * vector on chip, 3 = the same with the second block-diagonal stage computed in
+ * rounds of 8 output columns (transposed outputs wider than the middle vector,
+ * e.g. 768 -> 3072).  For the backward: 0 = generic FMA kernels, 1 = tensor-core
  * backward (row-tile kernels for dX and the middle vector, warp-level MMA for the
  * weight gradients).  Host-only. */
 MONARCH_API int monarch_fwd_path(const monarch_dims* d);

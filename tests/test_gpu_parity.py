@@ -158,14 +158,15 @@ def test_forward_of_identity_is_dense_matrix():
     np.testing.assert_allclose(MT.T, M, rtol=1e-6, atol=1e-6)
 
 
-@pytest.mark.parametrize("rows", [0, 1, 127, 128, 129, 255, 256, 257])
-def test_tc_forward_tile_edges(rows):
-    w = W["n1024_bf16"]
+@pytest.mark.parametrize("name,rows", [("n1024_bf16", r) for r in (0, 1, 127, 128, 129, 255, 256, 257)]
+                         + [("r768x3072_bf16", r) for r in (0, 1, 63, 64, 65, 191, 9473)])
+def test_tc_forward_tile_edges(name, rows):
+    w = W[name]
     shape = synthetic.shape_of(w)
     inp = synthetic.make_inputs(w, seed=8, rows=max(rows, 1))
     d = dev_inputs(inp)
     X = d["X"][:rows].contiguous()
-    Y = torch.full((rows, 1024), float("nan"), dtype=torch.bfloat16, device="cuda")
+    Y = torch.full((rows, w["nb2"] * w["out2"]), float("nan"), dtype=torch.bfloat16, device="cuda")
     bdl.fwd(X, d["R"], d["L"], shape, Y=Y)
     assert bdl.last_device_status() == 0
     if rows:
