@@ -1,17 +1,25 @@
 // Fused Monarch forward for transposed outputs wider than the middle vector
-// (out_transpose = 1, nb2*out2 > nb1*out1, e.g. 768 -> 3072), on tcgen05.
+// (out_transpose = 1, nb2*out2 > nb1*out1 and nb1*in1 <= nb1*out1, e.g. 768 -> 3072), on
+// tcgen05.  One tile of bm <= 64 rows of X per unit, the whole middle vector on chip.
 //
-// One 64-row tile of X per unit, the whole middle vector Z on chip (shared memory).
-//   1. R stage as in the row-tile kernel: M = 64 MMAs, 16 blocks per round, blocks
-//      k0..k0+7 at TMEM lane offset 0 and k0+8..k0+15 at offset 16.
-//   2. Permutation: 16-byte chunks of 8 consecutive k into the swizzled Z tile.
-//   3. L stage in rounds of 8 output columns o: round r issues one M = 64, N = 8 MMA
-//      per block j (and K step), so its result v[j][8r..8r+8) for all j is exactly the
-//      contiguous output run y[r*8*nb2 .. (r+1)*8*nb2) of every row (y[o*nb2 + j]).
-//   4. Each round's run is staged in its own shared-memory buffer and written with
-//      TMA tensor stores of 128-byte row segments while the next round computes.
+//   1. The whole X tile is loaded by TMA straight into the buffer that later holds the
+//      middle tile Z (128B-swizzled 64-column atoms), and all of R into the output
+//      staging area (idle until the L stage), so the R stage has no ring to wait on.
+//      R stage: M = 64 MMAs, blocks k0..k0+7 at TMEM lane offset 0 and k0+8..k0+15 at
+//      lane offset 16.
+//   2. Permutation: the drain warps write 16-byte chunks of 8 consecutive k into Z,
+//      over the (now consumed) X tile.
+//   3. L stage in rounds of 8 output columns o: round r issues one M = 64, N = 8 MMA per
+//      block j, so its result v[j][8r..8r+8) for all j is the contiguous output run
+//      y[r*8*nb2 .. (r+1)*8*nb2) of every row (y[o*nb2 + j]).  The L slices of a round
+//      come through a two-stage ring.
+//   4. Each round's run is staged in one of two shared-memory buffers and written with
+//      TMA tensor stores while the next round computes and drains into the other.
+// bm (rows per unit, a multiple of 8) is chosen on the host so the units spread evenly
+// over the SMs; MMAs always cover 64 rows, and rows >= bm of a tile are never stored.
 // Roles: warp 0 TMA producer (X), warp 1 MMA issuer + TMEM owner, warps 2..9 drain,
-// warps 10..13 factor loaders (cp.async, see tc_rows.cu).  All waits are bounded.
+// warps 10..13 factor loaders (16-byte cp.async, software 32B swizzle).  All waits are
+// bounded (tc_common.cuh).
 #include "tc_common.cuh"
 
 namespace monarch {
@@ -25,52 +33,44 @@ struct WideCfg {
   static constexpr int NB1 = NB1_, IN1 = IN1_, OUT1 = OUT1_, NB2 = NB2_, IN2 = IN2_, OUT2 = OUT2_;
   static constexpr int N_IN = NB1 * IN1, N_MID = NB1 * OUT1, N_OUT = NB2 * OUT2;
   static constexpr int BM = 64;
-  static constexpr int KS1 = IN1 / 16, KS2 = IN2 / 16;
-  static constexpr int NR1 = NB1 / 16;        // R-stage rounds of 16 blocks
-  static constexpr int SLOT1 = 8 * OUT1;      // TMEM columns of one R-stage round
-  static constexpr int S1_COLS = NR1 >= 2 ? 2 * SLOT1 : SLOT1;
+  static constexpr int KS2 = IN2 / 16;
+  static constexpr int SLOT1 = 8 * OUT1;      // TMEM columns of the R stage (16 blocks)
   static constexpr int JH = NB2 / 2;          // blocks j per lane half in an L-stage round
   static constexpr int NR2 = OUT2 / 8;        // L-stage rounds of 8 output columns o
   static constexpr int SLOT2 = 8 * JH;        // TMEM columns of one L-stage round
-  static constexpr int S2_COLS = 2 * SLOT2;
-  static constexpr int MAXC = S1_COLS > S2_COLS ? S1_COLS : S2_COLS;
-  static constexpr int TMEM_COLS = MAXC <= 64 ? 64 : (MAXC <= 128 ? 128 : (MAXC <= 256 ? 256 : 512));
-  static constexpr int NXB = N_IN / 64;
-  static constexpr int BPR = IN1 / 4;         // X boxes per R-stage round
-  static constexpr int XBOX_BYTES = BM * 128;
-  static constexpr int RPIECE = OUT1 * 32;    // R[k] rows x one 16-wide K slice (32B swizzle)
-  static constexpr int STAGE_BYTES = XBOX_BYTES + 4 * RPIECE;
+  static constexpr int MAXC = SLOT1 > 2 * SLOT2 ? SLOT1 : 2 * SLOT2;
+  static constexpr int TMEM_COLS = MAXC <= 128 ? 128 : (MAXC <= 256 ? 256 : 512);
+  static constexpr int NXB = N_IN / 64;       // X boxes (64 columns) per tile
+  static constexpr int ATOM = BM * 128;       // 64 rows x 64 bf16 columns, 128B swizzle
+  static constexpr int RPIECE = OUT1 * 32;    // R[k] rows x one 16-wide K slice, 32B swizzle
+  static constexpr int NRP = N_IN / 16;       // R slices (k, s) = column slice / 16
   static constexpr int LPIECE = 8 * 32;       // 8 rows (o) of L[j] x one 16-wide K slice
-  static constexpr int LPR = NB2 * KS2;       // L slices per L-stage round
-  static constexpr int LPS_MAX = STAGE_BYTES / LPIECE;
-  static constexpr int LPS = LPS_MAX >= LPR ? LPR : (LPS_MAX >= LPR / 2 ? LPR / 2 : (LPS_MAX >= LPR / 3 ? LPR / 3 : LPR / 4));
-  static constexpr int SPR = LPR / LPS;       // ring stages per L-stage round
-  static constexpr int NSTAGE2 = NR2 * SPR;
-  static constexpr int ATOM = BM * 128;
+  static constexpr int LPR = NB2 * KS2;       // L slices per round
+  static constexpr int LSTAGE = LPR * LPIECE;
   static constexpr int ZATOMS = N_MID / 64;
-  static constexpr int OW = 8 * NB2;          // output columns per L-stage round
+  static constexpr int OW = 8 * NB2;          // output columns per round
   static constexpr int OATOMS = OW / 64;
   static constexpr int Z_BYTES = ZATOMS * ATOM, STG_BYTES = OATOMS * ATOM;
-  static constexpr int NSTAGE_RAW = (kSmemBudget - Z_BYTES - STG_BYTES - 1024) / STAGE_BYTES;
-  static constexpr int NSTAGE = NSTAGE_RAW > 8 ? 8 : NSTAGE_RAW;
-  static constexpr int SMEM_BYTES = Z_BYTES + STG_BYTES + NSTAGE * STAGE_BYTES + 1024 + 1024;
+  static constexpr int SMEM_BYTES = Z_BYTES + 2 * STG_BYTES + 2 * LSTAGE + 1024 + 1024;
   static constexpr int P_HALF = OUT1 / 2;
 
-  static_assert(NB1 % 16 == 0 && NR1 <= 2, "R-stage rounds");
-  static_assert(OUT1 % 16 == 0 && S1_COLS <= 512, "R-stage TMEM");
-  static_assert(NB2 % 16 == 0 && OUT2 % 8 == 0, "L-stage rounds");
+  static_assert(NB1 == 16, "one R-stage round of 16 blocks");
+  static_assert(OUT1 % 16 == 0 && SLOT1 <= 512, "R-stage TMEM");
+  static_assert(NB2 % 16 == 0 && OUT2 % 8 == 0 && JH % 8 == 0, "L-stage rounds");
   static_assert(IN1 % 16 == 0 && IN2 % 16 == 0, "K steps of 16");
   static_assert(N_IN % 64 == 0 && N_MID % 64 == 0 && OW % 64 == 0, "64-column atoms");
-  static_assert(NXB == NR1 * BPR, "R-stage rounds align with X boxes");
-  static_assert(LPR % LPS == 0 && LPS * LPIECE <= STAGE_BYTES, "L slices per stage");
+  static_assert(N_IN <= N_MID, "the X tile is loaded into the middle-tile buffer");
+  static_assert(NRP * RPIECE <= 2 * STG_BYTES, "R is parked in the staging buffers");
+  static_assert(NXB <= 16, "X box barriers");
   static_assert(P_HALF % 8 == 0, "drain chunks");
-  static_assert(NSTAGE >= 3, "shared memory");
+  static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
 };
 
 struct WideBars {
-  uint64_t full[8], empty[8];
-  uint64_t a1_full[2], a2_full[2], a2_empty[2];
-  uint64_t z_full, tmem_free, stg_free, staged, mma_done;
+  uint64_t xfull[16];            // X box b and its four R slices (TMA bytes + loader arrivals)
+  uint64_t lfull[2], lempty[2];  // L ring
+  uint64_t a1_full, a2_full[2], a2_empty[2];
+  uint64_t z_full, tmem_free, rfree, stg_free, staged, mma_done;
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -91,29 +91,29 @@ template <class C>
 __global__ void __launch_bounds__(kWideThreads, 1)
     tc_wide_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmY,
                    const __nv_bfloat16* __restrict__ R, const __nv_bfloat16* __restrict__ L,
-                   int64_t rows, int* status) {
+                   int64_t rows, int bm, int* status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  uint8_t* zbuf = smem;
-  uint8_t* stg = smem + C::Z_BYTES;
-  uint8_t* ring = stg + C::STG_BYTES;
-  WideBars* bars = (WideBars*)(ring + C::NSTAGE * C::STAGE_BYTES);
+  uint8_t* zbuf = smem;                    // X tile, then Z tile
+  uint8_t* stg = smem + C::Z_BYTES;        // R during the R stage, then 2 output buffers
+  uint8_t* ring = stg + 2 * C::STG_BYTES;  // 2 L stages
+  WideBars* bars = (WideBars*)(ring + 2 * C::LSTAGE);
   int* abort_flag = &bars->abort_flag;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int64_t nunits = (rows + C::BM - 1) / C::BM;
+  const int64_t nunits = (rows + bm - 1) / bm;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < C::NSTAGE; ++i) {
-      ptx::mbar_init(&bars->full[i], 1 + kWideLoaderThreads);
-      ptx::mbar_init(&bars->empty[i], 1);
-    }
+    for (int i = 0; i < C::NXB; ++i) ptx::mbar_init(&bars->xfull[i], 1 + kWideLoaderThreads);
     for (int i = 0; i < 2; ++i) {
-      ptx::mbar_init(&bars->a1_full[i], 1);
+      ptx::mbar_init(&bars->lfull[i], kWideLoaderThreads);
+      ptx::mbar_init(&bars->lempty[i], 1);
       ptx::mbar_init(&bars->a2_full[i], 1);
       ptx::mbar_init(&bars->a2_empty[i], kWideDrainWarps);
     }
+    ptx::mbar_init(&bars->a1_full, 1);
     ptx::mbar_init(&bars->z_full, kWideDrainWarps);
     ptx::mbar_init(&bars->tmem_free, kWideDrainWarps);
+    ptx::mbar_init(&bars->rfree, 1);
     ptx::mbar_init(&bars->stg_free, 1);
     ptx::mbar_init(&bars->staged, kWideDrainWarps);
     ptx::mbar_init(&bars->mma_done, 1);
@@ -135,89 +135,74 @@ __global__ void __launch_bounds__(kWideThreads, 1)
       ptx::tma_prefetch_desc(&tmX);
       ptx::tma_prefetch_desc(&tmY);
       const uint64_t pol_x = ptx::policy_evict_first();
-      uint32_t it = 0;
-      bool ok = true;
-      for (int64_t u = blockIdx.x; u < nunits && ok; u += gridDim.x) {
-        const int row0 = (int)(u * C::BM);
-        for (int b = 0; b < C::NXB; ++b, ++it) {
-          const int st = it % C::NSTAGE;
-          if (!wait_or_abort(&bars->empty[st], ((it / C::NSTAGE) & 1) ^ 1, abort_flag, status)) { ok = false; break; }
-          ptx::mbar_arrive_expect_tx(&bars->full[st], C::XBOX_BYTES);
-          ptx::tma_load_2d(ring + st * C::STAGE_BYTES, &tmX, &bars->full[st], b * 64, row0, pol_x);
-        }
-        for (int sp = 0; sp < C::NSTAGE2 && ok; ++sp, ++it) {
-          const int st = it % C::NSTAGE;
-          if (!wait_or_abort(&bars->empty[st], ((it / C::NSTAGE) & 1) ^ 1, abort_flag, status)) { ok = false; break; }
-          ptx::mbar_arrive(&bars->full[st]);
+      const uint32_t xbytes = (uint32_t)bm * 128u;
+      uint32_t unit_n = 0;
+      for (int64_t u = blockIdx.x; u < nunits; u += gridDim.x, ++unit_n) {
+        // the previous unit's middle tile must be dead (its last L-stage round drained)
+        if (unit_n > 0 && !wait_or_abort(&bars->tmem_free, (unit_n - 1) & 1, abort_flag, status)) break;
+        const int row0 = (int)(u * bm);
+        for (int b = 0; b < C::NXB; ++b) {
+          ptx::mbar_arrive_expect_tx(&bars->xfull[b], xbytes);
+          ptx::tma_load_2d(zbuf + b * C::ATOM, &tmX, &bars->xfull[b], b * 64, row0, pol_x);
         }
       }
-      const uint32_t issued = it;
-      for (uint32_t k = (issued > (uint32_t)C::NSTAGE ? issued - C::NSTAGE : 0); k < issued; ++k)
-        ptx::mbar_wait_bounded(&bars->full[k % C::NSTAGE], (k / C::NSTAGE) & 1, kWaitLimitNs);
+      // no TMA load may still target this CTA's shared memory at exit
+      if (unit_n > 0)
+        for (int b = 0; b < C::NXB; ++b)
+          ptx::mbar_wait_bounded(&bars->xfull[b], (unit_n - 1) & 1, kWaitLimitNs);
     }
   } else if (warp == 1) {
     // ================================================================ MMA issuer (whole warp)
     constexpr uint32_t idesc1 = make_idesc(C::BM, C::OUT1);
     constexpr uint32_t idesc2 = make_idesc(C::BM, 8);
-    const uint64_t ring_a = make_sdesc(ptx::smem_u32(ring), 1024, 2);
-    const uint64_t ring_b = make_sdesc(ptx::smem_u32(ring), 256, 6);
     const uint64_t z_a = make_sdesc(ptx::smem_u32(zbuf), 1024, 2);
-    uint32_t it = 0, rnd2 = 0, unit_n = 0;
+    const uint64_t r_b = make_sdesc(ptx::smem_u32(stg), 256, 6);
+    const uint64_t ring_b = make_sdesc(ptx::smem_u32(ring), 256, 6);
+    uint32_t g2 = 0, unit_n = 0;
     bool ok = true;
     for (int64_t u = blockIdx.x; u < nunits && ok; u += gridDim.x, ++unit_n) {
       // TMEM is shared by both stages: the previous unit's L-stage rounds must be drained
       if (unit_n > 0 && !warp_wait_or_abort(lane, &bars->tmem_free, (unit_n - 1) & 1, abort_flag, status)) { ok = false; break; }
       ptx::tc_fence_after();
-      for (int r1 = 0; r1 < C::NR1 && ok; ++r1) {
-        const uint32_t dslot = tmem + (uint32_t)(r1 * C::SLOT1);
-        for (int bb = 0; bb < C::BPR; ++bb, ++it) {
-          const int st = it % C::NSTAGE;
-          if (!warp_wait_or_abort(lane, &bars->full[st], (it / C::NSTAGE) & 1, abort_flag, status)) { ok = false; break; }
-          ptx::fence_proxy_async_smem();
-          ptx::tc_fence_after();
-          const uint64_t soff = (uint64_t)((st * C::STAGE_BYTES) >> 4);
+      // ---- R stage: X box b holds columns [64 b, 64 b + 64) = R slices 4 b .. 4 b + 3
+      for (int b = 0; b < C::NXB; ++b) {
+        if (!warp_wait_or_abort(lane, &bars->xfull[b], unit_n & 1, abort_flag, status)) { ok = false; break; }
+        ptx::fence_proxy_async_smem();  // R slices were written by cp.async (generic proxy)
+        ptx::tc_fence_after();
 #pragma unroll
-          for (int t = 0; t < 4; ++t) {
-            const int c = bb * 64 + 16 * t;
-            const int kk = c / C::IN1, s16 = (c % C::IN1) / 16;
-            const uint32_t d = dslot + ((uint32_t)(kk >> 3) << 20) + (uint32_t)((kk & 7) * C::OUT1);
-            ptx::mma_bf16_ss_elect(d, ring_a + soff + (uint64_t)((32 * t) >> 4),
-                                   ring_b + soff + (uint64_t)((C::XBOX_BYTES + t * C::RPIECE) >> 4),
-                                   idesc1, s16 > 0 ? 1u : 0u);
-          }
-          ptx::mma_commit_elect(&bars->empty[st]);
+        for (int t = 0; t < 4; ++t) {
+          const int c = b * 64 + 16 * t;
+          const int kk = c / C::IN1, s16 = (c % C::IN1) / 16;
+          const uint32_t d = tmem + ((uint32_t)(kk >> 3) << 20) + (uint32_t)((kk & 7) * C::OUT1);
+          ptx::mma_bf16_ss_elect(d, z_a + (uint64_t)((b * C::ATOM + 32 * t) >> 4),
+                                 r_b + (uint64_t)(((4 * b + t) * C::RPIECE) >> 4), idesc1,
+                                 s16 > 0 ? 1u : 0u);
         }
-        if (!ok) break;
-        ptx::mma_commit_elect(&bars->a1_full[r1]);
       }
       if (!ok) break;
+      ptx::mma_commit_elect(&bars->a1_full);
       if (!warp_wait_or_abort(lane, &bars->z_full, unit_n & 1, abort_flag, status)) { ok = false; break; }
       ptx::tc_fence_after();
-      for (int r2 = 0; r2 < C::NR2 && ok; ++r2, ++rnd2) {
-        const int slot = rnd2 & 1;
-        if (!warp_wait_or_abort(lane, &bars->a2_empty[slot], ((rnd2 >> 1) & 1) ^ 1, abort_flag, status)) { ok = false; break; }
+      // ---- L stage
+      for (int r2 = 0; r2 < C::NR2 && ok; ++r2, ++g2) {
+        const int slot = g2 & 1;
+        if (!warp_wait_or_abort(lane, &bars->a2_empty[slot], ((g2 >> 1) & 1) ^ 1, abort_flag, status)) { ok = false; break; }
+        if (!warp_wait_or_abort(lane, &bars->lfull[slot], (g2 >> 1) & 1, abort_flag, status)) { ok = false; break; }
+        ptx::fence_proxy_async_smem();
         ptx::tc_fence_after();
         const uint32_t dslot = tmem + (uint32_t)(slot * C::SLOT2);
-        for (int sp = 0; sp < C::SPR; ++sp, ++it) {
-          const int st = it % C::NSTAGE;
-          if (!warp_wait_or_abort(lane, &bars->full[st], (it / C::NSTAGE) & 1, abort_flag, status)) { ok = false; break; }
-          ptx::fence_proxy_async_smem();
-          ptx::tc_fence_after();
-          const uint64_t soff = (uint64_t)((st * C::STAGE_BYTES) >> 4);
+        const uint64_t lb = ring_b + (uint64_t)((slot * C::LSTAGE) >> 4);
 #pragma unroll 4
-          for (int t = 0; t < C::LPS; ++t) {
-            const int piece = sp * C::LPS + t;  // within the round: j * KS2 + s
-            const int j = piece / C::KS2, s16 = piece % C::KS2;
-            const int h = j / C::JH, jj = j % C::JH;
-            const int zc = j * C::IN2 + 16 * s16;
-            const uint32_t d = dslot + ((uint32_t)h << 20) + (uint32_t)(jj * 8);
-            ptx::mma_bf16_ss_elect(d, z_a + (uint64_t)(((zc >> 6) * C::ATOM + (zc & 63) * 2) >> 4),
-                                   ring_b + soff + (uint64_t)((t * C::LPIECE) >> 4), idesc2,
-                                   s16 > 0 ? 1u : 0u);
-          }
-          ptx::mma_commit_elect(&bars->empty[st]);
+        for (int piece = 0; piece < C::LPR; ++piece) {  // piece = j * KS2 + s
+          const int j = piece / C::KS2, s16 = piece % C::KS2;
+          const int h = j / C::JH, jj = j % C::JH;
+          const int zc = j * C::IN2 + 16 * s16;
+          const uint32_t d = dslot + ((uint32_t)h << 20) + (uint32_t)(jj * 8);
+          ptx::mma_bf16_ss_elect(d, z_a + (uint64_t)(((zc >> 6) * C::ATOM + (zc & 63) * 2) >> 4),
+                                 lb + (uint64_t)((piece * C::LPIECE) >> 4), idesc2,
+                                 s16 > 0 ? 1u : 0u);
         }
-        if (!ok) break;
+        ptx::mma_commit_elect(&bars->lempty[slot]);
         ptx::mma_commit_elect(&bars->a2_full[slot]);
       }
     }
@@ -226,38 +211,40 @@ __global__ void __launch_bounds__(kWideThreads, 1)
     __syncwarp();
   } else if (warp >= 2 + kWideDrainWarps) {
     // ================================================================ factor loaders
+    // R slice pi = (k, s) (k = pi / (in1/16)) lands at stg + pi * RPIECE: row n of R[k] at
+    // n * 32, its two 16-byte chunks swapped when (n >> 2) is odd (32B swizzle).
+    // L round r2: slice j lands at stage + j * LPIECE, rows o = 8 r2 .. 8 r2 + 7.
     const int lt = (warp - 2 - kWideDrainWarps) * 32 + lane;
-    const uint32_t ring_s = ptx::smem_u32(ring);
-    uint32_t it = 0;
+    const uint32_t stg_s = ptx::smem_u32(stg), ring_s = ptx::smem_u32(ring);
+    uint32_t g2 = 0, unit_n = 0;
     bool ok = true;
-    for (int64_t u = blockIdx.x; u < nunits && ok; u += gridDim.x) {
-      for (int sq = 0; sq < C::NXB + C::NSTAGE2 && ok; ++sq, ++it) {
-        const int st = it % C::NSTAGE;
-        if (!wait_or_abort(&bars->empty[st], ((it / C::NSTAGE) & 1) ^ 1, abort_flag, status)) { ok = false; break; }
-        const uint32_t sb = ring_s + st * C::STAGE_BYTES;
-        if (sq < C::NXB) {
-          const int b = sq;
-          for (int g = lt; g < 4 * C::OUT1 * 2; g += kWideLoaderThreads) {
-            const int t = g / (C::OUT1 * 2), n = (g >> 1) % C::OUT1, c = g & 1;
-            const int col = b * 64 + t * 16;
-            const int k = col / C::IN1, s16 = col % C::IN1;
-            ptx::cp_async_16(sb + C::XBOX_BYTES + t * C::RPIECE + n * 32 + ((c ^ ((n >> 2) & 1)) << 4),
-                             R + ((int64_t)k * C::OUT1 + n) * C::IN1 + s16 + c * 8);
-          }
-        } else {
-          const int q = sq - C::NXB;
-          const int r2 = q / C::SPR, sp = q % C::SPR;
-          for (int g = lt; g < C::LPS * 16; g += kWideLoaderThreads) {  // 8 rows x 2 chunks per slice
-            const int t = g / 16, n = (g >> 1) & 7, c = g & 1;
-            const int piece = sp * C::LPS + t, j = piece / C::KS2, s16 = (piece % C::KS2) * 16;
-            ptx::cp_async_16(sb + t * C::LPIECE + n * 32 + ((c ^ ((n >> 2) & 1)) << 4),
-                             L + ((int64_t)j * C::OUT2 + r2 * 8 + n) * C::IN2 + s16 + c * 8);
-          }
+    for (int64_t u = blockIdx.x; u < nunits && ok; u += gridDim.x, ++unit_n) {
+      // R is parked in the staging buffers: the previous unit's stores must have read them
+      if (unit_n > 0 && !wait_or_abort(&bars->rfree, (unit_n - 1) & 1, abort_flag, status)) { ok = false; break; }
+      for (int b = 0; b < C::NXB; ++b) {
+        for (int g = lt; g < 4 * C::OUT1 * 2; g += kWideLoaderThreads) {
+          const int t = g / (C::OUT1 * 2), n = (g >> 1) % C::OUT1, c = g & 1;
+          const int pi = 4 * b + t;
+          const int col = pi * 16, k = col / C::IN1, s16 = col % C::IN1;
+          ptx::cp_async_16(stg_s + pi * C::RPIECE + n * 32 + ((c ^ ((n >> 2) & 1)) << 4),
+                           R + ((int64_t)k * C::OUT1 + n) * C::IN1 + s16 + c * 8);
         }
-        ptx::cp_async_mbar_arrive_noinc(&bars->full[st]);
+        ptx::cp_async_mbar_arrive_noinc(&bars->xfull[b]);
+      }
+      for (int r2 = 0; r2 < C::NR2; ++r2, ++g2) {
+        const int slot = g2 & 1;
+        if (!wait_or_abort(&bars->lempty[slot], ((g2 >> 1) & 1) ^ 1, abort_flag, status)) { ok = false; break; }
+        const uint32_t sb = ring_s + slot * C::LSTAGE;
+        for (int g = lt; g < C::LPR * 16; g += kWideLoaderThreads) {  // 8 rows x 2 chunks per slice
+          const int piece = g / 16, n = (g >> 1) & 7, c = g & 1;
+          const int j = piece / C::KS2, s16 = (piece % C::KS2) * 16;
+          ptx::cp_async_16(sb + piece * C::LPIECE + n * 32 + ((c ^ ((n >> 2) & 1)) << 4),
+                           L + ((int64_t)j * C::OUT2 + r2 * 8 + n) * C::IN2 + s16 + c * 8);
+        }
+        ptx::cp_async_mbar_arrive_noinc(&bars->lfull[slot]);
       }
     }
-    ptx::cp_async_wait<0>();
+    ptx::cp_async_wait<0>();  // no copy may still target this CTA's shared memory at exit
   } else {
     // ================================================================ drain (8 warps)
     const int quad = warp & 3, ph = (warp - 2) >> 2, half = lane >> 4;
@@ -265,52 +252,51 @@ __global__ void __launch_bounds__(kWideThreads, 1)
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
     const uint32_t z_s = ptx::smem_u32(zbuf), stg_s = ptx::smem_u32(stg);
     const bool leader = (warp == 2 && lane == 0);
-    uint32_t rnd2 = 0, unit_n = 0;
+    uint32_t g2 = 0, unit_n = 0;
     bool ok = true;
     for (int64_t u = blockIdx.x; u < nunits && ok; u += gridDim.x, ++unit_n) {
-      for (int r1 = 0; r1 < C::NR1 && ok; ++r1) {
-        if (!wait_or_abort(&bars->a1_full[r1], unit_n & 1, abort_flag, status)) { ok = false; break; }
-        __syncwarp();  // the leader lane may still be coming out of the previous unit's store branch
-        ptx::tc_fence_after();
-        const uint32_t tb = tmem + lane_off + (uint32_t)(r1 * C::SLOT1);
+      // ---- R stage -> Z (over the consumed X tile)
+      if (!wait_or_abort(&bars->a1_full, unit_n & 1, abort_flag, status)) { ok = false; break; }
+      __syncwarp();  // the leader lane may still be coming out of the previous unit's store branch
+      ptx::tc_fence_after();
 #pragma unroll 1
-        for (int pc = ph * C::P_HALF; pc < (ph + 1) * C::P_HALF; pc += 8) {
-          float v[8][8];
+      for (int pc = ph * C::P_HALF; pc < (ph + 1) * C::P_HALF; pc += 8) {
+        float v[8][8];
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            uint32_t rr[8];
-            ptx::tmem_ld8(tb + kk * C::OUT1 + pc, rr);
+        for (int kk = 0; kk < 8; ++kk) {
+          uint32_t rr[8];
+          ptx::tmem_ld8(tmem + lane_off + kk * C::OUT1 + pc, rr);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) v[kk][e] = __uint_as_float(rr[e]);
-          }
-          ptx::tmem_wait_ld();
+          for (int e = 0; e < 8; ++e) v[kk][e] = __uint_as_float(rr[e]);
+        }
+        ptx::tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const int t0 = (pc + e) * C::NB1 + r1 * 16 + half * 8;
-            ptx::st_shared_v4(z_s + wide_chunk_off(r, t0), ptx::pack_bf16x2(v[0][e], v[1][e]),
-                              ptx::pack_bf16x2(v[2][e], v[3][e]), ptx::pack_bf16x2(v[4][e], v[5][e]),
-                              ptx::pack_bf16x2(v[6][e], v[7][e]));
-          }
+        for (int e = 0; e < 8; ++e) {
+          const int t0 = (pc + e) * C::NB1 + half * 8;  // flat column p*nb1 + k, k = 8 half ..
+          ptx::st_shared_v4(z_s + wide_chunk_off(r, t0), ptx::pack_bf16x2(v[0][e], v[1][e]),
+                            ptx::pack_bf16x2(v[2][e], v[3][e]), ptx::pack_bf16x2(v[4][e], v[5][e]),
+                            ptx::pack_bf16x2(v[6][e], v[7][e]));
         }
       }
-      if (!ok) break;
       ptx::tc_fence_before();
       ptx::fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(&bars->z_full);
-      const int row0 = (int)(u * C::BM);
-      for (int r2 = 0; r2 < C::NR2 && ok; ++r2, ++rnd2) {
-        const int slot = rnd2 & 1;
-        if (!wait_or_abort(&bars->a2_full[slot], (rnd2 >> 1) & 1, abort_flag, status)) { ok = false; break; }
-        // the staging buffer must have been read out by the previous round's stores
+      const int row0 = (int)(u * bm);
+      // ---- L-stage rounds -> staged output runs
+      for (int r2 = 0; r2 < C::NR2 && ok; ++r2, ++g2) {
+        const int slot = g2 & 1;
+        if (!wait_or_abort(&bars->a2_full[slot], (g2 >> 1) & 1, abort_flag, status)) { ok = false; break; }
+        // staging buffer `slot` was last used two rounds ago; its stores must have read it
         if (leader) {
-          ptx::bulk_wait_read_all();
+          ptx::bulk_wait_read_allbut1();
           ptx::mbar_arrive(&bars->stg_free);
         }
-        if (!wait_or_abort(&bars->stg_free, rnd2 & 1, abort_flag, status)) { ok = false; break; }
+        if (!wait_or_abort(&bars->stg_free, g2 & 1, abort_flag, status)) { ok = false; break; }
         __syncwarp();  // tcgen05.ld is warp-collective
         ptx::tc_fence_after();
         const uint32_t tb = tmem + lane_off + (uint32_t)(slot * C::SLOT2);
+        const uint32_t sb = stg_s + (uint32_t)(slot * C::STG_BYTES);
 #pragma unroll 1
         for (int jc = 0; jc < C::JH / 8; ++jc) {
           float v[8][4];
@@ -325,7 +311,7 @@ __global__ void __launch_bounds__(kWideThreads, 1)
 #pragma unroll
           for (int e = 0; e < 4; ++e) {  // local column (o - 8 r2) * nb2 + j, 8 consecutive j
             const int lc = (4 * ph + e) * C::NB2 + half * C::JH + jc * 8;
-            ptx::st_shared_v4(stg_s + wide_chunk_off(r, lc), ptx::pack_bf16x2(v[0][e], v[1][e]),
+            ptx::st_shared_v4(sb + wide_chunk_off(r, lc), ptx::pack_bf16x2(v[0][e], v[1][e]),
                               ptx::pack_bf16x2(v[2][e], v[3][e]), ptx::pack_bf16x2(v[4][e], v[5][e]),
                               ptx::pack_bf16x2(v[6][e], v[7][e]));
           }
@@ -338,17 +324,23 @@ __global__ void __launch_bounds__(kWideThreads, 1)
           ptx::mbar_arrive(&bars->staged);
         }
         if (leader) {
-          if (!wait_or_abort(&bars->staged, rnd2 & 1, abort_flag, status)) {
+          if (!wait_or_abort(&bars->staged, g2 & 1, abort_flag, status)) {
             ok = false;
           } else {
             for (int a = 0; a < C::OATOMS; ++a)
-              ptx::tma_store_2d(&tmY, stg + a * C::ATOM, r2 * C::OW + a * 64, row0);
+              ptx::tma_store_2d(&tmY, stg + slot * C::STG_BYTES + a * C::ATOM, r2 * C::OW + a * 64, row0);
             ptx::bulk_commit_group();
           }
         }
       }
+      if (!ok) break;
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(&bars->tmem_free);
+      if (leader) {
+        // the staging buffers take the next unit's R once these stores have read them
+        ptx::bulk_wait_read_all();
+        ptx::mbar_arrive(&bars->rfree);
+      }
     }
     if (leader) ptx::bulk_wait_all();
   }
@@ -359,22 +351,35 @@ __global__ void __launch_bounds__(kWideThreads, 1)
   if (warp == 1) ptx::tmem_dealloc(tmem, C::TMEM_COLS);
 }
 
+// Rows per unit: a multiple of 8, at most 64, chosen so the units fill the SMs in as few
+// equal waves as possible (e.g. 8192 rows on 148 SMs: 56-row tiles, 147 units).
+static int balanced_bm(int64_t rows, int nsm) {
+  const int64_t per_wave = (int64_t)64 * nsm;
+  const int64_t waves = (rows + per_wave - 1) / per_wave;
+  const int64_t per_unit = (rows + waves * nsm - 1) / (waves * nsm);
+  int64_t bm = (per_unit + 7) / 8 * 8;
+  if (bm > 64) bm = 64;
+  if (bm < 8) bm = 8;
+  return (int)bm;
+}
+
 template <class C>
 static cudaError_t launch_wide(const void* X, const void* R, const void* L, void* Y, int64_t rows,
                                int* status, cudaStream_t st) {
   if (rows == 0) return cudaSuccess;
+  const int nsm = num_sms();
+  const int bm = balanced_bm(rows, nsm);
   CUtensorMap mX, mY;
-  if (!make_map_2d(&mX, X, C::N_IN, (uint64_t)rows, 64, C::BM, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_map_2d(&mY, Y, C::N_OUT, (uint64_t)rows, 64, C::BM, CU_TENSOR_MAP_SWIZZLE_128B))
+  if (!make_map_2d(&mX, X, C::N_IN, (uint64_t)rows, 64, (uint32_t)bm, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map_2d(&mY, Y, C::N_OUT, (uint64_t)rows, 64, (uint32_t)bm, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(tc_wide_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        C::SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  const int64_t nunits = (rows + C::BM - 1) / C::BM;
-  int64_t grid = num_sms();
-  if (grid > nunits) grid = nunits;
+  const int64_t nunits = (rows + bm - 1) / bm;
+  const int64_t grid = nunits < nsm ? nunits : nsm;
   tc_wide_kernel<C><<<(unsigned)grid, kWideThreads, C::SMEM_BYTES, st>>>(
-      mX, mY, (const __nv_bfloat16*)R, (const __nv_bfloat16*)L, rows, status);
+      mX, mY, (const __nv_bfloat16*)R, (const __nv_bfloat16*)L, rows, bm, status);
   return cudaGetLastError();
 }
 
