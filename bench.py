@@ -392,7 +392,8 @@ def main():
     fpath = bdl.fwd_path(shape, w["dtype"])
     fwd_tc = fpath >= 1
     bpath = bdl.bwd_path(shape, w["dtype"])
-    launches_per_step = (1 if do_fwd else 0) + ((6 if bpath == 1 else 3) if do_bwd else 0)
+    fwd_launches = (3 + int(shape.get("out_transpose", 1))) if fpath == 4 else 1
+    launches_per_step = (fwd_launches if do_fwd else 0) + ((6 if bpath == 1 else 3) if do_bwd else 0)
     # Roofline object: the forward kernel (one launch per forward pass, so the pass time
     # measured by the events is that kernel's launch duration).  The row-tile kernel
     # family is also the largest share of the step in the ncu launch list.  When only
@@ -401,9 +402,10 @@ def main():
     a = alg[dom]
     t_dom = fwd_avg_s if dom == "fwd" else bwd_avg_s
     bound = passes[dom]["bound"]
-    kname = ({2: "tc_rows_kernel", 3: "tc_wide_kernel", 1: "tc_fwd_kernel"}.get(fpath, "gen_fwd_kernel")
+    kname = ({2: "tc_rows_kernel", 3: "tc_wide_kernel", 4: "tc_bdgemm_kernel + permute_rows_kernel (pass of 4 kernels)",
+              1: "tc_fwd_kernel"}.get(fpath, "gen_fwd_kernel")
              if dom == "fwd" else "monarch_bwd")
-    srcs = ["block_diagonal_linear_b200/csrc/%s.cu" % {2: "tc_rows", 3: "tc_wide", 1: "tc_fwd"}.get(fpath, "generic"),
+    srcs = ["block_diagonal_linear_b200/csrc/%s.cu" % {2: "tc_rows", 3: "tc_wide", 4: "tc_split", 1: "tc_fwd"}.get(fpath, "generic"),
             "block_diagonal_linear_b200/csrc/ptx.cuh", "block_diagonal_linear_b200/csrc/tc_common.cuh"]
     if bound == "hbm":
         roof = {"bound": "hbm", "achieved": a["bytes"] / t_dom / 1e9, "peak": peaks["hbm_gbs"],

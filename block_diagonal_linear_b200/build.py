@@ -12,7 +12,7 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libmonarch.so")
-SOURCES = ["api.cu", "generic.cu", "tc_fwd.cu", "tc_rows.cu", "tc_wide.cu", "bwd_fast.cu", "noalloc.cu"]
+SOURCES = ["api.cu", "generic.cu", "tc_fwd.cu", "tc_rows.cu", "tc_wide.cu", "tc_split.cu", "bwd_fast.cu", "noalloc.cu"]
 HEADERS = ["common.cuh", "ptx.cuh", "tc_common.cuh"]
 
 NVCC_FLAGS = [

@@ -63,11 +63,13 @@ cudaError_t debug_wait_timeout(uint64_t timeout_ns, int* status, cudaStream_t st
 }
 
 // 0 = generic FMA kernels, 1 = tcgen05 group kernel, 2 = tcgen05 row-tile kernel,
-// 3 = tcgen05 row-tile kernel with the L stage in rounds of output columns.
+// 3 = tcgen05 row-tile kernel with the L stage in rounds of output columns,
+// 4 = tcgen05 block-diagonal GEMMs and row permutations as separate passes over Y.
 static int fwd_path(const Shape& s, int dtype) {
   if (dtype != MONARCH_BF16) return 0;
   if (tc_rows_supported(s)) return 2;
   if (tc_wide_supported(s)) return 3;
+  if (tc_split_supported(s)) return 4;
   if (tc_fwd_supported(s)) return 1;
   return 0;
 }
@@ -113,6 +115,7 @@ int monarch_fwd(const void* X, const void* R, const void* L, const monarch_dims*
     if (status == nullptr) return MONARCH_ERR_CUDA;
     e = path == 2   ? tc_rows_fwd(X, R, L, Y, s, status, st)
         : path == 3 ? tc_wide_fwd(X, R, L, Y, s, status, st)
+        : path == 4 ? tc_split_fwd(X, R, L, Y, s, status, st)
                     : tc_fwd(X, R, L, Y, s, status, st);
   } else {
     if (!generic_fwd_supported(s)) return MONARCH_ERR_UNSUPPORTED;

@@ -12,7 +12,7 @@
 // too small for a 64/128-row tcgen05 tile without wasting half of it, so they use
 // warp-level mma.sync (m16n8k16, bf16 -> fp32) with ldmatrix.trans operand loads.
 #include "common.cuh"
-#include "ptx.cuh"
+#include "tc_common.cuh"
 
 namespace monarch {
 
@@ -26,6 +26,8 @@ __global__ void transpose_factors_kernel(const __nv_bfloat16* __restrict__ R,
                                          const __nv_bfloat16* __restrict__ L,
                                          __nv_bfloat16* __restrict__ Rt,
                                          __nv_bfloat16* __restrict__ Lt, Shape s) {
+  ptx::griddep_wait();  // Rt, Lt may still be read by the previous backward's kernels
+  ptx::griddep_launch_dependents();
   const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   const int64_t nR = s.n_R(), nL = s.n_L();
   if (e < nR) {  // Rt[k][i][p] = R[k][p][i]
@@ -48,6 +50,8 @@ constexpr int kGatherWarps = 8;
 __global__ void __launch_bounds__(kGatherWarps * 32)
     gather_dv_kernel(const __nv_bfloat16* __restrict__ dY, __nv_bfloat16* __restrict__ dV, Shape s) {
   extern __shared__ __align__(16) uint32_t shw[];
+  ptx::griddep_wait();
+  ptx::griddep_launch_dependents();
   const int n = (int)s.n_out(), nb2 = s.nb2, out2 = s.out2;
   const int pitch = nb2 + 2;          // elements per staged grid row (o)
   const int wpitch = pitch / 2;       // 32-bit words per staged grid row
@@ -113,6 +117,8 @@ __global__ void __launch_bounds__(256, 1)
   constexpr int TILE = kWgChunk * PITCH;
   constexpr int MT = BS / 16, NT = BS / 8;
   extern __shared__ __align__(128) uint8_t smem[];
+  ptx::griddep_wait();
+  ptx::griddep_launch_dependents();
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int g = blockIdx.y;
   const bool is_l = g < ngroups_l;  // job: dL (A = dV, B = Z) or dR (A = dU, B = X)
@@ -206,6 +212,8 @@ __global__ void __launch_bounds__(256, 1)
 __global__ void reduce_partials_kernel(const float* __restrict__ partial, __nv_bfloat16* __restrict__ dR,
                                        __nv_bfloat16* __restrict__ dL, int64_t nR, int64_t nP,
                                        int nsplit) {
+  ptx::griddep_wait();
+  ptx::griddep_launch_dependents();
   const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (e >= nP) return;
   float acc = 0.f;
@@ -267,14 +275,18 @@ cudaError_t fast_bwd(const void* dY, const void* X, const void* R, const void* L
   float* part = (float*)(base + w.part);
   const int64_t nR = s.n_R(), nP = s.n_R() + s.n_L();
   cudaError_t e;
-  transpose_factors_kernel<<<(unsigned)((nP + 255) / 256), 256, 0, st>>>(
-      (const __nv_bfloat16*)R, (const __nv_bfloat16*)L, Rt, Lt, s);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  // All six launches use programmatic dependent launch: each kernel waits for the previous
+  // grid of the stream (griddep_wait) before touching its data, so the next launch and its
+  // prologue overlap the tail of the current one.
+  if ((e = launch_kernel(transpose_factors_kernel, dim3((unsigned)((nP + 255) / 256)), dim3(256), 0, st,
+                         true, (const __nv_bfloat16*)R, (const __nv_bfloat16*)L, Rt, Lt, s)) != cudaSuccess)
+    return e;
   const int nsplit = wg_nsplit(s);
   if (s.rows > 0) {
     const size_t gsm = (size_t)kGatherWarps * (size_t)s.out2 * (size_t)(s.nb2 + 2) * 2;
-    gather_dv_kernel<<<2 * 148, kGatherWarps * 32, gsm, st>>>((const __nv_bfloat16*)dY, dV, s);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if ((e = launch_kernel(gather_dv_kernel, dim3(2 * 148), dim3(kGatherWarps * 32), gsm, st, true,
+                           (const __nv_bfloat16*)dY, dV, s)) != cudaSuccess)
+      return e;
     if ((e = tc_rows_middle(X, R, Z, s, status, st)) != cudaSuccess) return e;
     if ((e = tc_rows_dual(dV, Lt, Rt, dX, dU, s, status, st)) != cudaSuccess) return e;
   }
@@ -286,20 +298,21 @@ cudaError_t fast_bwd(const void* dY, const void* X, const void* R, const void* L
     if ((e = cudaFuncSetAttribute(wgrad_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   smem)) != cudaSuccess)
       return e;
-    wgrad_kernel<32><<<grid, 256, smem, st>>>(dV, Z, dU, (const __nv_bfloat16*)X, ngl, s.rows,
-                                              nsplit, part, nR, nP, ncols);
+    e = launch_kernel(wgrad_kernel<32>, grid, dim3(256), smem, st, true, (const __nv_bfloat16*)dV,
+                      (const __nv_bfloat16*)Z, (const __nv_bfloat16*)dU, (const __nv_bfloat16*)X, ngl,
+                      s.rows, nsplit, part, nR, nP, ncols);
   } else {
     constexpr int smem = 2 * 2 * kWgChunk * (8 * 16 * 2 + 16);
     if ((e = cudaFuncSetAttribute(wgrad_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   smem)) != cudaSuccess)
       return e;
-    wgrad_kernel<16><<<grid, 256, smem, st>>>(dV, Z, dU, (const __nv_bfloat16*)X, ngl, s.rows,
-                                              nsplit, part, nR, nP, ncols);
+    e = launch_kernel(wgrad_kernel<16>, grid, dim3(256), smem, st, true, (const __nv_bfloat16*)dV,
+                      (const __nv_bfloat16*)Z, (const __nv_bfloat16*)dU, (const __nv_bfloat16*)X, ngl,
+                      s.rows, nsplit, part, nR, nP, ncols);
   }
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  reduce_partials_kernel<<<(unsigned)((nP + 255) / 256), 256, 0, st>>>(
-      part, (__nv_bfloat16*)dR, (__nv_bfloat16*)dL, nR, nP, nsplit);
-  return cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  return launch_kernel(reduce_partials_kernel, dim3((unsigned)((nP + 255) / 256)), dim3(256), 0, st, true,
+                       (const float*)part, (__nv_bfloat16*)dR, (__nv_bfloat16*)dL, nR, nP, nsplit);
 }
 
 }  // namespace monarch

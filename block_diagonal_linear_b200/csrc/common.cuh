@@ -74,6 +74,12 @@ bool tc_wide_supported(const Shape& s);
 cudaError_t tc_wide_fwd(const void* X, const void* R, const void* L, void* Y, const Shape& s,
                         int* status, cudaStream_t st);
 
+// Large square blocks (64 x 64, nb1 = nb2): block-diagonal tcgen05 GEMMs and row permutations
+// as four passes over Y (no scratch).
+bool tc_split_supported(const Shape& s);
+cudaError_t tc_split_fwd(const void* X, const void* R, const void* L, void* Y, const Shape& s,
+                         int* status, cudaStream_t st);
+
 // Tensor-core backward of the square small-block shapes (bf16).
 bool fast_bwd_supported(const Shape& s);
 size_t fast_bwd_workspace(const Shape& s);

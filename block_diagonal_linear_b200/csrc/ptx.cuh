@@ -64,6 +64,17 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
   }
 }
 
+// ---------------------------------------------------------------- programmatic dependent launch
+// Wait until the grids this grid depends on (the previous kernels of the stream, when this one
+// was launched with programmatic stream serialization) have completed and their memory
+// operations are visible.  Returns at once for a kernel launched without that attribute.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// Let the next grid of the stream begin launching (it still waits for this grid's completion
+// in its own griddep_wait before touching memory this grid writes).
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- fences
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");

@@ -90,6 +90,25 @@ inline bool make_map_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Launch `kernel` on `st`; with pdl = true it may begin launching while the previous kernel of
+// the stream is still running (programmatic stream serialization).  Every kernel launched this
+// way calls ptx::griddep_wait() before it touches global memory that earlier kernels write.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_kernel(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                                 cudaStream_t st, bool pdl, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kernel, ((KArgs)args)...);
+}
+
 inline int num_sms() {
   static int n = 0;
   if (n == 0) {

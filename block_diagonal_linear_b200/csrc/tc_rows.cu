@@ -137,6 +137,10 @@ __global__ void __launch_bounds__(kRowsThreads, 1)
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
+  // launched with programmatic stream serialization inside the backward: the inputs are
+  // written by the previous kernels of the stream
+  ptx::griddep_wait();
+  ptx::griddep_launch_dependents();
 
   if (warp == 0) {
     // ================================================================ TMA producer (X)
@@ -429,7 +433,7 @@ __global__ void __launch_bounds__(kRowsThreads, 1)
 // (MODE 0/1); Zout (rows, N_MID) middle tile (MODE 1/2).
 template <class C>
 static cudaError_t launch_rows(const void* X, const void* W1, const void* W2, void* Y, void* Zout,
-                               int64_t rows, int* status, cudaStream_t st) {
+                               int64_t rows, int* status, cudaStream_t st, bool pdl = false) {
   if (rows == 0) return cudaSuccess;
   CUtensorMap mX, mY, mZ;
   if (!make_map_2d(&mX, X, C::N_IN, (uint64_t)rows, 64, C::BM, CU_TENSOR_MAP_SWIZZLE_128B))
@@ -448,9 +452,8 @@ static cudaError_t launch_rows(const void* X, const void* W1, const void* W2, vo
   const int64_t nunits = (rows + C::BM - 1) / C::BM;
   int64_t grid = num_sms();
   if (grid > nunits) grid = nunits;
-  tc_rows_kernel<C><<<(unsigned)grid, kRowsThreads, C::SMEM_BYTES, st>>>(
-      mX, mY, mZ, (const __nv_bfloat16*)W1, (const __nv_bfloat16*)W2, rows, status);
-  return cudaGetLastError();
+  return launch_kernel(tc_rows_kernel<C>, dim3((unsigned)grid), dim3(kRowsThreads), C::SMEM_BYTES, st,
+                       pdl, mX, mY, mZ, (const __nv_bfloat16*)W1, (const __nv_bfloat16*)W2, rows, status);
 }
 
 using RowsSq16 = RowsCfg<16, 16, 16, 16, 16, 16, 1>;  // n = 256 = 16^2
@@ -484,16 +487,16 @@ cudaError_t tc_rows_fwd(const void* X, const void* R, const void* L, void* Y, co
 // Z = P R x for every row (block-contiguous middle vector, bf16).
 cudaError_t tc_rows_middle(const void* X, const void* R, void* Z, const Shape& s, int* status,
                            cudaStream_t st) {
-  if (rows_shape_is<RowsSq16>(s)) return launch_rows<RowsSq16Z>(X, R, nullptr, nullptr, Z, s.rows, status, st);
-  if (rows_shape_is<RowsSq32>(s)) return launch_rows<RowsSq32Z>(X, R, nullptr, nullptr, Z, s.rows, status, st);
+  if (rows_shape_is<RowsSq16>(s)) return launch_rows<RowsSq16Z>(X, R, nullptr, nullptr, Z, s.rows, status, st, true);
+  if (rows_shape_is<RowsSq32>(s)) return launch_rows<RowsSq32Z>(X, R, nullptr, nullptr, Z, s.rows, status, st, true);
   return cudaErrorNotSupported;
 }
 
 // dX and dU from the block-contiguous dV with the transposed factors Lt, Rt.
 cudaError_t tc_rows_dual(const void* dV, const void* Lt, const void* Rt, void* dX, void* dU,
                          const Shape& s, int* status, cudaStream_t st) {
-  if (rows_shape_is<RowsSq16>(s)) return launch_rows<RowsSq16Bwd>(dV, Lt, Rt, dX, dU, s.rows, status, st);
-  if (rows_shape_is<RowsSq32>(s)) return launch_rows<RowsSq32Bwd>(dV, Lt, Rt, dX, dU, s.rows, status, st);
+  if (rows_shape_is<RowsSq16>(s)) return launch_rows<RowsSq16Bwd>(dV, Lt, Rt, dX, dU, s.rows, status, st, true);
+  if (rows_shape_is<RowsSq32>(s)) return launch_rows<RowsSq32Bwd>(dV, Lt, Rt, dX, dU, s.rows, status, st, true);
   return cudaErrorNotSupported;
 }
 

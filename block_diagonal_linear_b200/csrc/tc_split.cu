@@ -1,0 +1,298 @@
+// Monarch forward for large square blocks (nb1 = nb2, every block 64 x 64, e.g. n = 4096),
+// where a row tile's middle vector (64 rows x 4096 bf16 = 512 KB) cannot stay on chip.
+// The two block-diagonal stages and the two permutations run as four passes over Y, which
+// doubles as the only scratch (the middle vector has the width of the output):
+//   1. Y <- blockdiag(R) X          tcgen05 block-diagonal GEMM, u[k][p] at column k*out1 + p
+//   2. Y <- P Y                     per-row (nb1 x out1) -> (out1 x nb1) transpose, in place
+//   3. Y <- blockdiag(L) Y          the same GEMM; in place, since in2 = out2 makes every unit
+//                                   read and write the same 128-row x 64-column tile
+//   4. Y <- P_out Y                 (out_transpose only) per-row (nb2 x out2) -> (out2 x nb2)
+// GEMM kernel: one unit = (128-row tile, block k).  Warp 0 streams the X box and the W[k] box
+// of each 64-wide K step with TMA (128B swizzle; W has 128-byte rows, so both operands are
+// TMA-friendly), warp 1 issues M = 128, N = 64 MMAs into one of two TMEM slots, warps 2..5
+// drain TMEM (one row per thread), round to bf16 into one of two 128B-swizzled staging tiles
+// and one thread writes the tile with TMA stores.  All waits are bounded (tc_common.cuh).
+#include "tc_common.cuh"
+
+namespace monarch {
+
+constexpr int kBdThreads = 192;
+constexpr int kBdDrainWarps = 4;
+
+template <int KB_, int NB_>
+struct BdCfg {
+  static constexpr int KB = KB_, NB = NB_;  // block input (K) and output (N) widths
+  static constexpr int BM = 128;
+  static constexpr int NKB = KB / 64;                  // 64-wide K boxes per unit
+  static constexpr int XBOX = BM * 128;                // 128 rows x 64 bf16
+  static constexpr int WBOX = NB * 128;                // NB rows of W[k] x 64 bf16
+  static constexpr int STAGE = XBOX + WBOX;
+  static constexpr int ATOM = BM * 128;
+  static constexpr int OATOMS = NB / 64;
+  static constexpr int OUT_BYTES = OATOMS * ATOM;      // one staged output tile
+  static constexpr int TMEM_COLS = 2 * NB <= 32 ? 32 : (2 * NB <= 64 ? 64 : (2 * NB <= 128 ? 128 : (2 * NB <= 256 ? 256 : 512)));
+  static constexpr int NSTAGE_RAW = (kSmemBudget - 2 * OUT_BYTES - 1024) / STAGE;
+  static constexpr int NSTAGE = NSTAGE_RAW > 8 ? 8 : NSTAGE_RAW;
+  static constexpr int SMEM_BYTES = 2 * OUT_BYTES + NSTAGE * STAGE + 1024 + 1024;
+  static_assert(KB % 64 == 0 && NB % 64 == 0 && NB <= 256, "block sizes");
+  static_assert(2 * NB <= 512, "two TMEM slots");
+  static_assert(NSTAGE >= 2, "shared memory");
+};
+
+struct BdBars {
+  uint64_t full[8], empty[8];
+  uint64_t acc_full[2], acc_empty[2];
+  uint64_t staged, stg_free, mma_done;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+// Byte offset of the 16-byte chunk holding columns [c, c+8) of row r in a tile of 64-column,
+// 128B-swizzled atoms of 128 rows.
+__device__ __forceinline__ uint32_t bd_chunk_off(int r, int c) {
+  const uint32_t chunk = (uint32_t)((c & 63) >> 3);
+  return (uint32_t)(c >> 6) * (128 * 128) + (uint32_t)(r >> 3) * 1024 + (uint32_t)(r & 7) * 128 +
+         ((chunk ^ (uint32_t)(r & 7)) << 4);
+}
+
+template <class C>
+__global__ void __launch_bounds__(kBdThreads, 1)
+    tc_bdgemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
+                     const __grid_constant__ CUtensorMap tmY, int nb, int64_t rows, int* status) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  uint8_t* stg = smem;                       // 2 staged output tiles
+  uint8_t* ring = smem + 2 * C::OUT_BYTES;   // NSTAGE x (X box + W box)
+  BdBars* bars = (BdBars*)(ring + C::NSTAGE * C::STAGE);
+  int* abort_flag = &bars->abort_flag;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int64_t ntiles = (rows + C::BM - 1) / C::BM;
+  const int64_t nunits = ntiles * nb;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < C::NSTAGE; ++i) {
+      ptx::mbar_init(&bars->full[i], 1);
+      ptx::mbar_init(&bars->empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      ptx::mbar_init(&bars->acc_full[i], 1);
+      ptx::mbar_init(&bars->acc_empty[i], kBdDrainWarps);
+    }
+    ptx::mbar_init(&bars->staged, kBdDrainWarps);
+    ptx::mbar_init(&bars->stg_free, 1);
+    ptx::mbar_init(&bars->mma_done, 1);
+    bars->abort_flag = 0;
+    ptx::fence_mbar_init();
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc(&bars->tmem_base, C::TMEM_COLS);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+  // the input may be written by the previous kernel of the stream
+  ptx::griddep_wait();
+  ptx::griddep_launch_dependents();
+
+  if (warp == 0) {
+    // ================================================================ TMA producer
+    if (lane == 0) {
+      ptx::tma_prefetch_desc(&tmX);
+      ptx::tma_prefetch_desc(&tmW);
+      ptx::tma_prefetch_desc(&tmY);
+      const uint64_t pol_x = ptx::policy_evict_first(), pol_w = ptx::policy_evict_last();
+      uint32_t it = 0;
+      bool ok = true;
+      for (int64_t u = blockIdx.x; u < nunits && ok; u += gridDim.x) {
+        const int tile = (int)(u / nb), k = (int)(u % nb);
+        for (int kb = 0; kb < C::NKB; ++kb, ++it) {
+          const int st = it % C::NSTAGE;
+          if (!wait_or_abort(&bars->empty[st], ((it / C::NSTAGE) & 1) ^ 1, abort_flag, status)) { ok = false; break; }
+          uint8_t* sb = ring + st * C::STAGE;
+          ptx::mbar_arrive_expect_tx(&bars->full[st], C::STAGE);
+          ptx::tma_load_2d(sb, &tmX, &bars->full[st], k * C::KB + kb * 64, tile * C::BM, pol_x);
+          ptx::tma_load_2d(sb + C::XBOX, &tmW, &bars->full[st], kb * 64, k * C::NB, pol_w);
+        }
+      }
+      const uint32_t issued = it;
+      for (uint32_t q = (issued > (uint32_t)C::NSTAGE ? issued - C::NSTAGE : 0); q < issued; ++q)
+        ptx::mbar_wait_bounded(&bars->full[q % C::NSTAGE], (q / C::NSTAGE) & 1, kWaitLimitNs);
+    }
+  } else if (warp == 1) {
+    // ================================================================ MMA issuer (whole warp)
+    constexpr uint32_t idesc = make_idesc(C::BM, C::NB);
+    const uint64_t ring_d = make_sdesc(ptx::smem_u32(ring), 1024, 2);
+    uint32_t it = 0, n = 0;
+    bool ok = true;
+    for (int64_t u = blockIdx.x; u < nunits && ok; u += gridDim.x, ++n) {
+      const int slot = n & 1;
+      if (!warp_wait_or_abort(lane, &bars->acc_empty[slot], ((n >> 1) & 1) ^ 1, abort_flag, status)) { ok = false; break; }
+      ptx::tc_fence_after();
+      const uint32_t d = tmem + (uint32_t)(slot * C::NB);
+      for (int kb = 0; kb < C::NKB; ++kb, ++it) {
+        const int st = it % C::NSTAGE;
+        if (!warp_wait_or_abort(lane, &bars->full[st], (it / C::NSTAGE) & 1, abort_flag, status)) { ok = false; break; }
+        ptx::tc_fence_after();
+        const uint64_t soff = (uint64_t)((st * C::STAGE) >> 4);
+#pragma unroll
+        for (int t = 0; t < 4; ++t)
+          ptx::mma_bf16_ss_elect(d, ring_d + soff + (uint64_t)((32 * t) >> 4),
+                                 ring_d + soff + (uint64_t)((C::XBOX + 32 * t) >> 4), idesc,
+                                 (kb > 0 || t > 0) ? 1u : 0u);
+        ptx::mma_commit_elect(&bars->empty[st]);
+      }
+      if (!ok) break;
+      ptx::mma_commit_elect(&bars->acc_full[slot]);
+    }
+    ptx::mma_commit_elect(&bars->mma_done);
+    if (lane == 0) ptx::mbar_wait_bounded(&bars->mma_done, 0, kWaitLimitNs);
+    __syncwarp();
+  } else {
+    // ================================================================ drain (4 warps, one row per thread)
+    const int quad = warp & 3;
+    const int r = quad * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+    const uint32_t stg_s = ptx::smem_u32(stg);
+    const bool leader = (warp == 2 && lane == 0);
+    uint32_t n = 0;
+    bool ok = true;
+    for (int64_t u = blockIdx.x; u < nunits && ok; u += gridDim.x, ++n) {
+      const int slot = n & 1;
+      const int tile = (int)(u / nb), k = (int)(u % nb);
+      if (!wait_or_abort(&bars->acc_full[slot], (n >> 1) & 1, abort_flag, status)) { ok = false; break; }
+      // staging tile `slot` was last written two units ago; its stores must have read it
+      if (leader) {
+        ptx::bulk_wait_read_allbut1();
+        ptx::mbar_arrive(&bars->stg_free);
+      }
+      if (!wait_or_abort(&bars->stg_free, n & 1, abort_flag, status)) { ok = false; break; }
+      __syncwarp();  // tcgen05.ld is warp-collective
+      ptx::tc_fence_after();
+      const uint32_t tb = tmem + lane_off + (uint32_t)(slot * C::NB);
+      const uint32_t sb = stg_s + (uint32_t)(slot * C::OUT_BYTES);
+#pragma unroll 1
+      for (int c = 0; c < C::NB; c += 32) {
+        uint32_t v0[16], v1[16];
+        ptx::tmem_ld16(tb + c, v0);
+        ptx::tmem_ld16(tb + c + 16, v1);
+        ptx::tmem_wait_ld();
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+          const uint32_t* v = h < 2 ? v0 : v1;
+          const int e = (h & 1) * 8;
+          ptx::st_shared_v4(sb + bd_chunk_off(r, c + 8 * h),
+                            ptx::pack_bf16x2(__uint_as_float(v[e + 0]), __uint_as_float(v[e + 1])),
+                            ptx::pack_bf16x2(__uint_as_float(v[e + 2]), __uint_as_float(v[e + 3])),
+                            ptx::pack_bf16x2(__uint_as_float(v[e + 4]), __uint_as_float(v[e + 5])),
+                            ptx::pack_bf16x2(__uint_as_float(v[e + 6]), __uint_as_float(v[e + 7])));
+        }
+      }
+      ptx::tc_fence_before();
+      ptx::fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        ptx::mbar_arrive(&bars->acc_empty[slot]);
+        ptx::mbar_arrive(&bars->staged);
+      }
+      if (leader) {
+        if (!wait_or_abort(&bars->staged, n & 1, abort_flag, status)) {
+          ok = false;
+        } else {
+          for (int a = 0; a < C::OATOMS; ++a)
+            ptx::tma_store_2d(&tmY, stg + slot * C::OUT_BYTES + a * C::ATOM, k * C::NB + a * 64, tile * C::BM);
+          ptx::bulk_commit_group();
+        }
+      }
+    }
+    if (leader) ptx::bulk_wait_all();
+  }
+
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  if (warp == 1) ptx::tmem_dealloc(tmem, C::TMEM_COLS);
+}
+
+// dst[r][b*A + a] = src[r][a*B + b]: per row an (A x B) -> (B x A) transpose.  One warp per
+// row: the whole row is read with 16-byte loads into shared memory (odd word pitch, so the
+// column reads hit 32 banks) before any of it is written, so src may equal dst.
+constexpr int kPermWarps = 8;
+__global__ void __launch_bounds__(kPermWarps * 32)
+    permute_rows_kernel(const __nv_bfloat16* src, __nv_bfloat16* dst, int64_t rows, int A, int B) {
+  extern __shared__ __align__(16) uint32_t shw[];
+  ptx::griddep_wait();
+  ptx::griddep_launch_dependents();
+  const int n = A * B, pitch = B + 2, wpitch = pitch / 2;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  uint32_t* buf = shw + warp * (A * wpitch);
+  const uint16_t* hb = (const uint16_t*)buf;
+  for (int64_t r = (int64_t)blockIdx.x * kPermWarps + warp; r < rows; r += (int64_t)gridDim.x * kPermWarps) {
+    const __nv_bfloat16* s = src + r * n;
+    for (int c = lane; c < n / 8; c += 32) {  // source chunk: a = 8c / B, b0 = 8c % B
+      const uint4 v = *(const uint4*)(s + c * 8);
+      uint32_t* d = buf + ((c * 8) / B) * wpitch + ((c * 8) % B) / 2;
+      d[0] = v.x; d[1] = v.y; d[2] = v.z; d[3] = v.w;
+    }
+    __syncwarp();
+    __nv_bfloat16* d = dst + r * n;
+    for (int c = lane; c < n / 8; c += 32) {  // destination chunk: b = 8c / A, a0 = 8c % A
+      const int b = (c * 8) / A, a0 = (c * 8) % A;
+      uint32_t w[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        w[e] = (uint32_t)hb[(a0 + 2 * e) * pitch + b] | ((uint32_t)hb[(a0 + 2 * e + 1) * pitch + b] << 16);
+      *(uint4*)(d + c * 8) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+    __syncwarp();
+  }
+}
+
+template <class C>
+static cudaError_t launch_bdgemm(const void* X, const void* W, void* Y, int nb, int64_t rows,
+                                 int* status, cudaStream_t st, bool pdl) {
+  CUtensorMap mX, mW, mY;
+  if (!make_map_2d(&mX, X, (uint64_t)nb * C::KB, (uint64_t)rows, 64, C::BM, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map_2d(&mW, W, C::KB, (uint64_t)nb * C::NB, 64, C::NB, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map_2d(&mY, Y, (uint64_t)nb * C::NB, (uint64_t)rows, 64, C::BM, CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(tc_bdgemm_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       C::SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  const int64_t nunits = (rows + C::BM - 1) / C::BM * nb;
+  const int64_t grid = nunits < num_sms() ? nunits : num_sms();
+  return launch_kernel(tc_bdgemm_kernel<C>, dim3((unsigned)grid), dim3(kBdThreads), C::SMEM_BYTES, st, pdl,
+                       mX, mW, mY, nb, rows, status);
+}
+
+static cudaError_t launch_permute(__nv_bfloat16* Y, int64_t rows, int A, int B, cudaStream_t st) {
+  const size_t smem = (size_t)kPermWarps * (size_t)A * (size_t)(B + 2) * 2;
+  cudaError_t e = cudaFuncSetAttribute(permute_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem);
+  if (e != cudaSuccess) return e;
+  return launch_kernel(permute_rows_kernel, dim3(2 * 148), dim3(kPermWarps * 32), smem, st, true,
+                       (const __nv_bfloat16*)Y, Y, rows, A, B);
+}
+
+using Bd64 = BdCfg<64, 64>;
+
+bool tc_split_supported(const Shape& s) {
+  return s.nb1 == s.nb2 && s.in1 == 64 && s.out1 == 64 && s.in2 == 64 && s.out2 == 64 &&
+         s.nb1 >= 1 && s.nb1 <= 256;
+}
+
+cudaError_t tc_split_fwd(const void* X, const void* R, const void* L, void* Y, const Shape& s,
+                         int* status, cudaStream_t st) {
+  if (!tc_split_supported(s)) return cudaErrorNotSupported;
+  if (s.rows == 0) return cudaSuccess;
+  __nv_bfloat16* y = (__nv_bfloat16*)Y;
+  cudaError_t e;
+  if ((e = launch_bdgemm<Bd64>(X, R, Y, s.nb1, s.rows, status, st, false)) != cudaSuccess) return e;
+  if ((e = launch_permute(y, s.rows, s.nb1, s.out1, st)) != cudaSuccess) return e;
+  if ((e = launch_bdgemm<Bd64>(Y, L, Y, s.nb2, s.rows, status, st, true)) != cudaSuccess) return e;
+  if (s.out_transpose) return launch_permute(y, s.rows, s.nb2, s.out2, st);
+  return cudaSuccess;
+}
+
+}  // namespace monarch

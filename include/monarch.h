@@ -166,7 +166,9 @@ MONARCH_API int monarch_debug_wait_timeout(uint64_t timeout_ns, void* stream);
  * group) units, 2 = tcgen05 fused kernel over 64-row tiles with the whole middle
  * vector on chip, 3 = the same with the second block-diagonal stage computed in
  * rounds of 8 output columns (transposed outputs wider than the middle vector,
- * e.g. 768 -> 3072).  For the backward: 0 = generic FMA kernels, 1 = tensor-core
+ * e.g. 768 -> 3072), 4 = for square 64 x 64 blocks with nb1 = nb2 (e.g. n = 4096):
+ * two tcgen05 block-diagonal GEMM passes and two row-permutation passes over Y (Y
+ * doubles as the middle vector's storage; no scratch).  For the backward: 0 = generic FMA kernels, 1 = tensor-core
  * backward (row-tile kernels for dX and the middle vector, warp-level MMA for the
  * weight gradients).  Host-only. */
 MONARCH_API int monarch_fwd_path(const monarch_dims* d);

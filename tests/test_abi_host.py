@@ -88,6 +88,8 @@ def test_kernel_family_selection():
     assert bdl.fwd_path(synthetic.shape_of(W["n1024_bf16"]), "bf16") == 2
     assert bdl.fwd_path(synthetic.shape_of(W["r768x3072_bf16"]), "bf16") == 3
     assert bdl.fwd_path(synthetic.shape_of(W["nblk4_1024x4096_bf16"]), "bf16") == 1
+    assert bdl.fwd_path(synthetic.shape_of(W["n4096_bf16"]), "bf16") == 4
+    assert bdl.fwd_path(synthetic.shape_of(W["n4096_bf16"]), "f32") == 0
     assert bdl.fwd_path(synthetic.shape_of(W["n256_fp32"]), "f32") == 0
     assert bdl.fwd_path(synthetic.shape_of(W["n256_fp32"]), "bf16") == 2
     assert bdl.fwd_path(dict(nb1=3, in1=5, out1=4, nb2=2, in2=6, out2=7, out_transpose=1), "bf16") == 0

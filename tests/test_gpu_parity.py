@@ -159,7 +159,8 @@ def test_forward_of_identity_is_dense_matrix():
 
 
 @pytest.mark.parametrize("name,rows", [("n1024_bf16", r) for r in (0, 1, 127, 128, 129, 255, 256, 257)]
-                         + [("r768x3072_bf16", r) for r in (0, 1, 63, 64, 65, 191, 9473, 20000)])
+                         + [("r768x3072_bf16", r) for r in (0, 1, 63, 64, 65, 191, 9473, 20000)]
+                         + [("n4096_bf16", r) for r in (0, 1, 127, 129, 1000)])
 def test_tc_forward_tile_edges(name, rows):
     w = W[name]
     shape = synthetic.shape_of(w)
