@@ -393,7 +393,8 @@ def main():
     fwd_tc = fpath >= 1
     bpath = bdl.bwd_path(shape, w["dtype"])
     fwd_launches = (3 + int(shape.get("out_transpose", 1))) if fpath == 4 else 1
-    launches_per_step = (fwd_launches if do_fwd else 0) + ((6 if bpath == 1 else 3) if do_bwd else 0)
+    bwd_launches = ((8 + int(shape.get("out_transpose", 1))) if shape["in1"] == 64 else 6) if bpath == 1 else 3
+    launches_per_step = (fwd_launches if do_fwd else 0) + (bwd_launches if do_bwd else 0)
     # Roofline object: the forward kernel (one launch per forward pass, so the pass time
     # measured by the events is that kernel's launch duration).  The row-tile kernel
     # family is also the largest share of the step in the ncu launch list.  When only
@@ -415,7 +416,7 @@ def main():
                 "peak": peaks["bf16_tflops"], "unit": "TFLOP/s"}
     roof["frac"] = roof["achieved"] / roof["peak"]
     roof["traffic"] = measured_traffic(kname, srcs) if dom == "fwd" and fwd_tc else None
-    roof["kernel"] = kname + (" (pass of %d kernels)" % (6 if bpath == 1 else 3) if dom == "bwd" else "")
+    roof["kernel"] = kname + (" (pass of %d kernels)" % bwd_launches if dom == "bwd" else "")
     roof["algorithmic_bytes_per_launch"] = a["bytes"]
     roof["peak_source"] = peak_src
 

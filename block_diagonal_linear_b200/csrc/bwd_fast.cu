@@ -107,14 +107,14 @@ __device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4],
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-template <int BS>
+template <int BS, int CH = kWgChunk>  // CH: rows per shared-memory chunk
 __global__ void __launch_bounds__(256, 1)
     wgrad_kernel(const __nv_bfloat16* __restrict__ Al, const __nv_bfloat16* __restrict__ Bl,
                  const __nv_bfloat16* __restrict__ Ar, const __nv_bfloat16* __restrict__ Br,
                  int ngroups_l, int64_t rows, int nsplit, float* __restrict__ partial,
                  int64_t nR, int64_t nP, int ncols) {
   constexpr int PITCH = 8 * BS * 2 + 16;  // bytes per staged row (+16: conflict-free ldmatrix)
-  constexpr int TILE = kWgChunk * PITCH;
+  constexpr int TILE = CH * PITCH;
   constexpr int MT = BS / 16, NT = BS / 8;
   extern __shared__ __align__(128) uint8_t smem[];
   ptx::griddep_wait();
@@ -126,14 +126,14 @@ __global__ void __launch_bounds__(256, 1)
   const __nv_bfloat16* A = is_l ? Al : Ar;
   const __nv_bfloat16* B = is_l ? Bl : Br;
   const int64_t ra = rows * blockIdx.x / nsplit, rb = rows * (blockIdx.x + 1) / nsplit;
-  const int nchunks = (int)((rb - ra + kWgChunk - 1) / kWgChunk);
+  const int nchunks = (int)((rb - ra + CH - 1) / CH);
   const uint32_t sbase = ptx::smem_u32(smem);
   constexpr int CPR = 8 * BS * 2 / 16;  // 16-byte chunks per staged row per tensor
 
   auto load = [&](int c, int buf) {
-    const int64_t r0 = ra + (int64_t)c * kWgChunk;
-    for (int q = threadIdx.x; q < 2 * kWgChunk * CPR; q += blockDim.x) {
-      const int t = q / (kWgChunk * CPR), rem = q % (kWgChunk * CPR);
+    const int64_t r0 = ra + (int64_t)c * CH;
+    for (int q = threadIdx.x; q < 2 * CH * CPR; q += blockDim.x) {
+      const int t = q / (CH * CPR), rem = q % (CH * CPR);
       const int rr = rem / CPR, cc = rem % CPR;
       const int64_t r = r0 + rr;
       const bool valid = r < rb;
@@ -165,7 +165,7 @@ __global__ void __launch_bounds__(256, 1)
     const uint32_t tb = sbase + (uint32_t)((buf * 2 + 1) * TILE);
     const int qm = lane >> 3, ri = lane & 7;
 #pragma unroll
-    for (int ks = 0; ks < kWgChunk / 16; ++ks) {
+    for (int ks = 0; ks < CH / 16; ++ks) {
       uint32_t a[MT][4], b[NT][2];
 #pragma unroll
       for (int mt = 0; mt < MT; ++mt) {
@@ -231,7 +231,11 @@ static bool is_fast_square(const Shape& s) {
   return sq && (s.nb1 == 16 || s.nb1 == 32) && s.out_transpose == 1;
 }
 
-bool fast_bwd_supported(const Shape& s) { return is_fast_square(s); }
+// 64 x 64 blocks with nb1 = nb2 (e.g. n = 4096): the middle vector does not fit on chip, so the
+// row stages run as block-diagonal GEMM and row-permutation passes (tc_split.cu).
+static bool is_split_square(const Shape& s) { return tc_split_supported(s); }
+
+bool fast_bwd_supported(const Shape& s) { return is_fast_square(s) || is_split_square(s); }
 
 static int wg_nsplit(const Shape& s) {
   const int ngroups = (s.nb1 + s.nb2) / 8;
@@ -282,7 +286,18 @@ cudaError_t fast_bwd(const void* dY, const void* X, const void* R, const void* L
                          true, (const __nv_bfloat16*)R, (const __nv_bfloat16*)L, Rt, Lt, s)) != cudaSuccess)
     return e;
   const int nsplit = wg_nsplit(s);
-  if (s.rows > 0) {
+  const bool split = is_split_square(s);
+  if (split && !s.out_transpose) dV = (__nv_bfloat16*)dY;  // dV[j][o] = dy[j*out2 + o]: no copy
+  if (s.rows > 0 && split) {
+    // dV = P_out^-1 dY;  Z = P (blockdiag(R) X);  dZ = blockdiag(L^T) dV;  dU = P^-1 dZ;
+    // dX = blockdiag(R^T) dU.  Z and dZ/dU are permuted in place.
+    if (s.out_transpose && (e = permute_rows(dY, dV, s.rows, s.out2, s.nb2, st)) != cudaSuccess) return e;
+    if ((e = bdgemm64(X, R, Z, s.nb1, s.rows, status, st, true)) != cudaSuccess) return e;
+    if ((e = permute_rows(Z, Z, s.rows, s.nb1, s.out1, st)) != cudaSuccess) return e;
+    if ((e = bdgemm64(dV, Lt, dU, s.nb2, s.rows, status, st, true)) != cudaSuccess) return e;
+    if ((e = permute_rows(dU, dU, s.rows, s.out1, s.nb1, st)) != cudaSuccess) return e;
+    if ((e = bdgemm64(dU, Rt, dX, s.nb1, s.rows, status, st, true)) != cudaSuccess) return e;
+  } else if (s.rows > 0) {
     const size_t gsm = (size_t)kGatherWarps * (size_t)s.out2 * (size_t)(s.nb2 + 2) * 2;
     if ((e = launch_kernel(gather_dv_kernel, dim3(2 * 148), dim3(kGatherWarps * 32), gsm, st, true,
                            (const __nv_bfloat16*)dY, dV, s)) != cudaSuccess)
@@ -293,7 +308,15 @@ cudaError_t fast_bwd(const void* dY, const void* X, const void* R, const void* L
   const int ngl = s.nb2 / 8, ngr = s.nb1 / 8;
   dim3 grid((unsigned)nsplit, (unsigned)(ngl + ngr));
   const int ncols = (int)s.n_mid();  // dV, Z, dU, X all have n_mid = n_in = n_out columns here
-  if (s.nb1 == 32) {
+  if (split) {
+    constexpr int smem = 2 * 2 * 32 * (8 * 64 * 2 + 16);
+    if ((e = cudaFuncSetAttribute(wgrad_kernel<64, 32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  smem)) != cudaSuccess)
+      return e;
+    e = launch_kernel(wgrad_kernel<64, 32>, grid, dim3(256), smem, st, true, (const __nv_bfloat16*)dV,
+                      (const __nv_bfloat16*)Z, (const __nv_bfloat16*)dU, (const __nv_bfloat16*)X, ngl,
+                      s.rows, nsplit, part, nR, nP, ncols);
+  } else if (s.nb1 == 32) {
     constexpr int smem = 2 * 2 * kWgChunk * (8 * 32 * 2 + 16);
     if ((e = cudaFuncSetAttribute(wgrad_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   smem)) != cudaSuccess)

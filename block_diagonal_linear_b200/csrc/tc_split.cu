@@ -266,16 +266,23 @@ static cudaError_t launch_bdgemm(const void* X, const void* W, void* Y, int nb, 
                        mX, mW, mY, nb, rows, status);
 }
 
-static cudaError_t launch_permute(__nv_bfloat16* Y, int64_t rows, int A, int B, cudaStream_t st) {
+cudaError_t permute_rows(const void* src, void* dst, int64_t rows, int A, int B, cudaStream_t st) {
+  if (rows == 0) return cudaSuccess;
   const size_t smem = (size_t)kPermWarps * (size_t)A * (size_t)(B + 2) * 2;
   cudaError_t e = cudaFuncSetAttribute(permute_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return e;
   return launch_kernel(permute_rows_kernel, dim3(2 * 148), dim3(kPermWarps * 32), smem, st, true,
-                       (const __nv_bfloat16*)Y, Y, rows, A, B);
+                       (const __nv_bfloat16*)src, (__nv_bfloat16*)dst, rows, A, B);
 }
 
 using Bd64 = BdCfg<64, 64>;
+
+cudaError_t bdgemm64(const void* X, const void* W, void* Y, int nb, int64_t rows, int* status,
+                     cudaStream_t st, bool pdl) {
+  if (rows == 0) return cudaSuccess;
+  return launch_bdgemm<Bd64>(X, W, Y, nb, rows, status, st, pdl);
+}
 
 bool tc_split_supported(const Shape& s) {
   return s.nb1 == s.nb2 && s.in1 == 64 && s.out1 == 64 && s.in2 == 64 && s.out2 == 64 &&
@@ -289,9 +296,9 @@ cudaError_t tc_split_fwd(const void* X, const void* R, const void* L, void* Y, c
   __nv_bfloat16* y = (__nv_bfloat16*)Y;
   cudaError_t e;
   if ((e = launch_bdgemm<Bd64>(X, R, Y, s.nb1, s.rows, status, st, false)) != cudaSuccess) return e;
-  if ((e = launch_permute(y, s.rows, s.nb1, s.out1, st)) != cudaSuccess) return e;
+  if ((e = permute_rows(y, y, s.rows, s.nb1, s.out1, st)) != cudaSuccess) return e;
   if ((e = launch_bdgemm<Bd64>(Y, L, Y, s.nb2, s.rows, status, st, true)) != cudaSuccess) return e;
-  if (s.out_transpose) return launch_permute(y, s.rows, s.nb2, s.out2, st);
+  if (s.out_transpose) return permute_rows(y, y, s.rows, s.nb2, s.out2, st);
   return cudaSuccess;
 }
 
