@@ -244,7 +244,9 @@ __global__ void __launch_bounds__(kWideThreads, 1)
         ptx::cp_async_mbar_arrive_noinc(&bars->lfull[slot]);
       }
     }
-    ptx::cp_async_wait<0>();  // no copy may still target this CTA's shared memory at exit
+    // no copy may still target this CTA's shared memory at exit: the copies were never
+    // committed to a group (the mbarrier tracks them), so commit and wait for all of them
+    asm volatile("cp.async.wait_all;" ::: "memory");
   } else {
     // ================================================================ drain (8 warps)
     const int quad = warp & 3, ph = (warp - 2) >> 2, half = lane >> 4;
