@@ -91,7 +91,10 @@ MONARCH_API int monarch_validate(const monarch_dims* d);
  * In:  X (rows, nb1*in1), R (nb1,out1,in1), L (nb2,out2,in2).
  * Out: Y (rows, nb2*out2), overwritten.
  * bf16 path: bf16 inputs, fp32 accumulation on the tensor cores, the middle
- * vector rounded to bf16 on chip, Y rounded to bf16.  fp32 path: fp32 FMA. */
+ * vector rounded to bf16 on chip, Y rounded to bf16.  fp32 path: fp32 FMA.
+ * Y must not overlap X, R or L.  For square 64 x 64 blocks with nb1 = nb2
+ * (monarch_fwd_path 4) Y also holds the middle vector between the passes, so
+ * its contents are unspecified until the call's work on the stream is done. */
 MONARCH_API int monarch_fwd(const void* X, const void* R, const void* L, const monarch_dims* d, void* Y,
                 void* stream);
 
