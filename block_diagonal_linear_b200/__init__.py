@@ -34,6 +34,7 @@ STATUS = {
     -7: "MONARCH_ERR_TIMEOUT",
     -8: "MONARCH_ERR_UNSUPPORTED",
     -9: "MONARCH_ERR_SCRATCH",
+    -10: "MONARCH_ERR_ALIAS",
 }
 CODES = {v: k for k, v in STATUS.items()}
 

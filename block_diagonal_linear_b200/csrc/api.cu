@@ -43,6 +43,29 @@ static int check_ptrs(std::initializer_list<const void*> ps) {
   return MONARCH_OK;
 }
 
+// Byte range of a tensor argument; empty for a null pointer or no elements.
+struct Span {
+  uintptr_t p;
+  uint64_t n;
+};
+static Span span(const void* p, int64_t elems, int64_t elem_bytes) {
+  return {(uintptr_t)p, (p != nullptr && elems > 0) ? (uint64_t)elems * (uint64_t)elem_bytes : 0};
+}
+static bool overlap(const Span& a, const Span& b) {
+  return a.n != 0 && b.n != 0 && a.p < b.p + b.n && b.p < a.p + a.n;
+}
+// Every output must be disjoint from every input and from every other output: kernels read
+// inputs after earlier kernels of the same call have written outputs.
+static int check_alias(std::initializer_list<Span> outs, std::initializer_list<Span> ins) {
+  for (const Span* o = outs.begin(); o != outs.end(); ++o) {
+    for (const Span& i : ins)
+      if (overlap(*o, i)) return MONARCH_ERR_ALIAS;
+    for (const Span* o2 = o + 1; o2 != outs.end(); ++o2)
+      if (overlap(*o, *o2)) return MONARCH_ERR_ALIAS;
+  }
+  return MONARCH_OK;
+}
+
 __global__ void debug_wait_kernel(uint64_t timeout_ns, int* status) {
   __shared__ __align__(8) uint64_t bar;
   if (threadIdx.x == 0) {
@@ -107,6 +130,11 @@ int monarch_fwd(const void* X, const void* R, const void* L, const monarch_dims*
   if (d->rows == 0) return MONARCH_OK;
   if ((rc = check_ptrs({X, R, L, Y})) != MONARCH_OK) return rc;
   const Shape s = to_shape(*d);
+  const int64_t es = d->dtype == MONARCH_BF16 ? 2 : 4;
+  if ((rc = check_alias({span(Y, s.rows * s.n_out(), es)},
+                        {span(X, s.rows * s.n_in(), es), span(R, s.n_R(), es), span(L, s.n_L(), es)})) !=
+      MONARCH_OK)
+    return rc;
   cudaStream_t st = (cudaStream_t)stream;
   cudaError_t e;
   const int path = fwd_path(s, d->dtype);
@@ -140,6 +168,12 @@ int monarch_bwd(const void* dY, const void* X, const void* R, const void* L, con
   const size_t need = bwd_workspace(s, d->dtype);
   if (workspace == nullptr || workspace_bytes < need) return MONARCH_ERR_WORKSPACE;
   if (((uintptr_t)workspace & 255u) != 0) return MONARCH_ERR_ALIGN;
+  const int64_t es = d->dtype == MONARCH_BF16 ? 2 : 4;
+  if ((rc = check_alias({span(dX, s.rows * s.n_in(), es), span(dR, s.n_R(), es), span(dL, s.n_L(), es),
+                         span(workspace, (int64_t)need, 1)},
+                        {span(dY, s.rows * s.n_out(), es), span(X, s.rows * s.n_in(), es),
+                         span(R, s.n_R(), es), span(L, s.n_L(), es)})) != MONARCH_OK)
+    return rc;
   cudaError_t e;
   if (bwd_path(s, d->dtype) == 1) {
     int* status = status_ptr();
@@ -157,6 +191,11 @@ int monarch_materialise(const void* R, const void* L, const monarch_dims* d, voi
   int rc = check_dims(d);
   if (rc != MONARCH_OK) return rc;
   if ((rc = check_ptrs({R, L, M})) != MONARCH_OK) return rc;
+  const Shape ms = to_shape(*d);
+  const int64_t es = d->dtype == MONARCH_BF16 ? 2 : 4;
+  if ((rc = check_alias({span(M, ms.n_out() * ms.n_in(), 4)}, {span(R, ms.n_R(), es), span(L, ms.n_L(), es)})) !=
+      MONARCH_OK)
+    return rc;
   cudaError_t e = generic_materialise(R, L, (float*)M, to_shape(*d), d->dtype, (cudaStream_t)stream);
   return e == cudaSuccess ? MONARCH_OK : MONARCH_ERR_CUDA;
 }
@@ -173,6 +212,7 @@ const char* monarch_status_string(int status) {
     case MONARCH_ERR_TIMEOUT: return "bounded device wait timed out";
     case MONARCH_ERR_UNSUPPORTED: return "shape not supported by any kernel";
     case MONARCH_ERR_SCRATCH: return "problem larger than the fixed scratch of monarch_bwd_noalloc";
+    case MONARCH_ERR_ALIAS: return "an output or the workspace overlaps another argument";
     default: return "unknown status";
   }
 }

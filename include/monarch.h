@@ -33,6 +33,9 @@
  *     monarch_last_device_status().
  *   - The library allocates no device memory.  monarch_bwd takes a caller-owned
  *     workspace of at least monarch_bwd_workspace_bytes(d) bytes.
+ *   - Outputs (and the workspace) must not overlap any input or one another;
+ *     overlapping byte ranges are rejected with MONARCH_ERR_ALIAS before any
+ *     device work.
  *   - Return value: MONARCH_OK (0) or a negative MONARCH_ERR_* code.  Nothing
  *     aborts, throws or prints.  A failed call leaves its outputs unspecified.
  *   - Kernel-side bounded waits that give up record MONARCH_ERR_TIMEOUT in a
@@ -69,7 +72,8 @@ enum {
   MONARCH_ERR_CUDA = -6,        /* a CUDA runtime call or kernel launch failed */
   MONARCH_ERR_TIMEOUT = -7,     /* a bounded device wait gave up (device status) */
   MONARCH_ERR_UNSUPPORTED = -8, /* shape too large for any kernel of this build */
-  MONARCH_ERR_SCRATCH = -9      /* monarch_bwd_noalloc: problem needs more than its fixed scratch */
+  MONARCH_ERR_SCRATCH = -9,     /* monarch_bwd_noalloc: problem needs more than its fixed scratch */
+  MONARCH_ERR_ALIAS = -10       /* an output (or the workspace) overlaps an input or another output */
 };
 
 /* Shape of one Monarch map.  Scatterbrain thread, MonarchLinear __init__ and

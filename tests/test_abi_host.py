@@ -98,3 +98,35 @@ def test_kernel_family_selection():
     assert bdl.bwd_path(synthetic.shape_of(W["n256_fp32"]), "f32") == 0
     assert bdl.bwd_path(synthetic.shape_of(W["n4096_bf16"]), "bf16") == 1
     assert bdl.bwd_path(synthetic.shape_of(W["r768x3072_bf16"]), "bf16") == 0
+
+
+def test_overlapping_outputs_rejected_before_device_work():
+    """Outputs (and the backward workspace) must not overlap inputs or each other: the 64x64
+    path keeps the middle vector in Y, and the backward's kernels read inputs after earlier
+    kernels of the same call wrote outputs.  Fake, aligned addresses: every case returns
+    before any CUDA call."""
+    lib = bdl.lib()
+    shape = dict(nb1=4, in1=8, out1=8, nb2=4, in2=8, out2=8, out_transpose=1)
+    rows = 5
+    d = bdl.make_dims(shape, rows, "f32")
+    A = lambda a: ctypes.c_void_p(a)
+    x, r, l = 1 << 20, 2 << 20, 3 << 20       # X: 5*32*4 = 640 B, R and L: 1024 B each
+    alias = bdl.CODES["MONARCH_ERR_ALIAS"]
+    assert lib.monarch_fwd(A(x), A(r), A(l), ctypes.byref(d), A(x + 624), None) == alias  # Y overlaps X
+    assert lib.monarch_fwd(A(x), A(r), A(l), ctypes.byref(d), A(r - 16), None) == alias   # Y runs into R
+    assert lib.monarch_fwd(A(x), A(r), A(l), ctypes.byref(d), A(l), None) == alias        # Y is L
+    need = bdl.bwd_workspace_bytes(shape, rows, "f32")
+    dy, dx, dr, dl, ws = 4 << 20, 5 << 20, 6 << 20, 7 << 20, 8 << 20
+    ok = dict(dy=dy, x=x, r=r, l=l, dx=dx, dr=dr, dl=dl, ws=ws)
+
+    def bwd(**kw):
+        a = dict(ok, **kw)
+        return lib.monarch_bwd(A(a["dy"]), A(a["x"]), A(a["r"]), A(a["l"]), ctypes.byref(d), A(a["dx"]),
+                               A(a["dr"]), A(a["dl"]), A(a["ws"]), ctypes.c_size_t(need), None)
+
+    assert bwd(dx=dy) == alias                 # dX is dY
+    assert bwd(dr=dl) == alias                 # dR is dL
+    assert bwd(dl=r + 512) == alias            # dL overlaps R
+    assert bwd(ws=x - 256) == alias            # workspace runs into X
+    assert bwd(ws=dx) == alias                 # workspace is dX
+    assert bdl.status_string(alias) != "unknown status"
