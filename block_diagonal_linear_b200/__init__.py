@@ -138,6 +138,24 @@ def _stream(stream):
     return ctypes.c_void_p(s.cuda_stream)
 
 
+def _check_tensors(shape: dict, rows: int, dtype, **ts):
+    """Shapes and dtypes of the tensor arguments against the Monarch dims (raises ValueError)."""
+    n_in = shape["nb1"] * shape["in1"]
+    n_out = shape["nb2"] * shape["out2"]
+    want = {
+        "X": (rows, n_in), "dX": (rows, n_in), "Y": (rows, n_out), "dY": (rows, n_out),
+        "R": (shape["nb1"], shape["out1"], shape["in1"]), "dR": (shape["nb1"], shape["out1"], shape["in1"]),
+        "L": (shape["nb2"], shape["out2"], shape["in2"]), "dL": (shape["nb2"], shape["out2"], shape["in2"]),
+    }
+    for name, t in ts.items():
+        if t is None:
+            continue
+        if tuple(t.shape) != want[name]:
+            raise ValueError("%s has shape %s, the dims need %s" % (name, tuple(t.shape), want[name]))
+        if t.dtype != dtype:
+            raise ValueError("%s is %s, X is %s: every tensor must have one dtype" % (name, t.dtype, dtype))
+
+
 def _require_cuda(*ts):
     for t in ts:
         if t is not None and (not t.is_cuda or not t.is_contiguous()):
@@ -168,6 +186,7 @@ def fwd(X, R, L, shape: dict, Y=None, stream=None):
     code = dtype_code(X.dtype)
     n_out = shape["nb2"] * shape["out2"]
     rows = X.shape[0]
+    _check_tensors(shape, rows, X.dtype, X=X, R=R, L=L, Y=Y)
     if Y is None:
         Y = torch.empty((rows, n_out), dtype=X.dtype, device=X.device)
     _require_cuda(X, R, L, Y)
@@ -182,6 +201,7 @@ def bwd(dY, X, R, L, shape: dict, dX=None, dR=None, dL=None, workspace=None, str
     import torch
     code = dtype_code(X.dtype)
     rows = X.shape[0]
+    _check_tensors(shape, rows, X.dtype, dY=dY, X=X, R=R, L=L, dX=dX, dR=dR, dL=dL)
     if dX is None:
         dX = torch.empty_like(X)
     if dR is None:
@@ -207,6 +227,7 @@ def bwd_noalloc(dY, X, R, L, shape: dict, dX=None, dR=None, dL=None, stream=None
     the GPU share that scratch and must not run concurrently."""
     import torch
     code = dtype_code(X.dtype)
+    _check_tensors(shape, X.shape[0], X.dtype, dY=dY, X=X, R=R, L=L, dX=dX, dR=dR, dL=dL)
     if dX is None:
         dX = torch.empty_like(X)
     if dR is None:
@@ -225,6 +246,7 @@ def materialise(R, L, shape: dict, M=None, stream=None):
     """Dense M (n_out, n_in) as float32 with Y = X M^T."""
     import torch
     code = dtype_code(R.dtype)
+    _check_tensors(shape, 0, R.dtype, R=R, L=L)
     n_in = shape["nb1"] * shape["in1"]
     n_out = shape["nb2"] * shape["out2"]
     if M is None:

@@ -130,3 +130,29 @@ def test_overlapping_outputs_rejected_before_device_work():
     assert bwd(ws=x - 256) == alias            # workspace runs into X
     assert bwd(ws=dx) == alias                 # workspace is dX
     assert bdl.status_string(alias) != "unknown status"
+
+
+def test_binding_checks_tensor_shapes_and_dtypes_first():
+    """The binding compares every tensor with the dims before anything reaches the library,
+    so mismatched factors fail loudly instead of being read with the wrong layout."""
+    import torch
+    shape = dict(nb1=4, in1=8, out1=8, nb2=4, in2=8, out2=16, out_transpose=1)
+    X = torch.zeros(5, 32, dtype=torch.bfloat16)
+    R = torch.zeros(4, 8, 8, dtype=torch.bfloat16)
+    L = torch.zeros(4, 16, 8, dtype=torch.bfloat16)
+    dY = torch.zeros(5, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="L has shape"):
+        bdl.fwd(X, R, L.transpose(1, 2), shape)
+    with pytest.raises(ValueError, match="X has shape"):
+        bdl.fwd(X[:, :16], R, L, shape)
+    with pytest.raises(ValueError, match="one dtype"):
+        bdl.fwd(X, R.float(), L, shape)
+    with pytest.raises(ValueError, match="dY has shape"):
+        bdl.bwd(dY[:, :32], X, R, L, shape)
+    with pytest.raises(ValueError, match="Y has shape"):
+        bdl.fwd(X, R, L, shape, Y=torch.zeros(5, 32, dtype=torch.bfloat16))
+    with pytest.raises(ValueError, match="R has shape"):
+        bdl.materialise(R[:2], L, shape)
+    # correct shapes get past the check and stop at the CUDA-tensor requirement
+    with pytest.raises(ValueError, match="CUDA"):
+        bdl.fwd(X, R, L, shape)
