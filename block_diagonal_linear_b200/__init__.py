@@ -168,11 +168,14 @@ def validate(shape: dict, rows: int = 0, dtype="bf16") -> int:
 
 
 def fwd_path(shape: dict, dtype="bf16") -> int:
-    """0 = generic FMA kernels, 1 = fused tcgen05 kernel (host-only query)."""
+    """Forward kernel family (host-only query): 0 generic FMA, 1 tcgen05 (row tile x block
+    group), 2 tcgen05 row tile, 3 tcgen05 row tile with the L stage in output-column rounds,
+    4 tcgen05 block-diagonal GEMM and row-permutation passes (64 x 64 blocks)."""
     return lib().monarch_fwd_path(ctypes.byref(make_dims(shape, 1, dtype)))
 
 
 def bwd_path(shape: dict, dtype="bf16") -> int:
+    """Backward kernel family (host-only query): 0 generic FMA, 1 tensor-core kernels."""
     return lib().monarch_bwd_path(ctypes.byref(make_dims(shape, 1, dtype)))
 
 
