@@ -156,3 +156,25 @@ def test_binding_checks_tensor_shapes_and_dtypes_first():
     # correct shapes get past the check and stop at the CUDA-tensor requirement
     with pytest.raises(ValueError, match="CUDA"):
         bdl.fwd(X, R, L, shape)
+
+
+def test_shape_beyond_every_kernel_is_unsupported_before_device_work():
+    """A middle vector wider than the generic kernels' shared-memory row (fp32, 60000 wide)
+    is rejected with MONARCH_ERR_UNSUPPORTED on the host (fake, disjoint, aligned pointers)."""
+    lib = bdl.lib()
+    shape = dict(nb1=1, in1=16, out1=60000, nb2=1, in2=60000, out2=16, out_transpose=1)
+    d = bdl.make_dims(shape, 2, "f32")
+    assert bdl.validate(shape, 2, "f32") == 0
+    A = lambda i: ctypes.c_void_p(i << 24)  # 16 MiB apart: no argument overlaps another
+    unsupported = bdl.CODES["MONARCH_ERR_UNSUPPORTED"]
+    assert lib.monarch_fwd(A(1), A(2), A(3), ctypes.byref(d), A(4), None) == unsupported
+    need = bdl.bwd_workspace_bytes(shape, 2, "f32")
+    assert 0 < need < (16 << 24)
+    rc = lib.monarch_bwd(A(5), A(1), A(2), A(3), ctypes.byref(d), A(6), A(7), A(8), A(16),
+                         ctypes.c_size_t(need), None)
+    assert rc == unsupported
+
+
+def test_oversized_dims_rejected():
+    assert bdl.validate(dict(nb1=1 << 21, in1=1 << 20, out1=1, nb2=1, in2=1 << 21, out2=1), 1, "bf16") == \
+        bdl.CODES["MONARCH_ERR_DIMS"]
