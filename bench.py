@@ -35,6 +35,8 @@ from block_diagonal_linear_b200 import synthetic  # noqa: E402
 DEFAULT_WORKLOAD = "n1024_bf16"
 METRIC = "Monarch fwd/bwd rows/s and TFLOP/s at 1 B200; achieved % of roofline per shape"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# fp32 FMA peak (not measured): 148 SMs x 128 FMA lanes x 2 flops x 1.965 GHz
+FFMA_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 
 
 def describe(name: str, w: dict) -> str:
@@ -211,6 +213,104 @@ def run_reference(args, w, name):
     }), flush=True)
 
 
+# --------------------------------------------------------------------------- kernel paths
+FWD_KERNEL = {2: "tc_rows_kernel", 3: "tc_wide_kernel", 4: "tc_bdgemm_kernel + permute_rows_kernel",
+              1: "tc_fwd_kernel"}
+FWD_SOURCE = {2: "tc_rows", 3: "tc_wide", 4: "tc_split", 1: "tc_fwd"}
+
+
+def launches(shape: dict, dtype: str, pname: str) -> int:
+    """Kernels one forward or backward call launches, counted by the library itself on a
+    one-row call (the count does not depend on the row count)."""
+    import torch
+    import block_diagonal_linear_b200 as bdl
+    w = dict(shape, rows=1, dtype=dtype)
+    n_in, _, n_out = synthetic.sizes(w)
+    dt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    X = torch.zeros((1, n_in), dtype=dt, device="cuda")
+    R = torch.zeros((shape["nb1"], shape["out1"], shape["in1"]), dtype=dt, device="cuda")
+    L = torch.zeros((shape["nb2"], shape["out2"], shape["in2"]), dtype=dt, device="cuda")
+    dY = torch.zeros((1, n_out), dtype=dt, device="cuda")
+    n0 = bdl.kernel_launches()
+    if pname == "fwd":
+        bdl.fwd(X, R, L, shape)
+    else:
+        bdl.bwd(dY, X, R, L, shape)
+    torch.cuda.synchronize()
+    return bdl.kernel_launches() - n0
+
+
+# --------------------------------------------------------------------------- per shape
+PER_SHAPE = ("n256_fp32", "n1024_bf16", "r768x3072_bf16", "n4096_bf16", "nblk4_1024x4096_bf16",
+             "nblk4_1024x4096_bf16_b1000")
+
+
+def device_inputs(w, seed, dev):
+    import torch
+    inp = synthetic.make_inputs(w, seed=seed)
+    out = {}
+    for k in ("X", "R", "L", "dY"):
+        t = inp[k]
+        if t.dtype == "bf16":
+            out[k] = torch.from_numpy(t.bits.view(np.int16).copy()).view(torch.bfloat16).to(dev)
+        else:
+            out[k] = torch.from_numpy(np.ascontiguousarray(t.bits)).to(dev)
+    return out
+
+
+def time_shape(name, dev, flush, peaks, reps=10, warmup=3, spin_cycles=400000):
+    """Forward and backward of one workload, each pass timed alone with CUDA events on the
+    launching stream after an untimed L2 flush and GPU-side spin; averages over `reps`."""
+    import torch
+    import block_diagonal_linear_b200 as bdl
+    w = dict(synthetic.WORKLOADS[name], name=name)
+    shape = synthetic.shape_of(w)
+    rows = w["rows"]
+    d = device_inputs(w, seed=2000, dev=dev)
+    X, R, L, dY = d["X"], d["R"], d["L"], d["dY"]
+    Y = torch.empty((rows, synthetic.sizes(w)[2]), dtype=X.dtype, device=dev)
+    dX, dR, dL = torch.empty_like(X), torch.empty_like(R), torch.empty_like(L)
+    ws = torch.empty(max(bdl.bwd_workspace_bytes(shape, rows, w["dtype"]), 256), dtype=torch.uint8,
+                     device=dev)
+    stream = torch.cuda.current_stream()
+    runs = {"fwd": lambda: bdl.fwd(X, R, L, shape, Y=Y),
+            "bwd": lambda: bdl.bwd(dY, X, R, L, shape, dX=dX, dR=dR, dL=dL, workspace=ws)}
+    alg = algorithmic(w, rows)
+    hbm, tpk = peaks["hbm_gbs"] * 1e9, peaks["bf16_tflops"] * 1e12
+    if w["dtype"] == "f32":
+        tpk = FFMA_TFLOPS * 1e12
+    res = {"workload": describe(name, w), "fwd_path": bdl.fwd_path(shape, w["dtype"]),
+           "bwd_path": bdl.bwd_path(shape, w["dtype"])}
+    for pname, fn in runs.items():
+        evs = []
+        for i in range(warmup + reps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            flush.zero_()
+            torch.cuda._sleep(spin_cycles)
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+            if i >= warmup:
+                evs.append((e0, e1))
+        torch.cuda.synchronize()
+        ms = sum(a.elapsed_time(b) for a, b in evs) / len(evs)
+        t = ms / 1e3
+        a = alg[pname]
+        t_roof = max(a["bytes"] / hbm, a["flops"] / tpk)
+        res[pname] = {
+            "ms": ms, "rows_per_s": rows / t, "tflops": a["flops"] / t / 1e12,
+            "gbs": a["bytes"] / t / 1e9, "roofline_ms": t_roof * 1e3, "roofline_frac": t_roof / t,
+            "bound": "hbm" if a["bytes"] / hbm >= a["flops"] / tpk else
+                     ("fma" if w["dtype"] == "f32" else "tensor"),
+            "launches": launches(shape, w["dtype"], pname),
+        }
+    if bdl.last_device_status() != 0:
+        raise SystemExit("device status not OK after timing %s" % name)
+    del X, R, L, dY, Y, dX, dR, dL, ws, d
+    torch.cuda.empty_cache()
+    return res
+
+
 # --------------------------------------------------------------------------- GPU arm
 def main():
     ap = argparse.ArgumentParser()
@@ -221,6 +321,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end timing")
+    ap.add_argument("--no-per-shape", dest="per_shape", action="store_false",
+                    help="skip the per-workload forward/backward timings")
     ap.add_argument("--pass", dest="only", default="step", choices=["step", "fwd", "bwd"],
                     help="time the whole step (default) or one pass only")
     args = ap.parse_args()
@@ -310,10 +412,12 @@ def main():
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
+    launches0 = bdl.kernel_launches()
     with sampler:
         for k in range(args.steps):
             step(evs[k])
         torch.cuda.synchronize()
+    launches_timed = bdl.kernel_launches() - launches0
     if world > 1:
         dist.barrier()
     fwd_ms = [e[0].elapsed_time(e[1]) for e in evs]
@@ -390,35 +494,47 @@ def main():
             "bound": "hbm" if a["bytes"] / hbm >= a["flops"] / tpk else "tensor",
         }
     fpath = bdl.fwd_path(shape, w["dtype"])
-    fwd_tc = fpath >= 1
     bpath = bdl.bwd_path(shape, w["dtype"])
-    fwd_launches = (3 + int(shape.get("out_transpose", 1))) if fpath == 4 else 1
-    bwd_launches = ((8 + int(shape.get("out_transpose", 1))) if shape["in1"] == 64 else 6) if bpath == 1 else 3
-    launches_per_step = (fwd_launches if do_fwd else 0) + (bwd_launches if do_bwd else 0)
-    # Roofline object: the forward kernel (one launch per forward pass, so the pass time
-    # measured by the events is that kernel's launch duration).  The row-tile kernel
-    # family is also the largest share of the step in the ncu launch list.  When only
-    # the backward is timed, the backward pass (several launches) is reported instead.
-    dom = "fwd" if do_fwd else "bwd"
-    a = alg[dom]
-    t_dom = fwd_avg_s if dom == "fwd" else bwd_avg_s
-    bound = passes[dom]["bound"]
-    kname = ({2: "tc_rows_kernel", 3: "tc_wide_kernel", 4: "tc_bdgemm_kernel + permute_rows_kernel (pass of 4 kernels)",
-              1: "tc_fwd_kernel"}.get(fpath, "gen_fwd_kernel")
-             if dom == "fwd" else "monarch_bwd")
-    srcs = ["block_diagonal_linear_b200/csrc/%s.cu" % {2: "tc_rows", 3: "tc_wide", 4: "tc_split", 1: "tc_fwd"}.get(fpath, "generic"),
-            "block_diagonal_linear_b200/csrc/ptx.cuh", "block_diagonal_linear_b200/csrc/tc_common.cuh"]
-    if bound == "hbm":
-        roof = {"bound": "hbm", "achieved": a["bytes"] / t_dom / 1e9, "peak": peaks["hbm_gbs"],
-                "unit": "GB/s"}
-    else:
-        roof = {"bound": "tensor", "achieved": a["flops"] / t_dom / 1e12,
-                "peak": peaks["bf16_tflops"], "unit": "TFLOP/s"}
-    roof["frac"] = roof["achieved"] / roof["peak"]
-    roof["traffic"] = measured_traffic(kname, srcs) if dom == "fwd" and fwd_tc else None
-    roof["kernel"] = kname + (" (pass of %d kernels)" % bwd_launches if dom == "bwd" else "")
-    roof["algorithmic_bytes_per_launch"] = a["bytes"]
-    roof["peak_source"] = peak_src
+    fwd_launches = launches(shape, w["dtype"], "fwd")
+    bwd_launches = launches(shape, w["dtype"], "bwd")
+    # Roofline objects.  `roofline`: the forward kernel (one launch per forward pass, so the pass
+    # time measured by the events is that kernel's launch duration).  `roofline_bwd`: the backward
+    # pass (several launches), against the backward's algorithmic bytes and flops.
+    def roof_of(pname, t_s, kname, srcs):
+        a = alg[pname]
+        if passes[pname]["bound"] == "hbm":
+            r = {"bound": "hbm", "achieved": a["bytes"] / t_s / 1e9, "peak": peaks["hbm_gbs"],
+                 "unit": "GB/s"}
+        else:
+            r = {"bound": "tensor", "achieved": a["flops"] / t_s / 1e12,
+                 "peak": peaks["bf16_tflops"], "unit": "TFLOP/s"}
+        r["frac"] = r["achieved"] / r["peak"]
+        r["traffic"] = measured_traffic(kname, srcs) if srcs else None
+        r["kernel"] = kname
+        r["algorithmic_bytes_per_launch"] = a["bytes"]
+        r["algorithmic_flops_per_launch"] = a["flops"]
+        r["peak_source"] = peak_src
+        return r
+
+    roof, roof_bwd = None, None
+    if do_fwd:
+        kname = FWD_KERNEL.get(fpath, "gen_fwd_kernel")
+        if fwd_launches > 1:
+            kname += " (pass of %d kernels)" % fwd_launches
+        srcs = (["block_diagonal_linear_b200/csrc/%s.cu" % FWD_SOURCE[fpath],
+                 "block_diagonal_linear_b200/csrc/ptx.cuh", "block_diagonal_linear_b200/csrc/tc_common.cuh"]
+                if fpath in FWD_SOURCE and fwd_launches == 1 else None)
+        roof = roof_of("fwd", fwd_avg_s, kname, srcs)
+    if do_bwd:
+        roof_bwd = roof_of("bwd", bwd_avg_s, "monarch_bwd (pass of %d kernels)" % bwd_launches, None)
+    if roof is None:
+        roof, roof_bwd = roof_bwd, None
+
+    per_shape = None
+    if args.per_shape and world == 1:
+        per_shape = {}
+        for pn in PER_SHAPE:
+            per_shape[pn] = time_shape(pn, dev_, flush, peaks)
 
     value = world * rows * K / (tot_ms / 1e3)
     out = {
@@ -435,10 +551,13 @@ def main():
         "tflops": (alg["fwd"]["flops"] + alg["bwd"]["flops"]) * world * K / (tot_ms / 1e3) / 1e12,
         "passes": passes,
         "roofline": roof,
+        "roofline_bwd": roof_bwd,
+        "per_shape": per_shape,
         "e2e": ({"value": world * rows * n_e2e / (e2e_ms / 1e3), "unit": "rows/s",
                  "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": n_e2e}
                 if n_e2e else None),
-        "gpu_launches": launches_per_step * K,
+        "gpu_launches": launches_timed,
+        "launches_per_step": {"fwd": fwd_launches if do_fwd else 0, "bwd": bwd_launches if do_bwd else 0},
         "clocks": sampler.summary(),
         "device_status": status,
     }

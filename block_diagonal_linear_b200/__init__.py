@@ -42,6 +42,7 @@ EXPORTED = (
     "monarch_validate", "monarch_fwd", "monarch_bwd", "monarch_bwd_workspace_bytes",
     "monarch_materialise", "monarch_status_string", "monarch_last_device_status",
     "monarch_debug_wait_timeout", "monarch_fwd_path", "monarch_bwd_path", "monarch_bwd_noalloc",
+    "monarch_kernel_launches",
 )
 
 
@@ -91,6 +92,8 @@ def lib() -> ctypes.CDLL:
         L.monarch_bwd_noalloc.argtypes = [vp, vp, vp, vp, dp, vp, vp, vp, vp]
         L.monarch_fwd_path.argtypes = [dp]
         L.monarch_bwd_path.argtypes = [dp]
+        L.monarch_kernel_launches.argtypes = []
+        L.monarch_kernel_launches.restype = ctypes.c_uint64
         for name in ("monarch_validate", "monarch_fwd", "monarch_bwd", "monarch_materialise",
                      "monarch_last_device_status", "monarch_debug_wait_timeout",
                      "monarch_fwd_path", "monarch_bwd_path", "monarch_bwd_noalloc"):
@@ -268,6 +271,11 @@ def last_device_status(stream=None) -> int:
 
 def debug_wait_timeout(timeout_ns: int, stream=None) -> int:
     return lib().monarch_debug_wait_timeout(ctypes.c_uint64(int(timeout_ns)), _stream(stream))
+
+
+def kernel_launches() -> int:
+    """Kernels the library has launched in this process (host-side count)."""
+    return int(lib().monarch_kernel_launches())
 
 
 def status_string(code: int) -> str:

@@ -81,8 +81,7 @@ __global__ void debug_wait_kernel(uint64_t timeout_ns, int* status) {
 }
 
 cudaError_t debug_wait_timeout(uint64_t timeout_ns, int* status, cudaStream_t st) {
-  debug_wait_kernel<<<1, 32, 0, st>>>(timeout_ns, status);
-  return cudaGetLastError();
+  return launch_kernel(debug_wait_kernel, dim3(1), dim3(32), 0, st, false, timeout_ns, status);
 }
 
 // 0 = generic FMA kernels, 1 = tcgen05 group kernel, 2 = tcgen05 row-tile kernel,
@@ -224,6 +223,8 @@ int monarch_last_device_status(void* stream) {
   if (cudaMemcpyToSymbol(g_status, &zero, sizeof(int)) != cudaSuccess) return MONARCH_ERR_CUDA;
   return v == kStatusTimeout ? MONARCH_ERR_TIMEOUT : MONARCH_OK;
 }
+
+uint64_t monarch_kernel_launches(void) { return launch_counter().load(std::memory_order_relaxed); }
 
 int monarch_debug_wait_timeout(uint64_t timeout_ns, void* stream) {
   int* status = status_ptr();

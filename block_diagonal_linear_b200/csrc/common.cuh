@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "../../include/monarch.h"
 
 namespace monarch {
@@ -43,6 +45,33 @@ __device__ __forceinline__ float ld_as_f32(const __nv_bfloat16* p) {
 __device__ __forceinline__ void st_from_f32(float* p, float v) { *p = v; }
 __device__ __forceinline__ void st_from_f32(__nv_bfloat16* p, float v) {
   *p = __float2bfloat16_rn(v);
+}
+
+// Kernels launched by this library in this process (host-side count of successful launches).
+inline std::atomic<unsigned long long>& launch_counter() {
+  static std::atomic<unsigned long long> n{0};
+  return n;
+}
+
+// Launch `kernel` on `st`; with pdl = true it may begin launching while the previous kernel of
+// the stream is still running (programmatic stream serialization).  Every kernel launched this
+// way calls ptx::griddep_wait() before it touches global memory that earlier kernels write.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_kernel(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                                 cudaStream_t st, bool pdl, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, ((KArgs)args)...);
+  if (e == cudaSuccess) launch_counter().fetch_add(1, std::memory_order_relaxed);
+  return e;
 }
 
 // Device status word values (written by kernels, read by the host).

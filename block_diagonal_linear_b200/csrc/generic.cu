@@ -239,9 +239,8 @@ static cudaError_t launch_fwd(const void* X, const void* R, const void* L, void*
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const int64_t grid = (s.rows + rpc - 1) / rpc;
-  gen_fwd_kernel<T><<<(unsigned)grid, kGenThreads, smem, st>>>(
-      (const T*)X, (const T*)R, (const T*)L, (T*)Y, s, rpc);
-  return cudaGetLastError();
+  return launch_kernel(gen_fwd_kernel<T>, dim3((unsigned)grid), dim3(kGenThreads), smem, st, false,
+                       (const T*)X, (const T*)R, (const T*)L, (T*)Y, s, rpc);
 }
 
 cudaError_t generic_fwd(const void* X, const void* R, const void* L, void* Y, const Shape& s,
@@ -288,17 +287,17 @@ static cudaError_t launch_bwd(const void* dY, const void* X, const void* R, cons
                              (int)smem);
     if (e != cudaSuccess) return e;
     const int64_t grid = (s.rows + rpc - 1) / rpc;
-    gen_bwd_rows_kernel<T><<<(unsigned)grid, kGenThreads, smem, st>>>(
-        (const T*)dY, (const T*)X, (const T*)R, (const T*)L, (T*)dX, wsZ, wsdZ, s, rpc);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if ((e = launch_kernel(gen_bwd_rows_kernel<T>, dim3((unsigned)grid), dim3(kGenThreads), smem, st, false,
+                           (const T*)dY, (const T*)X, (const T*)R, (const T*)L, (T*)dX, wsZ, wsdZ, s,
+                           rpc)) != cudaSuccess)
+      return e;
   }
   dim3 g((unsigned)((nP + kGenThreads - 1) / kGenThreads), (unsigned)nsplit);
-  gen_bwd_wgrad_kernel<T><<<g, kGenThreads, 0, st>>>((const T*)dY, (const T*)X, wsZ, wsdZ, partial,
-                                                     s, nsplit);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  gen_bwd_reduce_kernel<T><<<(unsigned)((nP + kGenThreads - 1) / kGenThreads), kGenThreads, 0, st>>>(
-      partial, (T*)dR, (T*)dL, s, nsplit);
-  return cudaGetLastError();
+  if ((e = launch_kernel(gen_bwd_wgrad_kernel<T>, g, dim3(kGenThreads), 0, st, false, (const T*)dY,
+                         (const T*)X, (const float*)wsZ, (const float*)wsdZ, partial, s, nsplit)) != cudaSuccess)
+    return e;
+  return launch_kernel(gen_bwd_reduce_kernel<T>, dim3((unsigned)((nP + kGenThreads - 1) / kGenThreads)),
+                       dim3(kGenThreads), 0, st, false, (const float*)partial, (T*)dR, (T*)dL, s, nsplit);
 }
 
 cudaError_t generic_bwd(const void* dY, const void* X, const void* R, const void* L, void* dX,
@@ -313,12 +312,10 @@ cudaError_t generic_materialise(const void* R, const void* L, float* M, const Sh
   const int64_t n = s.n_in() * s.n_out();
   const unsigned grid = (unsigned)((n + kGenThreads - 1) / kGenThreads);
   if (dtype == MONARCH_BF16)
-    gen_materialise_kernel<__nv_bfloat16><<<grid, kGenThreads, 0, st>>>(
-        (const __nv_bfloat16*)R, (const __nv_bfloat16*)L, M, s);
-  else
-    gen_materialise_kernel<float><<<grid, kGenThreads, 0, st>>>((const float*)R, (const float*)L,
-                                                                M, s);
-  return cudaGetLastError();
+    return launch_kernel(gen_materialise_kernel<__nv_bfloat16>, dim3(grid), dim3(kGenThreads), 0, st, false,
+                         (const __nv_bfloat16*)R, (const __nv_bfloat16*)L, M, s);
+  return launch_kernel(gen_materialise_kernel<float>, dim3(grid), dim3(kGenThreads), 0, st, false,
+                       (const float*)R, (const float*)L, M, s);
 }
 
 }  // namespace monarch

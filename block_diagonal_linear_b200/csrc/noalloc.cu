@@ -11,35 +11,25 @@
 //
 // The array lives at file scope as a __device__ variable, so every GPU on which
 // the library is loaded holds it until the process exits.  Host code cannot use
-// the array's name as a device address, so the address is looked up with
-// cudaGetSymbolAddress once per device, on the first call made with that device
-// current, and cached.
-#include <mutex>
-
+// the array's name as a device address, so every call looks the address up with
+// cudaGetSymbolAddress in the calling thread's current context.  The lookup is a
+// host-side query that allocates nothing; doing it per call (rather than caching
+// one address per device) keeps the address right after cudaDeviceReset or when
+// the caller runs in a context other than the device's primary one.
 #include "common.cuh"
 
 namespace {
 
 // Upper bound of the scratch this entry point can use (32 MiB).
 constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;
-constexpr int kMaxDevices = 64;
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
-std::mutex g_scratch_mutex;
-void* g_scratch_ptr[kMaxDevices] = {};
-
-// Device address of g_noalloc_scratch on the current device (nullptr on error).
-void* scratch_for_current_device() {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
-  std::lock_guard<std::mutex> lock(g_scratch_mutex);
-  if (g_scratch_ptr[dev] == nullptr) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return nullptr;
-    g_scratch_ptr[dev] = p;
-  }
-  return g_scratch_ptr[dev];
+// Device address of g_noalloc_scratch in the current context (nullptr on error).
+void* scratch_for_current_context() {
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) return nullptr;
+  return p;
 }
 
 }  // namespace
@@ -51,7 +41,7 @@ int monarch_bwd_noalloc(const void* dY, const void* X, const void* R, const void
   const int rc = monarch_validate(d);
   if (rc != MONARCH_OK) return rc;
   if (monarch_bwd_workspace_bytes(d) > kNoAllocScratchBytes) return MONARCH_ERR_SCRATCH;
-  void* scratch = scratch_for_current_device();
+  void* scratch = scratch_for_current_context();
   if (scratch == nullptr) return MONARCH_ERR_CUDA;
   return monarch_bwd(dY, X, R, L, d, dX, dR, dL, scratch, kNoAllocScratchBytes, stream);
 }

@@ -49,6 +49,16 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, in
   }
 }
 
+// Wait for the MMA issuer's final commit (every MMA of this CTA has completed).  A wait that runs
+// out records the timeout like wait_or_abort does, so the host sees MONARCH_ERR_TIMEOUT instead of
+// an incomplete result with status OK.
+__device__ __forceinline__ void wait_mma_done(uint64_t* bar, int* abort_flag, int* status) {
+  if (!ptx::mbar_wait_bounded(bar, 0, kWaitLimitNs)) {
+    *(volatile int*)abort_flag = 1;
+    atomicExch(status, kStatusTimeout);
+  }
+}
+
 // Warp-uniform version: lane 0 waits, the outcome is broadcast to the warp.
 __device__ __forceinline__ bool warp_wait_or_abort(int lane, uint64_t* bar, uint32_t parity,
                                                    int* abort_flag, int* status) {
@@ -88,25 +98,6 @@ inline bool make_map_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-// Launch `kernel` on `st`; with pdl = true it may begin launching while the previous kernel of
-// the stream is still running (programmatic stream serialization).  Every kernel launched this
-// way calls ptx::griddep_wait() before it touches global memory that earlier kernels write.
-template <typename... KArgs, typename... Args>
-inline cudaError_t launch_kernel(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
-                                 cudaStream_t st, bool pdl, Args... args) {
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = grid;
-  cfg.blockDim = block;
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = pdl ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, kernel, ((KArgs)args)...);
 }
 
 inline int num_sms() {

@@ -267,7 +267,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       }
       // Teardown: wait for every issued MMA before TMEM is freed.
       ptx::mma_commit(&bars->mma_done);
-      ptx::mbar_wait_bounded(&bars->mma_done, 0, kWaitLimitNs);
+      wait_mma_done(&bars->mma_done, &bars->abort_flag, status);
     }
   } else {
     // ================================================================ TMEM drain (rows)
@@ -435,15 +435,11 @@ static cudaError_t launch_tc_fwd(const void* X, const void* R, const void* L, vo
   const int64_t units_rounded = ((nunits + C::NGROUPS - 1) / C::NGROUPS) * C::NGROUPS;
   if (grid > units_rounded) grid = units_rounded;
   if (grid < C::NGROUPS) grid = C::NGROUPS;
-  tc_fwd_kernel<C><<<(unsigned)grid, kTcThreads, C::SMEM_BYTES, st>>>(
-      mX, mR, mL, (__nv_bfloat16*)Y, s.rows, status);
-  return cudaGetLastError();
+  return launch_kernel(tc_fwd_kernel<C>, dim3((unsigned)grid), dim3(kTcThreads), C::SMEM_BYTES, st, false,
+                       mX, mR, mL, (__nv_bfloat16*)Y, s.rows, status);
 }
 
-// Instantiated shapes (nb1, in1, out1, nb2, in2, out2, out_transpose, G).
-using CfgSq16 = FwdCfg<16, 16, 16, 16, 16, 16, 1, 16>;      // n = 256 = 16^2
-using CfgSq32 = FwdCfg<32, 32, 32, 32, 32, 32, 1, 16>;      // n = 1024 = 32^2
-using CfgR768 = FwdCfg<16, 48, 48, 48, 16, 64, 1, 16>;      // 768 -> 3072
+// Instantiated shape (nb1, in1, out1, nb2, in2, out2, out_transpose, G).
 using CfgNb4 = FwdCfg<4, 256, 256, 4, 256, 1024, 0, 1>;     // nblocks = 4, 1024 -> 4096
 
 template <class C>
@@ -453,15 +449,11 @@ static bool shape_is(const Shape& s) {
 }
 
 bool tc_fwd_supported(const Shape& s) {
-  return shape_is<CfgSq16>(s) || shape_is<CfgSq32>(s) || shape_is<CfgR768>(s) ||
-         shape_is<CfgNb4>(s);
+  return shape_is<CfgNb4>(s);
 }
 
 cudaError_t tc_fwd(const void* X, const void* R, const void* L, void* Y, const Shape& s,
                    int* status, cudaStream_t st) {
-  if (shape_is<CfgSq16>(s)) return launch_tc_fwd<CfgSq16>(X, R, L, Y, s, status, st);
-  if (shape_is<CfgSq32>(s)) return launch_tc_fwd<CfgSq32>(X, R, L, Y, s, status, st);
-  if (shape_is<CfgR768>(s)) return launch_tc_fwd<CfgR768>(X, R, L, Y, s, status, st);
   if (shape_is<CfgNb4>(s)) return launch_tc_fwd<CfgNb4>(X, R, L, Y, s, status, st);
   return cudaErrorNotSupported;
 }

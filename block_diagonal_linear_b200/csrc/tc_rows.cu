@@ -240,7 +240,7 @@ __global__ void __launch_bounds__(kRowsThreads, 1)
       }
     }
     ptx::mma_commit_elect(&bars->mma_done);
-    if (lane == 0) ptx::mbar_wait_bounded(&bars->mma_done, 0, kWaitLimitNs);
+    if (lane == 0) wait_mma_done(&bars->mma_done, abort_flag, status);
     __syncwarp();
   } else if (warp >= 2 + kRowsDrainWarps) {
     // ================================================================ weight loaders
@@ -281,7 +281,7 @@ __global__ void __launch_bounds__(kRowsThreads, 1)
         ptx::cp_async_mbar_arrive_noinc(&bars->full[st]);
       }
     }
-    ptx::cp_async_wait<0>();  // no copy may still target this CTA's shared memory at exit
+    ptx::cp_async_wait_all();  // no copy may still target this CTA's shared memory at exit
   } else {
     // ================================================================ drain (8 warps)
     const int quad = warp & 3;              // TMEM lane quadrant of this warp

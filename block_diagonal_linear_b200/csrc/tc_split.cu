@@ -147,7 +147,7 @@ __global__ void __launch_bounds__(kBdThreads, 1)
       ptx::mma_commit_elect(&bars->acc_full[slot]);
     }
     ptx::mma_commit_elect(&bars->mma_done);
-    if (lane == 0) ptx::mbar_wait_bounded(&bars->mma_done, 0, kWaitLimitNs);
+    if (lane == 0) wait_mma_done(&bars->mma_done, abort_flag, status);
     __syncwarp();
   } else {
     // ================================================================ drain (4 warps, one row per thread)

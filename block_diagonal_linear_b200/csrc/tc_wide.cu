@@ -207,7 +207,7 @@ __global__ void __launch_bounds__(kWideThreads, 1)
       }
     }
     ptx::mma_commit_elect(&bars->mma_done);
-    if (lane == 0) ptx::mbar_wait_bounded(&bars->mma_done, 0, kWaitLimitNs);
+    if (lane == 0) wait_mma_done(&bars->mma_done, abort_flag, status);
     __syncwarp();
   } else if (warp >= 2 + kWideDrainWarps) {
     // ================================================================ factor loaders
@@ -246,7 +246,7 @@ __global__ void __launch_bounds__(kWideThreads, 1)
     }
     // no copy may still target this CTA's shared memory at exit: the copies were never
     // committed to a group (the mbarrier tracks them), so commit and wait for all of them
-    asm volatile("cp.async.wait_all;" ::: "memory");
+    ptx::cp_async_wait_all();
   } else {
     // ================================================================ drain (8 warps)
     const int quad = warp & 3, ph = (warp - 2) >> 2, half = lane >> 4;
@@ -380,9 +380,8 @@ static cudaError_t launch_wide(const void* X, const void* R, const void* L, void
   if (e != cudaSuccess) return e;
   const int64_t nunits = (rows + bm - 1) / bm;
   const int64_t grid = nunits < nsm ? nunits : nsm;
-  tc_wide_kernel<C><<<(unsigned)grid, kWideThreads, C::SMEM_BYTES, st>>>(
-      mX, mY, (const __nv_bfloat16*)R, (const __nv_bfloat16*)L, rows, bm, status);
-  return cudaGetLastError();
+  return launch_kernel(tc_wide_kernel<C>, dim3((unsigned)grid), dim3(kWideThreads), C::SMEM_BYTES, st, false,
+                       mX, mY, (const __nv_bfloat16*)R, (const __nv_bfloat16*)L, rows, bm, status);
 }
 
 using WideR768 = WideCfg<16, 48, 48, 48, 16, 64>;  // 768 -> 3072

@@ -109,3 +109,29 @@ def make_integer_inputs(w: dict, seed: int = 0, rows: int | None = None, vmax: i
     L = rng.integers(-vmax, vmax + 1, size=(w["nb2"], w["out2"], w["in2"])).astype(np.float64)
     dY = rng.integers(-vmax, vmax + 1, size=(rows, n_out)).astype(np.float64)
     return {"X": X, "R": R, "L": L, "dY": dY}
+
+
+def sparse_sign_blocks(rng, nb: int, out_b: int, in_b: int, nnz: int) -> np.ndarray:
+    """(nb, out_b, in_b) blocks whose rows each hold `nnz` draws of +-1 at random columns
+    (draws may land on the same column, giving 0 or +-2 there)."""
+    W = np.zeros((nb, out_b, in_b), dtype=np.float64)
+    for b in range(nb):
+        for o in range(out_b):
+            cols = rng.integers(0, in_b, size=nnz)
+            signs = rng.choice([-1.0, 1.0], size=nnz)
+            np.add.at(W[b, o], cols, signs)
+    return W
+
+
+def make_sparse_sign_inputs(w: dict, seed: int = 0, rows: int | None = None, nnz: int = 2):
+    """Inputs for exact-equality checks: X and dY in {-1, 0, 1} (zero with probability 1/2),
+    factor blocks from :func:`sparse_sign_blocks`.  Every row of a block has absolute sum
+    <= nnz, so every intermediate of the method stays a small integer; float64 arrays."""
+    rows = int(w["rows"] if rows is None else rows)
+    n_in, _, n_out = sizes(w)
+    rng = np.random.default_rng(seed)
+    X = rng.choice([-1.0, 0.0, 0.0, 1.0], size=(rows, n_in))
+    R = sparse_sign_blocks(rng, w["nb1"], w["out1"], w["in1"], nnz)
+    L = sparse_sign_blocks(rng, w["nb2"], w["out2"], w["in2"], nnz)
+    dY = rng.choice([-1.0, 0.0, 0.0, 1.0], size=(rows, n_out))
+    return {"X": X, "R": R, "L": L, "dY": dY}

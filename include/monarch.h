@@ -129,9 +129,11 @@ MONARCH_API int monarch_bwd(const void* dY, const void* X, const void* R, const 
  *     bf16 shape that is about 2000 rows; larger batches must use monarch_bwd).
  *   - Every GPU that loads the library holds the 32 MiB array until the process
  *     exits.
- *   - The first call made with a given device current looks up the array's device
- *     address (cudaGetSymbolAddress) and caches it; make that first call before
- *     any stream capture.
+ *   - Every call looks up the array's device address in the calling thread's
+ *     current context (cudaGetSymbolAddress, a host-side query), so the address
+ *     stays valid after cudaDeviceReset and in non-primary contexts.  The first
+ *     call on a device may also load the library's device code; make that first
+ *     call before any stream capture.
  *   - All calls share the one array and it keeps the previous call's contents
  *     (nothing in it needs to start at zero).  Calls whose execution overlaps on
  *     the GPU (different streams, or several host threads on one device) race on
@@ -167,6 +169,11 @@ MONARCH_API int monarch_last_device_status(void* stream);
  * Returns the launch status; read the outcome with
  * monarch_last_device_status(). */
 MONARCH_API int monarch_debug_wait_timeout(uint64_t timeout_ns, void* stream);
+
+/* Number of kernels this library has launched in this process (every device and
+ * stream), counted on the host at each successful launch.  Host-only; a caller
+ * reads it before and after a region to count that region's launches. */
+MONARCH_API uint64_t monarch_kernel_launches(void);
 
 /* Which kernel family monarch_fwd / monarch_bwd would run for this shape:
  * 0 = generic FMA kernels, 1 = tcgen05 fused kernel over (128-row tile, block

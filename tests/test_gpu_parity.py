@@ -124,8 +124,10 @@ def test_full_size_sampled_rows_and_directional_identities(name):
     check(np.array(lhs), np.array(rhs), w["dtype"], "directional dR/dL")
 
 
-@pytest.mark.parametrize("name", ["n1024_bf16", "r768x3072_bf16"])
+@pytest.mark.parametrize("name", ["n1024_bf16", "r768x3072_bf16", "n4096_bf16", "nblk4_1024x4096_bf16",
+                                  "nblk4_1024x4096_bf16_b1000"])
 def test_full_size_bwd_weight_grads_vs_oracle(name):
+    """Full workload size: every entry of dX, dR and dL against the fp64 oracle."""
     w = W[name]
     shape = synthetic.shape_of(w)
     inp = synthetic.make_inputs(w, seed=4)

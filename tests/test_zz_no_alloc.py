@@ -38,6 +38,8 @@ def _noalloc(d, shape, rows, dtype):
 
 @pytest.mark.parametrize("name,rows", [("n1024_bf16", 1024), ("n256_fp32", 64), ("n256_fp32", 301)])
 def test_noalloc_matches_workspace_entry_point_twice(name, rows):
+    """Both entry points run the same deterministic kernels, so their results must be
+    bitwise equal; the first call is also checked against the fp64 oracle."""
     w = synthetic.WORKLOADS[name]
     shape = synthetic.shape_of(w)
     assert bdl.bwd_workspace_bytes(shape, rows, w["dtype"]) <= (32 << 20)
@@ -49,8 +51,12 @@ def test_noalloc_matches_workspace_entry_point_twice(name, rows):
         ref = bdl.bwd(d["dY"], d["X"], d["R"], d["L"], shape)
         assert bdl.last_device_status() == 0
         for g, r, what in zip(got, ref, ("dX", "dR", "dL")):
-            err = oracle.normwise_rel_err(to_f64(g), to_f64(r))
-            assert err <= TOL[w["dtype"]], "%s seed %d: %.3e" % (what, seed, err)
+            assert torch.equal(g, r), "%s seed %d differs from monarch_bwd" % (what, seed)
+        if seed == 40:
+            want = oracle.backward(shape, inp["dY"].f64, inp["X"].f64, inp["R"].f64, inp["L"].f64)
+            for g, r, what in zip(got, want, ("dX", "dR", "dL")):
+                err = oracle.normwise_rel_err(to_f64(g), r)
+                assert err <= TOL[w["dtype"]], "%s vs oracle: %.3e" % (what, err)
 
 
 def test_noalloc_rejects_problems_beyond_its_scratch():
