@@ -6,6 +6,7 @@
 
 #include "common.cuh"
 #include "ptx.cuh"
+#include "tc_gemm.cuh"
 
 namespace monarch {
 
@@ -109,12 +110,24 @@ int monarch_fwd_path(const monarch_dims* d) {
   return fwd_path(to_shape(*d), d->dtype);
 }
 
+// 0 = generic FMA kernels, 1 = row-tile / block-GEMM passes with tcgen05 weight gradients,
+// 2 = tcgen05 GEMM passes (permutation folded into 64-column gathers), 3 = packed
+// block-diagonal tcgen05 GEMM passes with row-transpose passes for the permutations.
 static int bwd_path(const Shape& s, int dtype) {
-  return (dtype == MONARCH_BF16 && fast_bwd_supported(s)) ? 1 : 0;
+  if (dtype != MONARCH_BF16) return 0;
+  if (fast_bwd_supported(s)) return 1;
+  if (gemm_bwd_supported(s)) return 2;
+  if (packed_bwd_supported(s)) return 3;
+  return 0;
 }
 
 static size_t bwd_workspace(const Shape& s, int dtype) {
-  return bwd_path(s, dtype) == 1 ? fast_bwd_workspace(s) : generic_bwd_workspace(s);
+  switch (bwd_path(s, dtype)) {
+    case 1: return fast_bwd_workspace(s);
+    case 2: return gemm_bwd_workspace(s);
+    case 3: return packed_bwd_workspace(s);
+    default: return generic_bwd_workspace(s);
+  }
 }
 
 int monarch_bwd_path(const monarch_dims* d) {
@@ -174,10 +187,13 @@ int monarch_bwd(const void* dY, const void* X, const void* R, const void* L, con
                          span(R, s.n_R(), es), span(L, s.n_L(), es)})) != MONARCH_OK)
     return rc;
   cudaError_t e;
-  if (bwd_path(s, d->dtype) == 1) {
+  const int path = bwd_path(s, d->dtype);
+  if (path != 0) {
     int* status = status_ptr();
     if (status == nullptr) return MONARCH_ERR_CUDA;
-    e = fast_bwd(dY, X, R, L, dX, dR, dL, workspace, s, status, (cudaStream_t)stream);
+    e = path == 1   ? fast_bwd(dY, X, R, L, dX, dR, dL, workspace, s, status, (cudaStream_t)stream)
+        : path == 2 ? gemm_bwd(dY, X, R, L, dX, dR, dL, workspace, s, status, (cudaStream_t)stream)
+                    : packed_bwd(dY, X, R, L, dX, dR, dL, workspace, s, status, (cudaStream_t)stream);
   } else {
     if (!generic_bwd_supported(s)) return MONARCH_ERR_UNSUPPORTED;
     e = generic_bwd(dY, X, R, L, dX, dR, dL, workspace, s, d->dtype, (cudaStream_t)stream);

@@ -1,0 +1,365 @@
+// Backward on the generic tcgen05 GEMM (tc_gemm.cu), for shapes whose permutation P moves
+// whole 64-column groups: no output transpose, in2 a multiple of nb1, and in2 / nb1 (the
+// run of middle positions p that one L block takes from each R block) a multiple of 64 --
+// e.g. the nblocks = 4 layer 1024 -> 4096 (R: 4 blocks 256 x 256, L: 4 blocks 1024 x 256).
+//
+// Index facts used (notation of monarch.h; G = in2 / nb1):
+//   Z[j][q] = u[k][p]  with  q = p'*nb1 + k,  p = j*G + p'   (p' < G, k < nb1).
+// Reordering the K index of the L stage as kappa = k*G + p' turns Z_j into nb1 column ranges
+// u[k][j*G .. j*G + G) of the block-contiguous middle vector U, i.e. whole 64-column groups.
+// The same reordering applied to the rows of L^T makes the dual stage write dU directly.
+//
+//   1. Rt[k][i][p] = R[k][p][i];  Ltp[j][kappa][o] = L[j][o][q(kappa)]      (prep kernel)
+//   2. U  = blockdiag(R) X                   (GEMM, block-contiguous u[k][p])
+//   3. dU = blockdiag(Ltp) dY                 (GEMM; output groups scattered to u[k][p] order)
+//   4. dX = blockdiag(Rt) dU                  (GEMM)
+//   5. dR[k] = sum_rows dU_k^T X_k,  dL[j] = sum_rows dY_j^T Z_j   (weight-gradient GEMMs, rows
+//      as K, split into chunks; Z_j read from U through the same 64-column groups, its
+//      columns mapped back from kappa to q when the partials are written)
+//   6. dR, dL = fixed-order sum of the partials (reduce_partials_kernel)
+#include "common.cuh"
+#include "tc_common.cuh"
+#include "tc_gemm.cuh"
+
+namespace monarch {
+
+__global__ void reduce_partials_kernel(const float* __restrict__ partial, __nv_bfloat16* __restrict__ dR,
+                                       __nv_bfloat16* __restrict__ dL, int64_t nR, int64_t nP, int nsplit);
+
+static int pick_bn(int n) { return n % 256 == 0 ? 256 : (n % 128 == 0 ? 128 : 64); }
+
+bool gemm_bwd_supported(const Shape& s) {
+  if (s.out_transpose) return false;
+  if (s.in1 % 64 || s.out1 % 128 || s.out2 % 128 || s.in2 % s.nb1) return false;
+  const int G = s.in2 / s.nb1;
+  if (G % 64) return false;
+  if (s.nb1 * s.out1 != s.nb2 * s.in2) return false;
+  return s.n_in() <= (1 << 20) && s.n_out() <= (1 << 20);
+}
+
+// ---------------------------------------------------------------- prep
+__global__ void gemm_bwd_prep_kernel(const __nv_bfloat16* __restrict__ R, const __nv_bfloat16* __restrict__ L,
+                                     __nv_bfloat16* __restrict__ Rt, __nv_bfloat16* __restrict__ Ltp, Shape s) {
+  ptx::griddep_wait();
+  ptx::griddep_launch_dependents();
+  const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int64_t nR = s.n_R(), nL = s.n_L();
+  if (e < nR) {  // Rt[k][i][p] = R[k][p][i]
+    const int64_t k = e / ((int64_t)s.in1 * s.out1), rem = e % ((int64_t)s.in1 * s.out1);
+    const int i = (int)(rem / s.out1), p = (int)(rem % s.out1);
+    Rt[e] = R[(k * s.out1 + p) * s.in1 + i];
+  } else if (e < nR + nL) {  // Ltp[j][kappa][o] = L[j][o][q],  kappa = k*G + p',  q = p'*nb1 + k
+    const int64_t f = e - nR;
+    const int G = s.in2 / s.nb1;
+    const int64_t j = f / ((int64_t)s.in2 * s.out2), rem = f % ((int64_t)s.in2 * s.out2);
+    const int kappa = (int)(rem / s.out2), o = (int)(rem % s.out2);
+    const int q = (kappa % G) * s.nb1 + kappa / G;
+    Ltp[f] = L[(j * s.out2 + o) * s.in2 + q];
+  }
+}
+
+// ---------------------------------------------------------------- weight gradient
+// Split of the rows for the weight-gradient GEMMs: chunks of a multiple of 64 rows, enough of
+// them that both launches together give about two units per SM, but at least 512 rows each
+// (every chunk costs one fp32 copy of the parameters in partials), and none of them empty
+// (an empty chunk would leave its partials unwritten).
+WgradSplit wgrad_split(int64_t rows, int64_t units_per_split) {
+  int64_t n = (2 * 148 + units_per_split - 1) / (units_per_split > 0 ? units_per_split : 1);
+  const int64_t maxs = rows / 512;
+  if (n > maxs) n = maxs;
+  if (n < 1) n = 1;
+  WgradSplit w;
+  const int64_t per = (rows + n - 1) / n;
+  w.rows_per_split = ((per + 63) / 64) * 64;
+  if (w.rows_per_split < 64) w.rows_per_split = 64;
+  w.nsplit = (int)((rows + w.rows_per_split - 1) / w.rows_per_split);
+  if (w.nsplit < 1) w.nsplit = 1;
+  return w;
+}
+
+// dW[b][m][n] = sum_rows A1[r][b*blk_a + m] * gathered(A2)[r][b*blk_b + n] as fp32 partials.
+// A1 is block-contiguous with blocks of blk_a columns; A2's block b occupies the logical
+// columns [b*blk_b, (b+1)*blk_b).  With b_grp = 0, A2 is block-contiguous too; otherwise its
+// 64-column groups are gathered: group g of block b starts at b*b_base + (g / b_grp)*b_gs +
+// (g % b_grp)*64, and the in-block logical column n maps back to (n % pm_a)*pm_b + n / pm_a.
+cudaError_t wgrad_tc(const void* A1, int64_t a_cols, int64_t blk_a, const void* A2, int64_t b_cols, int64_t blk_b,
+                     int64_t nblocks, int b_base, int b_grp, int b_gs, int64_t pm_a, int64_t pm_b, int64_t rows,
+                     WgradSplit sp, float* partial, int64_t p_stride, int64_t p_off, int* status, cudaStream_t st) {
+  GemmJob j = {};
+  // M side: a group of 128 columns of A1 holding bpg whole blocks, or one block per group in
+  // 128-row tiles (rows of a tile beyond the block belong to the next block and are dropped)
+  int64_t bpg = 1;  // blocks per group
+  if (blk_a <= 128 && 128 % blk_a == 0 && nblocks % (128 / blk_a) == 0) bpg = 128 / blk_a;
+  j.mtiles = (int)((blk_a + 127) / 128);
+  const int64_t nw = bpg * blk_b;  // B columns a group needs
+  const int BN = nw >= 256 ? 256 : (nw > 64 ? 128 : 64);
+  if ((bpg * blk_a) % 8 || (bpg * b_base) % 8 || nw % 8) return cudaErrorInvalidValue;  // 16-byte TMA x
+  j.nb = (int)(nblocks / bpg);
+  j.ntiles = (int)((nw + BN - 1) / BN);
+  j.nsplit = sp.nsplit;
+  j.split_rows = sp.rows_per_split;
+  j.a_b = (int)(bpg * blk_a);
+  j.b_lb = (int)nw;
+  if (b_grp == 0) {  // contiguous
+    j.b_b = (int)nw;
+    j.b_grp = 1 << 30;
+    j.b_gs = 0;
+  } else {
+    j.b_b = (int)(bpg * b_base);
+    j.b_grp = b_grp;
+    j.b_gs = b_gs;
+  }
+  j.blk_a = blk_a;
+  j.blk_b = blk_b;
+  j.pm_a = pm_a;
+  j.pm_b = pm_b;
+  j.p_stride = p_stride;
+  j.p_off = p_off;
+  return gemm_wgrad(A1, a_cols, A2, b_cols, rows, BN, j, partial, status, st, true);
+}
+
+// ---------------------------------------------------------------- host
+static size_t al256(size_t b) { return (b + 255) & ~size_t(255); }
+
+struct GemmBwdWs {
+  size_t rt, ltp, u, du, part, total;
+  WgradSplit sp;
+};
+
+static int64_t gemm_bwd_units_per_split(const Shape& s) {
+  // dR: nb1 groups x out1/128 m tiles x in1/BN n tiles; dL: nb2 x out2/128 x in2/BN
+  const int bn1 = s.in1 >= 256 ? 256 : (s.in1 > 64 ? 128 : 64);
+  const int bn2 = s.in2 >= 256 ? 256 : (s.in2 > 64 ? 128 : 64);
+  return (int64_t)s.nb1 * (s.out1 / 128) * ((s.in1 + bn1 - 1) / bn1) +
+         (int64_t)s.nb2 * (s.out2 / 128) * ((s.in2 + bn2 - 1) / bn2);
+}
+
+static GemmBwdWs gemm_bwd_layout(const Shape& s) {
+  GemmBwdWs w;
+  const size_t nR = (size_t)s.n_R(), nL = (size_t)s.n_L();
+  w.sp = wgrad_split(s.rows, gemm_bwd_units_per_split(s));
+  w.rt = 0;
+  w.ltp = w.rt + al256(nR * 2);
+  w.u = w.ltp + al256(nL * 2);
+  w.du = w.u + al256((size_t)s.rows * (size_t)s.n_mid() * 2);
+  w.part = w.du + al256((size_t)s.rows * (size_t)s.n_mid() * 2);
+  w.total = w.part + al256((size_t)w.sp.nsplit * (nR + nL) * 4);
+  return w;
+}
+
+size_t gemm_bwd_workspace(const Shape& s) { return gemm_bwd_layout(s).total; }
+
+cudaError_t gemm_bwd(const void* dY, const void* X, const void* R, const void* L, void* dX, void* dR, void* dL,
+                     void* ws, const Shape& s, int* status, cudaStream_t st) {
+  const GemmBwdWs w = gemm_bwd_layout(s);
+  char* base = (char*)ws;
+  __nv_bfloat16* Rt = (__nv_bfloat16*)(base + w.rt);
+  __nv_bfloat16* Ltp = (__nv_bfloat16*)(base + w.ltp);
+  __nv_bfloat16* U = (__nv_bfloat16*)(base + w.u);
+  __nv_bfloat16* dU = (__nv_bfloat16*)(base + w.du);
+  float* part = (float*)(base + w.part);
+  const int64_t nR = s.n_R(), nL = s.n_L(), nP = nR + nL;
+  const int G = s.in2 / s.nb1;
+  cudaError_t e;
+  if ((e = launch_kernel(gemm_bwd_prep_kernel, dim3((unsigned)((nP + 255) / 256)), dim3(256), 0, st, true,
+                         (const __nv_bfloat16*)R, (const __nv_bfloat16*)L, Rt, Ltp, s)) != cudaSuccess)
+    return e;
+  if (s.rows > 0) {
+    // 2. U = blockdiag(R) X
+    GemmJob j = {};
+    int bn = pick_bn(s.out1);
+    j.nb = s.nb1; j.ntiles = s.out1 / bn; j.kboxes = s.in1 / 64;
+    j.a_b = s.in1; j.a_grp = s.in1 / 64; j.a_gs = 0;
+    j.b_b = s.out1;
+    j.y_b = s.out1; j.y_grp = s.out1 / 64; j.y_gs = 0;
+    if ((e = gemm_bd(X, s.rows, s.n_in(), R, (int64_t)s.nb1 * s.out1, s.in1, U, s.n_mid(), bn, j, status, st,
+                     true)) != cudaSuccess)
+      return e;
+    // 3. dU = blockdiag(Ltp) dY, output group g of block j -> u[k][j*G + 64*(g % (G/64))], k = g / (G/64)
+    j = GemmJob{};
+    bn = pick_bn(s.in2);
+    j.nb = s.nb2; j.ntiles = s.in2 / bn; j.kboxes = s.out2 / 64;
+    j.a_b = s.out2; j.a_grp = s.out2 / 64; j.a_gs = 0;
+    j.b_b = s.in2;
+    j.y_b = G; j.y_grp = G / 64; j.y_gs = s.out1;
+    if ((e = gemm_bd(dY, s.rows, s.n_out(), Ltp, (int64_t)s.nb2 * s.in2, s.out2, dU, s.n_mid(), bn, j, status,
+                     st, true)) != cudaSuccess)
+      return e;
+    // 4. dX = blockdiag(Rt) dU
+    j = GemmJob{};
+    bn = pick_bn(s.in1);
+    j.nb = s.nb1; j.ntiles = s.in1 / bn; j.kboxes = s.out1 / 64;
+    j.a_b = s.out1; j.a_grp = s.out1 / 64; j.a_gs = 0;
+    j.b_b = s.in1;
+    j.y_b = s.in1; j.y_grp = s.in1 / 64; j.y_gs = 0;
+    if ((e = gemm_bd(dU, s.rows, s.n_mid(), Rt, (int64_t)s.nb1 * s.in1, s.out1, dX, s.n_in(), bn, j, status, st,
+                     true)) != cudaSuccess)
+      return e;
+    // 5. weight gradients
+    if ((e = wgrad_tc(dU, s.n_mid(), s.out1, X, s.n_in(), s.in1, s.nb1, 0, 0, 0, s.in1, 1, s.rows,
+                      w.sp, part, nP, 0, status, st)) != cudaSuccess)
+      return e;
+    if ((e = wgrad_tc(dY, s.n_out(), s.out2, U, s.n_mid(), s.in2, s.nb2, G, G / 64, s.out1, G, s.nb1, s.rows,
+                      w.sp, part, nP, nR, status, st)) != cudaSuccess)
+      return e;
+  } else {
+    if ((e = cudaMemsetAsync(part, 0, sizeof(float) * (size_t)w.sp.nsplit * (size_t)nP, st)) != cudaSuccess) return e;
+  }
+  return launch_kernel(reduce_partials_kernel, dim3((unsigned)((nP + 255) / 256)), dim3(256), 0, st, true,
+                       (const float*)part, (__nv_bfloat16*)dR, (__nv_bfloat16*)dL, nR, nP, w.sp.nsplit);
+}
+
+// ================================================================ packed block-diagonal path
+// Any bf16 shape whose small blocks pack into 64-multiples: g consecutive blocks of a
+// block-diagonal stage are one GEMM against a (g*N) x (g*K) block-diagonal weight tile with
+// zeros off the diagonal (g times the flops, which the tensor cores have to spare on these
+// memory-bound shapes).  The permutations are per-row transposes:
+//   dV = P_out^-1 dY,  dZ = packed(L^T) dV,  dU = P^-1 dZ,  dX = packed(R^T) dU,
+//   U = packed(R) X,  Z = P U,  then the weight-gradient GEMMs and the partial sum.
+static int pack_factor(int nblocks, int kw, int nw) {
+  for (int g = 1; g <= 8; ++g)
+    if (nblocks % g == 0 && (g * kw) % 64 == 0 && (g * nw) % 64 == 0) return g;
+  return 0;
+}
+
+struct PackInfo {
+  int gz, gx;  // blocks per packed group: L^T stage (K = out2, N = in2), R / R^T stages
+};
+static PackInfo pack_info(const Shape& s) {
+  PackInfo p;
+  p.gz = pack_factor(s.nb2, s.out2, s.in2);
+  const int a = pack_factor(s.nb1, s.in1, s.out1), b = pack_factor(s.nb1, s.out1, s.in1);
+  p.gx = a > b ? a : b;
+  if (p.gx && (s.nb1 % p.gx || (p.gx * s.in1) % 64 || (p.gx * s.out1) % 64)) p.gx = 0;
+  return p;
+}
+
+bool packed_bwd_supported(const Shape& s) {
+  const PackInfo p = pack_info(s);
+  if (p.gz == 0 || p.gx == 0) return false;
+  // the row-transpose passes move 16-byte chunks (8 elements of one grid row)
+  if (s.nb1 % 8 || s.out1 % 8 || (s.out_transpose && (s.nb2 % 8 || s.out2 % 8))) return false;
+  // packed operand widths (K stages of 64, N tiles of 64..256) and the row-transpose passes
+  if ((int64_t)p.gz * s.out2 > 4096 || (int64_t)p.gx * s.in1 > 4096 || (int64_t)p.gx * s.out1 > 4096) return false;
+  if (s.n_in() > 65536 || s.n_mid() > 65536 || s.n_out() > 65536) return false;
+  if ((int64_t)8 * s.out2 * (s.nb2 + 2) * 2 > 200 * 1024 || (int64_t)8 * s.nb1 * (s.out1 + 2) * 2 > 200 * 1024 ||
+      (int64_t)8 * s.out1 * (s.nb1 + 2) * 2 > 200 * 1024)
+    return false;
+  return true;
+}
+
+// Wz[g][jj*in2 + q][jj'*out2 + o] = L[g*gz + jj][o][q] if jj == jj'  (dZ = Wz-stage of dV)
+// Wx[g][kk*in1 + i][kk'*out1 + p] = R[g*gx + kk][p][i]                (dX = Wx-stage of dU)
+// Wu[g][kk*out1 + p][kk'*in1 + i] = R[g*gx + kk][p][i]                (U  = Wu-stage of X)
+__global__ void pack_weights_kernel(const __nv_bfloat16* __restrict__ R, const __nv_bfloat16* __restrict__ L,
+                                    __nv_bfloat16* __restrict__ Wz, __nv_bfloat16* __restrict__ Wx,
+                                    __nv_bfloat16* __restrict__ Wu, Shape s, int gz, int gx) {
+  ptx::griddep_wait();
+  ptx::griddep_launch_dependents();
+  const int64_t nz = (int64_t)s.nb2 * s.in2 * gz * s.out2;
+  const int64_t nx = (int64_t)s.nb1 * s.in1 * gx * s.out1;
+  const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const __nv_bfloat16 zero = __float2bfloat16_rn(0.f);
+  if (e < nz) {
+    const int64_t kw = (int64_t)gz * s.out2, n = e / kw, k = e % kw;  // n = g*gz*in2 + jj*in2 + q
+    const int64_t g = n / ((int64_t)gz * s.in2), nn = n % ((int64_t)gz * s.in2);
+    const int jj = (int)(nn / s.in2), q = (int)(nn % s.in2), jk = (int)(k / s.out2), o = (int)(k % s.out2);
+    Wz[e] = jj == jk ? L[((g * gz + jj) * s.out2 + o) * s.in2 + q] : zero;
+  } else if (e < nz + nx) {
+    const int64_t f = e - nz, kw = (int64_t)gx * s.out1, n = f / kw, k = f % kw;
+    const int64_t g = n / ((int64_t)gx * s.in1), nn = n % ((int64_t)gx * s.in1);
+    const int kk = (int)(nn / s.in1), i = (int)(nn % s.in1), kq = (int)(k / s.out1), p = (int)(k % s.out1);
+    Wx[f] = kk == kq ? R[((g * gx + kk) * s.out1 + p) * s.in1 + i] : zero;
+  } else if (e < nz + 2 * nx) {
+    const int64_t f = e - nz - nx, kw = (int64_t)gx * s.in1, n = f / kw, k = f % kw;
+    const int64_t g = n / ((int64_t)gx * s.out1), nn = n % ((int64_t)gx * s.out1);
+    const int kk = (int)(nn / s.out1), p = (int)(nn % s.out1), kq = (int)(k / s.in1), i = (int)(k % s.in1);
+    Wu[f] = kk == kq ? R[((g * gx + kk) * s.out1 + p) * s.in1 + i] : zero;
+  }
+}
+
+struct PackedWs {
+  size_t wz, wx, wu, dv, dz, du, u, z, part, total;
+  WgradSplit sp;
+};
+
+static int64_t wgrad_units(int64_t nblocks, int64_t blk_a, int64_t blk_b) {
+  int64_t bpg = 1;
+  if (blk_a <= 128 && 128 % blk_a == 0 && nblocks % (128 / blk_a) == 0) bpg = 128 / blk_a;
+  const int64_t nw = bpg * blk_b;
+  const int64_t bn = nw >= 256 ? 256 : (nw > 64 ? 128 : 64);
+  return (nblocks / bpg) * ((blk_a + 127) / 128) * ((nw + bn - 1) / bn);
+}
+
+static PackedWs packed_layout(const Shape& s) {
+  const PackInfo pk = pack_info(s);
+  PackedWs w;
+  const size_t rows = (size_t)s.rows;
+  w.sp = wgrad_split(s.rows, wgrad_units(s.nb1, s.out1, s.in1) + wgrad_units(s.nb2, s.out2, s.in2));
+  w.wz = 0;
+  w.wx = w.wz + al256((size_t)s.nb2 * s.in2 * pk.gz * s.out2 * 2);
+  w.wu = w.wx + al256((size_t)s.nb1 * s.in1 * pk.gx * s.out1 * 2);
+  w.dv = w.wu + al256((size_t)s.nb1 * s.in1 * pk.gx * s.out1 * 2);
+  w.dz = w.dv + (s.out_transpose ? al256(rows * (size_t)s.n_out() * 2) : 0);
+  w.du = w.dz + al256(rows * (size_t)s.n_mid() * 2);
+  w.u = w.du + al256(rows * (size_t)s.n_mid() * 2);
+  w.z = w.u + al256(rows * (size_t)s.n_mid() * 2);
+  w.part = w.z + al256(rows * (size_t)s.n_mid() * 2);
+  w.total = w.part + al256((size_t)w.sp.nsplit * (size_t)(s.n_R() + s.n_L()) * 4);
+  return w;
+}
+
+size_t packed_bwd_workspace(const Shape& s) { return packed_layout(s).total; }
+
+// Y (rows x nb*nw) = packed block-diagonal stage of A (rows x nb*kw) with W (nb*nw x g*kw per group).
+static cudaError_t packed_stage(const void* A, int64_t rows, const void* W, void* Y, int nb, int kw, int nw, int g,
+                                int* status, cudaStream_t st) {
+  GemmJob j = {};
+  const int K = g * kw, N = g * nw;
+  const int bn = pick_bn(N);
+  j.nb = nb / g; j.ntiles = N / bn; j.kboxes = K / 64;
+  j.a_b = K; j.a_grp = 1 << 30; j.a_gs = 0;
+  j.b_b = N;
+  j.y_b = N; j.y_grp = 1 << 30; j.y_gs = 0;
+  return gemm_bd(A, rows, (int64_t)nb * kw, W, (int64_t)nb * nw, K, Y, (int64_t)nb * nw, bn, j, status, st, true);
+}
+
+cudaError_t packed_bwd(const void* dY, const void* X, const void* R, const void* L, void* dX, void* dR, void* dL,
+                       void* ws, const Shape& s, int* status, cudaStream_t st) {
+  const PackInfo pk = pack_info(s);
+  const PackedWs w = packed_layout(s);
+  char* base = (char*)ws;
+  __nv_bfloat16 *Wz = (__nv_bfloat16*)(base + w.wz), *Wx = (__nv_bfloat16*)(base + w.wx),
+                *Wu = (__nv_bfloat16*)(base + w.wu);
+  __nv_bfloat16* dV = s.out_transpose ? (__nv_bfloat16*)(base + w.dv) : (__nv_bfloat16*)dY;
+  __nv_bfloat16 *dZ = (__nv_bfloat16*)(base + w.dz), *dU = (__nv_bfloat16*)(base + w.du),
+                *U = (__nv_bfloat16*)(base + w.u), *Z = (__nv_bfloat16*)(base + w.z);
+  float* part = (float*)(base + w.part);
+  const int64_t nR = s.n_R(), nL = s.n_L(), nP = nR + nL;
+  const int64_t nz = (int64_t)s.nb2 * s.in2 * pk.gz * s.out2, nx = (int64_t)s.nb1 * s.in1 * pk.gx * s.out1;
+  cudaError_t e;
+  if ((e = launch_kernel(pack_weights_kernel, dim3((unsigned)((nz + 2 * nx + 255) / 256)), dim3(256), 0, st, true,
+                         (const __nv_bfloat16*)R, (const __nv_bfloat16*)L, Wz, Wx, Wu, s, pk.gz, pk.gx)) !=
+      cudaSuccess)
+    return e;
+  if (s.rows > 0) {
+    if (s.out_transpose && (e = permute_rows(dY, dV, s.rows, s.out2, s.nb2, st)) != cudaSuccess) return e;
+    if ((e = packed_stage(dV, s.rows, Wz, dZ, s.nb2, s.out2, s.in2, pk.gz, status, st)) != cudaSuccess) return e;
+    if ((e = permute_rows(dZ, dU, s.rows, s.out1, s.nb1, st)) != cudaSuccess) return e;
+    if ((e = packed_stage(dU, s.rows, Wx, dX, s.nb1, s.out1, s.in1, pk.gx, status, st)) != cudaSuccess) return e;
+    if ((e = packed_stage(X, s.rows, Wu, U, s.nb1, s.in1, s.out1, pk.gx, status, st)) != cudaSuccess) return e;
+    if ((e = permute_rows(U, Z, s.rows, s.nb1, s.out1, st)) != cudaSuccess) return e;
+    if ((e = wgrad_tc(dU, s.n_mid(), s.out1, X, s.n_in(), s.in1, s.nb1, 0, 0, 0, s.in1, 1, s.rows, w.sp, part, nP, 0,
+                      status, st)) != cudaSuccess)
+      return e;
+    if ((e = wgrad_tc(dV, s.n_out(), s.out2, Z, s.n_mid(), s.in2, s.nb2, 0, 0, 0, s.in2, 1, s.rows, w.sp, part, nP,
+                      nR, status, st)) != cudaSuccess)
+      return e;
+  } else if ((e = cudaMemsetAsync(part, 0, sizeof(float) * (size_t)w.sp.nsplit * (size_t)nP, st)) != cudaSuccess) {
+    return e;
+  }
+  return launch_kernel(reduce_partials_kernel, dim3((unsigned)((nP + 255) / 256)), dim3(256), 0, st, true,
+                       (const float*)part, (__nv_bfloat16*)dR, (__nv_bfloat16*)dL, nR, nP, w.sp.nsplit);
+}
+
+}  // namespace monarch

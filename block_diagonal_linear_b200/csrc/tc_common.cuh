@@ -25,6 +25,19 @@ __device__ __forceinline__ uint64_t make_sdesc(uint32_t saddr, uint32_t sbo_byte
   return d;
 }
 
+// Same with an explicit leading byte offset (MN-major swizzled layouts: the byte distance
+// between consecutive 64-element M/N blocks).
+__device__ __forceinline__ uint64_t make_sdesc_lbo(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes,
+                                                   uint32_t swz) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFF);
+  d |= (uint64_t)((lbo_bytes >> 4) & 0x3FFF) << 16;
+  d |= (uint64_t)((sbo_bytes >> 4) & 0x3FFF) << 32;
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)swz << 61;
+  return d;
+}
+
 // Instruction descriptor: kind::f16, A = B = bf16, D = fp32, both K-major.
 __host__ __device__ constexpr uint32_t make_idesc(int M, int N) {
   return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) |

@@ -1,0 +1,339 @@
+// Generic tcgen05 GEMM for the Monarch passes that are (batched, gathered) GEMMs:
+//
+//   D[m][n] = sum_k A[m][k] * B[n][k]     128 x BN tiles, bf16 operands, fp32 in TMEM.
+//
+// Two kinds of job share the kernel:
+//   kind 0, block-diagonal stage (K-major operands): A is a row tile of an activation
+//     matrix (rows x cols, K contiguous), B a weight block W[b] (N x K, the nn.Linear
+//     layout); D is rounded to bf16 and written with TMA stores into a column range of
+//     the output.  The A columns of one unit may be gathered from several 64-column
+//     groups (col = b*a_b + (kb / a_grp)*a_gs + (kb % a_grp)*64), which lets a stage read
+//     its input through a permutation whose groups are 64 columns wide without a pass
+//     over memory.
+//   kind 1, weight gradient (MN-major operands, rows of the activations are K): for a
+//     group of blocks, A = act1[rows][cols] and B = act2[rows][cols], so
+//     D[m][n] = sum_r act1[r][m] act2[r][n]; the rows are split into chunks (split-K) and
+//     each unit writes the diagonal blocks of D (m and n in the same block) as fp32
+//     partials, summed in a fixed order by a separate kernel.
+// Roles: warp 0 TMA producer, warp 1 MMA issuer and TMEM owner, warps 2..5 epilogue
+// (one TMEM lane quadrant each: one D row per thread).  Operands move by TMA with 128B
+// swizzle into a ring of stages; two TMEM accumulator slots let the epilogue of one unit
+// overlap the MMAs of the next.  All waits are bounded (tc_common.cuh).
+#include "tc_common.cuh"
+#include "tc_gemm.cuh"
+
+namespace monarch {
+
+constexpr int kGemmThreads = 192;
+constexpr int kGemmEpiWarps = 4;
+
+template <int BN_, int KIND_>
+struct GemmCfg {
+  static constexpr int BN = BN_, KIND = KIND_;
+  static constexpr int BM = 128;
+  static constexpr int A_BYTES = BM * 128;          // 128 x 64 bf16 (K-major) or 2 x (64 x 64) (MN-major)
+  static constexpr int B_BYTES = BN * 128;          // BN x 64 (K-major) or BN/64 x (64 x 64) (MN-major)
+  static constexpr int STAGE = A_BYTES + B_BYTES;
+  static constexpr int STG_BYTES = KIND == 0 ? 2 * BM * 128 : 0;  // two 128 x 64 output chunks
+  static constexpr int TMEM_COLS = 2 * BN <= 32 ? 32 : (2 * BN <= 64 ? 64 : (2 * BN <= 128 ? 128 : (2 * BN <= 256 ? 256 : 512)));
+  static constexpr int NSTAGE_RAW = (kSmemBudget - STG_BYTES - 1024) / STAGE;
+  static constexpr int NSTAGE = NSTAGE_RAW > 8 ? 8 : NSTAGE_RAW;
+  static constexpr int SMEM_BYTES = STG_BYTES + NSTAGE * STAGE + 1024 + 1024;
+  static_assert(BN % 64 == 0 && BN <= 256, "BN");
+  static_assert(NSTAGE >= 2, "shared memory");
+};
+
+struct GemmBars {
+  uint64_t full[8], empty[8];
+  uint64_t acc_full[2], acc_empty[2];
+  uint64_t mma_done;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+// Unit index -> coordinates.  Kind 0: n tile fastest, then batch, then m tile (the units of
+// one row tile run together, so its A tile is re-read from L2).  Kind 1: m, n tiles, then
+// group, then split.
+struct UnitCoord {
+  int b, mt, nt, split;
+};
+__device__ __forceinline__ UnitCoord unit_coord(const GemmJob& j, int64_t u) {
+  UnitCoord c;
+  c.nt = (int)(u % j.ntiles);
+  u /= j.ntiles;
+  if (j.kind == 0) {
+    c.b = (int)(u % j.nb);
+    c.mt = (int)(u / j.nb);
+    c.split = 0;
+  } else {
+    c.mt = (int)(u % j.mtiles);
+    u /= j.mtiles;
+    c.b = (int)(u % j.nb);
+    c.split = (int)(u / j.nb);
+  }
+  return c;
+}
+
+// Number of 64-wide K stages of a unit.
+__device__ __forceinline__ int unit_kstages(const GemmJob& j, const UnitCoord& c) {
+  if (j.kind == 0) return j.kboxes;
+  const int64_t r0 = (int64_t)c.split * j.split_rows;
+  int64_t n = j.rows - r0;
+  if (n > j.split_rows) n = j.split_rows;
+  return (int)((n + 63) / 64);
+}
+
+template <class C>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                   const __grid_constant__ CUtensorMap tmY, const GemmJob job, float* __restrict__ partial,
+                   int* status) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  uint8_t* stg = smem;                      // kind 0: two 16 KB output staging chunks
+  uint8_t* ring = smem + C::STG_BYTES;
+  GemmBars* bars = (GemmBars*)(ring + C::NSTAGE * C::STAGE);
+  int* abort_flag = &bars->abort_flag;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int64_t nunits = job.units;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < C::NSTAGE; ++i) {
+      ptx::mbar_init(&bars->full[i], 1);
+      ptx::mbar_init(&bars->empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      ptx::mbar_init(&bars->acc_full[i], 1);
+      ptx::mbar_init(&bars->acc_empty[i], kGemmEpiWarps);
+    }
+    ptx::mbar_init(&bars->mma_done, 1);
+    bars->abort_flag = 0;
+    ptx::fence_mbar_init();
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc(&bars->tmem_base, C::TMEM_COLS);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+  // inputs may be written by the previous kernel of the stream
+  ptx::griddep_wait();
+  ptx::griddep_launch_dependents();
+
+  if (warp == 0) {
+    // ================================================================ TMA producer
+    if (lane == 0) {
+      ptx::tma_prefetch_desc(&tmA);
+      ptx::tma_prefetch_desc(&tmB);
+      if (C::KIND == 0) ptx::tma_prefetch_desc(&tmY);
+      const uint64_t pol = ptx::policy_evict_normal();
+      uint32_t it = 0;
+      bool ok = true;
+      for (int64_t u = blockIdx.x; u < nunits && ok; u += gridDim.x) {
+        const UnitCoord c = unit_coord(job, u);
+        const int nk = unit_kstages(job, c);
+        for (int kb = 0; kb < nk; ++kb, ++it) {
+          const int st = it % C::NSTAGE;
+          if (!wait_or_abort(&bars->empty[st], ((it / C::NSTAGE) & 1) ^ 1, abort_flag, status)) { ok = false; break; }
+          uint8_t* sa = ring + st * C::STAGE;
+          uint8_t* sb = sa + C::A_BYTES;
+          ptx::mbar_arrive_expect_tx(&bars->full[st], C::STAGE);
+          if (C::KIND == 0) {
+            const int ax = gcol(c.b, job.a_b, kb, job.a_grp, job.a_gs);
+            ptx::tma_load_2d(sa, &tmA, &bars->full[st], ax, c.mt * C::BM, pol);
+            ptx::tma_load_2d(sb, &tmB, &bars->full[st], kb * 64, c.b * job.b_b + c.nt * C::BN, pol);
+          } else {
+            const int row = (int)((int64_t)c.split * job.split_rows + (int64_t)kb * 64);
+            const int ax = c.b * job.a_b + c.mt * C::BM;
+            ptx::tma_load_2d(sa, &tmA, &bars->full[st], ax, row, pol);
+            ptx::tma_load_2d(sa + 8192, &tmA, &bars->full[st], ax + 64, row, pol);
+#pragma unroll
+            for (int h = 0; h < C::BN / 64; ++h)
+              ptx::tma_load_2d(sb + h * 8192, &tmB, &bars->full[st],
+                               gcol(c.b, job.b_b, c.nt * (C::BN / 64) + h, job.b_grp, job.b_gs), row, pol);
+          }
+        }
+      }
+      const uint32_t issued = it;
+      for (uint32_t k = (issued > (uint32_t)C::NSTAGE ? issued - C::NSTAGE : 0); k < issued; ++k)
+        ptx::mbar_wait_bounded(&bars->full[k % C::NSTAGE], (k / C::NSTAGE) & 1, kWaitLimitNs);
+    }
+  } else if (warp == 1) {
+    // ================================================================ MMA issuer
+    constexpr bool MN = C::KIND == 1;
+    constexpr uint32_t idesc = make_idesc(C::BM, C::BN) | (MN ? (1u << 15) | (1u << 16) : 0u);
+    // K-major: one 128-byte swizzled row per M/N index, a K step of 16 advances 32 bytes.
+    // MN-major: one 128-byte row per K index holding 64 M/N indices (LBO = 8 KB between
+    // the 64-wide M/N halves), a K step of 16 advances two 8-row groups (2 KB).
+    const uint64_t dA = MN ? make_sdesc_lbo(ptx::smem_u32(ring), 8192, 1024, 2) : make_sdesc(ptx::smem_u32(ring), 1024, 2);
+    const uint64_t dB = MN ? make_sdesc_lbo(ptx::smem_u32(ring + C::A_BYTES), 8192, 1024, 2)
+                           : make_sdesc(ptx::smem_u32(ring + C::A_BYTES), 1024, 2);
+    constexpr uint64_t kstep = MN ? (2048 >> 4) : (32 >> 4);
+    uint32_t it = 0, n = 0;
+    bool ok = true;
+    for (int64_t u = blockIdx.x; u < nunits && ok; u += gridDim.x, ++n) {
+      const UnitCoord c = unit_coord(job, u);
+      const int nk = unit_kstages(job, c);
+      const int slot = n & 1;
+      if (!warp_wait_or_abort(lane, &bars->acc_empty[slot], ((n >> 1) & 1) ^ 1, abort_flag, status)) { ok = false; break; }
+      ptx::tc_fence_after();
+      const uint32_t d = tmem + slot * C::BN;
+      for (int kb = 0; kb < nk; ++kb, ++it) {
+        const int st = it % C::NSTAGE;
+        if (!warp_wait_or_abort(lane, &bars->full[st], (it / C::NSTAGE) & 1, abort_flag, status)) { ok = false; break; }
+        ptx::tc_fence_after();
+        const uint64_t soff = (uint64_t)((st * C::STAGE) >> 4);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          ptx::mma_bf16_ss_elect(d, dA + soff + kk * kstep, dB + soff + kk * kstep, idesc,
+                                 (kb > 0 || kk > 0) ? 1u : 0u);
+        ptx::mma_commit_elect(&bars->empty[st]);
+      }
+      if (!ok) break;
+      ptx::mma_commit_elect(&bars->acc_full[slot]);
+    }
+    ptx::mma_commit_elect(&bars->mma_done);
+    if (lane == 0) wait_mma_done(&bars->mma_done, abort_flag, status);
+    __syncwarp();
+  } else {
+    // ================================================================ epilogue (4 warps)
+    const int quad = warp & 3;
+    const int r = quad * 32 + lane;  // D row of this thread
+    const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+    const bool leader = (warp == 2 && lane == 0);
+    const uint32_t stg_s = ptx::smem_u32(stg);
+    uint32_t n = 0, chunk_n = 0;
+    bool ok = true;
+    for (int64_t u = blockIdx.x; u < nunits && ok; u += gridDim.x, ++n) {
+      const UnitCoord c = unit_coord(job, u);
+      const int slot = n & 1;
+      if (!wait_or_abort(&bars->acc_full[slot], (n >> 1) & 1, abort_flag, status)) { ok = false; break; }
+      ptx::tc_fence_after();
+      const uint32_t tb = tmem + lane_off + slot * C::BN;
+      if (C::KIND == 0) {
+        for (int ch = 0; ch < C::BN / 64; ++ch, ++chunk_n) {
+          uint32_t v[64];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            uint32_t t16[16];
+            ptx::tmem_ld16(tb + ch * 64 + q * 16, t16);
+#pragma unroll
+            for (int e = 0; e < 16; ++e) v[q * 16 + e] = t16[e];
+          }
+          ptx::tmem_wait_ld();
+          const int sbuf = chunk_n & 1;
+          // the TMA store that last read this staging buffer must have finished reading it
+          if (leader) ptx::bulk_wait_read_allbut1();
+          ptx::named_bar_sync(1, kGemmEpiWarps * 32);
+          const uint32_t base = stg_s + sbuf * (C::BM * 128) + r * 128;
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            ptx::st_shared_v4(base + (((uint32_t)q ^ (uint32_t)(r & 7)) << 4),
+                              ptx::pack_bf16x2(__uint_as_float(v[8 * q + 0]), __uint_as_float(v[8 * q + 1])),
+                              ptx::pack_bf16x2(__uint_as_float(v[8 * q + 2]), __uint_as_float(v[8 * q + 3])),
+                              ptx::pack_bf16x2(__uint_as_float(v[8 * q + 4]), __uint_as_float(v[8 * q + 5])),
+                              ptx::pack_bf16x2(__uint_as_float(v[8 * q + 6]), __uint_as_float(v[8 * q + 7])));
+          ptx::fence_proxy_async_smem();
+          ptx::named_bar_sync(1, kGemmEpiWarps * 32);
+          if (leader) {
+            ptx::tma_store_2d(&tmY, stg + sbuf * (C::BM * 128),
+                              gcol(c.b, job.y_b, c.nt * (C::BN / 64) + ch, job.y_grp, job.y_gs), c.mt * C::BM);
+            ptx::bulk_commit_group();
+          }
+        }
+      } else {
+        // diagonal blocks of D as fp32 partials: row m belongs to block bm = ma / blk_a
+        const int64_t ma = (int64_t)c.b * job.a_b + (int64_t)c.mt * C::BM + r;
+        const int64_t nb0 = (int64_t)c.b * job.b_lb + (int64_t)c.nt * C::BN;
+        const bool row_ok = ma < job.a_cols;
+        const int64_t blk = ma / job.blk_a;
+        // columns of this warp's rows: [first row's block start, last row's block end)
+        const int64_t ma0 = (int64_t)c.b * job.a_b + (int64_t)c.mt * C::BM + quad * 32;
+        int64_t lo = (ma0 / job.blk_a) * job.blk_b - nb0;
+        int64_t hi = ((ma0 + 31) / job.blk_a + 1) * job.blk_b - nb0;
+        lo = lo < 0 ? 0 : (lo / 16) * 16;
+        hi = hi > C::BN ? C::BN : hi;
+        float* prow = partial + (int64_t)c.split * job.p_stride + job.p_off +
+                      blk * job.blk_a * job.blk_b + (ma % job.blk_a) * job.blk_b;
+        for (int c0 = (int)lo; c0 < (int)hi; c0 += 16) {
+          uint32_t t16[16];
+          ptx::tmem_ld16(tb + c0, t16);
+          ptx::tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const int64_t ng = nb0 + c0 + e;
+            if (row_ok && ng < job.b_cols && ng / job.blk_b == blk) {
+              const int64_t nl = ng % job.blk_b;
+              prow[(nl % job.pm_a) * job.pm_b + nl / job.pm_a] = __uint_as_float(t16[e]);
+            }
+          }
+        }
+      }
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(&bars->acc_empty[slot]);
+    }
+    if (C::KIND == 0 && leader) ptx::bulk_wait_all();
+  }
+
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  if (warp == 1) ptx::tmem_dealloc(tmem, C::TMEM_COLS);
+}
+
+template <int BN, int KIND>
+static cudaError_t launch_gemm_cfg(const CUtensorMap& mA, const CUtensorMap& mB, const CUtensorMap& mY,
+                                   const GemmJob& job, float* partial, int* status, cudaStream_t st,
+                                   bool pdl) {
+  using C = GemmCfg<BN, KIND>;
+  cudaError_t e = cudaFuncSetAttribute(tc_gemm_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       C::SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  int64_t grid = num_sms();
+  if (grid > job.units) grid = job.units;
+  return launch_kernel(tc_gemm_kernel<C>, dim3((unsigned)grid), dim3(kGemmThreads), C::SMEM_BYTES, st, pdl,
+                       mA, mB, mY, job, partial, status);
+}
+
+cudaError_t gemm_bd(const void* A, int64_t rows, int64_t a_cols, const void* W, int64_t w_rows, int K,
+                    void* Y, int64_t y_cols, int BN, GemmJob job, int* status, cudaStream_t st, bool pdl) {
+  if (rows == 0) return cudaSuccess;
+  CUtensorMap mA, mB, mY;
+  if (!make_map_2d(&mA, A, (uint64_t)a_cols, (uint64_t)rows, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map_2d(&mB, W, (uint64_t)K, (uint64_t)w_rows, 64, (uint32_t)BN, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map_2d(&mY, Y, (uint64_t)y_cols, (uint64_t)rows, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  job.kind = 0;
+  job.mtiles = (int)((rows + 127) / 128);
+  job.units = (int64_t)job.mtiles * job.nb * job.ntiles;
+  switch (BN) {
+    case 64: return launch_gemm_cfg<64, 0>(mA, mB, mY, job, nullptr, status, st, pdl);
+    case 128: return launch_gemm_cfg<128, 0>(mA, mB, mY, job, nullptr, status, st, pdl);
+    case 256: return launch_gemm_cfg<256, 0>(mA, mB, mY, job, nullptr, status, st, pdl);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+cudaError_t gemm_wgrad(const void* A1, int64_t a_cols, const void* A2, int64_t b_cols, int64_t rows, int BN,
+                       GemmJob job, float* partial, int* status, cudaStream_t st, bool pdl) {
+  CUtensorMap mA, mB;
+  if (!make_map_2d(&mA, A1, (uint64_t)a_cols, (uint64_t)rows, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map_2d(&mB, A2, (uint64_t)b_cols, (uint64_t)rows, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  job.kind = 1;
+  job.rows = rows;
+  job.a_cols = a_cols;
+  job.b_cols = b_cols;
+  job.units = (int64_t)job.mtiles * job.ntiles * job.nb * job.nsplit;
+  switch (BN) {
+    case 64: return launch_gemm_cfg<64, 1>(mA, mB, mA, job, partial, status, st, pdl);
+    case 128: return launch_gemm_cfg<128, 1>(mA, mB, mA, job, partial, status, st, pdl);
+    case 256: return launch_gemm_cfg<256, 1>(mA, mB, mA, job, partial, status, st, pdl);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace monarch

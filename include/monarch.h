@@ -182,9 +182,13 @@ MONARCH_API uint64_t monarch_kernel_launches(void);
  * rounds of 8 output columns (transposed outputs wider than the middle vector,
  * e.g. 768 -> 3072), 4 = for square 64 x 64 blocks with nb1 = nb2 (e.g. n = 4096):
  * two tcgen05 block-diagonal GEMM passes and two row-permutation passes over Y (Y
- * doubles as the middle vector's storage; no scratch).  For the backward: 0 = generic FMA kernels, 1 = tensor-core
- * backward (row-tile kernels for dX and the middle vector, warp-level MMA for the
- * weight gradients).  Host-only. */
+ * doubles as the middle vector's storage; no scratch).  For the backward: 0 = generic FMA
+ * kernels, 1 = tensor-core row-tile kernels (or block-GEMM passes for 64 x 64 blocks) for dX
+ * and the middle vector, 2 = tcgen05 GEMM passes for shapes whose permutation moves whole
+ * 64-column groups (e.g. nblocks = 4, 1024 -> 4096), 3 = packed block-diagonal tcgen05 GEMM
+ * passes (g small blocks as one zero-filled block-diagonal tile) with row-transpose passes for
+ * the permutations (e.g. 768 -> 3072); every tensor-core family computes the weight
+ * gradients as tcgen05 GEMMs over the rows.  Host-only. */
 MONARCH_API int monarch_fwd_path(const monarch_dims* d);
 MONARCH_API int monarch_bwd_path(const monarch_dims* d);
 

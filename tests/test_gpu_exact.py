@@ -31,7 +31,9 @@ CASES = [
     ("n1024_rows", synthetic.shape_of(W["n1024_bf16"]), "bf16", 300, 2, 1),
     ("r768x3072_wide", synthetic.shape_of(W["r768x3072_bf16"]), "bf16", 300, 3, None),
     ("n4096_split", synthetic.shape_of(W["n4096_bf16"]), "bf16", 300, 4, 1),
-    ("nblk4_group", synthetic.shape_of(W["nblk4_1024x4096_bf16"]), "bf16", 300, 1, None),
+    ("nblk4_group", synthetic.shape_of(W["nblk4_1024x4096_bf16"]), "bf16", 300, 1, 2),
+    # G = in2 / nb1 = 128: two 64-column groups per R block in the gathers
+    ("nblk2_gemm", dict(nb1=2, in1=128, out1=256, nb2=2, in2=256, out2=384, out_transpose=0), "bf16", 300, 0, 2),
     ("odd_generic_bf16", ODD, "bf16", 203, 0, 0),
 ]
 
