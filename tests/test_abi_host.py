@@ -97,7 +97,7 @@ def test_kernel_family_selection():
     assert bdl.bwd_path(synthetic.shape_of(W["n256_fp32"]), "bf16") == 1
     assert bdl.bwd_path(synthetic.shape_of(W["n256_fp32"]), "f32") == 0
     assert bdl.bwd_path(synthetic.shape_of(W["n4096_bf16"]), "bf16") == 1
-    assert bdl.bwd_path(synthetic.shape_of(W["r768x3072_bf16"]), "bf16") == 0
+    assert bdl.bwd_path(synthetic.shape_of(W["r768x3072_bf16"]), "bf16") == 3
     assert bdl.bwd_path(synthetic.shape_of(W["nblk4_1024x4096_bf16"]), "bf16") == 2
     assert bdl.bwd_path(synthetic.shape_of(W["nblk4_1024x4096_bf16"]), "f32") == 0
 

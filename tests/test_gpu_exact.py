@@ -29,7 +29,7 @@ CASES = [
     ("n256_fp32_generic", synthetic.shape_of(W["n256_fp32"]), "f32", 77, 0, 0),
     ("sq16_rows", SQ16, "bf16", 300, 2, 1),
     ("n1024_rows", synthetic.shape_of(W["n1024_bf16"]), "bf16", 300, 2, 1),
-    ("r768x3072_wide", synthetic.shape_of(W["r768x3072_bf16"]), "bf16", 300, 3, None),
+    ("r768x3072_wide", synthetic.shape_of(W["r768x3072_bf16"]), "bf16", 300, 3, 3),
     ("n4096_split", synthetic.shape_of(W["n4096_bf16"]), "bf16", 300, 4, 1),
     ("nblk4_group", synthetic.shape_of(W["nblk4_1024x4096_bf16"]), "bf16", 300, 1, 2),
     # G = in2 / nb1 = 128: two 64-column groups per R block in the gathers
@@ -84,8 +84,7 @@ def test_forward_exact(case):
 @pytest.mark.parametrize("case", CASES, ids=_ids)
 def test_backward_exact(case):
     _, shape, dtype, rows, _, bpath = case
-    if bpath is not None:
-        assert bdl.bwd_path(shape, dtype) == bpath
+    assert bdl.bwd_path(shape, dtype) == bpath
     inp = synthetic.make_sparse_sign_inputs(dict(shape, rows=rows), seed=22)
     _check_exact_range(inp)
     refs = oracle.backward(shape, inp["dY"], inp["X"], inp["R"], inp["L"])
