@@ -42,7 +42,8 @@ EXPORTED = (
     "monarch_validate", "monarch_fwd", "monarch_bwd", "monarch_bwd_workspace_bytes",
     "monarch_materialise", "monarch_status_string", "monarch_last_device_status",
     "monarch_debug_wait_timeout", "monarch_fwd_path", "monarch_bwd_path", "monarch_bwd_noalloc",
-    "monarch_kernel_launches",
+    "monarch_kernel_launches", "monarch_linear_shape", "monarch_linear_workspace_bytes",
+    "monarch_linear_fwd", "monarch_linear_bwd",
 )
 
 
@@ -57,6 +58,18 @@ class MonarchDims(ctypes.Structure):
         ("in2", ctypes.c_int32),
         ("out2", ctypes.c_int32),
         ("out_transpose", ctypes.c_int32),
+        ("dtype", ctypes.c_int32),
+    ]
+
+
+class MonarchLinearDims(ctypes.Structure):
+    """Mirror of ``monarch_linear_dims`` in include/monarch.h."""
+    _fields_ = [
+        ("rows", ctypes.c_int64),
+        ("in_features", ctypes.c_int32),
+        ("out_features", ctypes.c_int32),
+        ("nblocks", ctypes.c_int32),
+        ("has_bias", ctypes.c_int32),
         ("dtype", ctypes.c_int32),
     ]
 
@@ -94,6 +107,15 @@ def lib() -> ctypes.CDLL:
         L.monarch_bwd_path.argtypes = [dp]
         L.monarch_kernel_launches.argtypes = []
         L.monarch_kernel_launches.restype = ctypes.c_uint64
+        lp = ctypes.POINTER(MonarchLinearDims)
+        L.monarch_linear_shape.argtypes = [lp, dp]
+        L.monarch_linear_shape.restype = ctypes.c_int
+        L.monarch_linear_workspace_bytes.argtypes = [lp]
+        L.monarch_linear_workspace_bytes.restype = ctypes.c_size_t
+        L.monarch_linear_fwd.argtypes = [vp, vp, vp, vp, lp, vp, vp, ctypes.c_size_t, vp]
+        L.monarch_linear_fwd.restype = ctypes.c_int
+        L.monarch_linear_bwd.argtypes = [vp, vp, vp, vp, lp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp]
+        L.monarch_linear_bwd.restype = ctypes.c_int
         for name in ("monarch_validate", "monarch_fwd", "monarch_bwd", "monarch_materialise",
                      "monarch_last_device_status", "monarch_debug_wait_timeout",
                      "monarch_fwd_path", "monarch_bwd_path", "monarch_bwd_noalloc"):
@@ -271,6 +293,88 @@ def last_device_status(stream=None) -> int:
 
 def debug_wait_timeout(timeout_ns: int, stream=None) -> int:
     return lib().monarch_debug_wait_timeout(ctypes.c_uint64(int(timeout_ns)), _stream(stream))
+
+
+# ---------------------------------------------------------------- MonarchLinear front end
+def linear_dims(in_features: int, out_features: int, nblocks: int, rows: int, dtype="bf16",
+                bias: bool = False) -> MonarchLinearDims:
+    return MonarchLinearDims(int(rows), int(in_features), int(out_features), int(nblocks), int(bool(bias)),
+                             dtype_code(dtype))
+
+
+def linear_shape(in_features: int, out_features: int, nblocks: int, dtype="bf16") -> dict:
+    """Monarch shape (nb1, in1, out1, nb2, in2, out2, out_transpose) of
+    MonarchLinear(in_features, out_features, nblocks), computed by the library."""
+    d = MonarchDims()
+    ld = linear_dims(in_features, out_features, nblocks, 0, dtype)
+    _check("monarch_linear_shape", lib().monarch_linear_shape(ctypes.byref(ld), ctypes.byref(d)))
+    return dict(nb1=d.nb1, in1=d.in1, out1=d.out1, nb2=d.nb2, in2=d.in2, out2=d.out2,
+                out_transpose=d.out_transpose)
+
+
+def linear_workspace_bytes(in_features: int, out_features: int, nblocks: int, rows: int, dtype="bf16",
+                           bias: bool = False) -> int:
+    ld = linear_dims(in_features, out_features, nblocks, rows, dtype, bias)
+    return int(lib().monarch_linear_workspace_bytes(ctypes.byref(ld)))
+
+
+def _linear_check(X, R, L, shape, in_features, out_features, **ts):
+    rows = X.shape[0] if X is not None else ts["dY"].shape[0]
+    want = {"X": (rows, in_features), "dX": (rows, in_features), "Y": (rows, out_features),
+            "dY": (rows, out_features), "bias": (out_features,), "dbias": (out_features,),
+            "R": (shape["nb1"], shape["out1"], shape["in1"]), "dR": (shape["nb1"], shape["out1"], shape["in1"]),
+            "L": (shape["nb2"], shape["out2"], shape["in2"]), "dL": (shape["nb2"], shape["out2"], shape["in2"])}
+    for name, t in dict(ts, X=X, R=R, L=L).items():
+        if t is None:
+            continue
+        if tuple(t.shape) != want[name]:
+            raise ValueError("%s has shape %s, MonarchLinear needs %s" % (name, tuple(t.shape), want[name]))
+        if t.dtype != X.dtype:
+            raise ValueError("%s is %s, X is %s: every tensor must have one dtype" % (name, t.dtype, X.dtype))
+
+
+def linear_fwd(X, R, L, in_features: int, out_features: int, nblocks: int, bias=None, Y=None, workspace=None,
+               stream=None):
+    """MonarchLinear forward on the GPU: Y = crop(Monarch(pad(X))) + bias."""
+    import torch
+    rows = X.shape[0]
+    shape = linear_shape(in_features, out_features, nblocks, X.dtype)
+    _linear_check(X, R, L, shape, in_features, out_features, bias=bias, Y=Y)
+    if Y is None:
+        Y = torch.empty((rows, out_features), dtype=X.dtype, device=X.device)
+    ld = linear_dims(in_features, out_features, nblocks, rows, X.dtype, bias is not None)
+    need = int(lib().monarch_linear_workspace_bytes(ctypes.byref(ld)))
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=X.device)
+    _require_cuda(X, R, L, bias, Y, workspace)
+    _check("monarch_linear_fwd", lib().monarch_linear_fwd(
+        _ptr(X), _ptr(R), _ptr(L), _ptr(bias), ctypes.byref(ld), _ptr(Y), _ptr(workspace),
+        ctypes.c_size_t(workspace.numel() * workspace.element_size()), _stream(stream)))
+    return Y
+
+
+def linear_bwd(dY, X, R, L, in_features: int, out_features: int, nblocks: int, bias: bool = False, dX=None,
+               dR=None, dL=None, dbias=None, workspace=None, stream=None):
+    """MonarchLinear backward on the GPU: (dX, dR, dL, dbias); dbias is None without a bias."""
+    import torch
+    rows = X.shape[0]
+    shape = linear_shape(in_features, out_features, nblocks, X.dtype)
+    _linear_check(X, R, L, shape, in_features, out_features, dY=dY, dX=dX, dR=dR, dL=dL, dbias=dbias)
+    dX = torch.empty_like(X) if dX is None else dX
+    dR = torch.empty_like(R) if dR is None else dR
+    dL = torch.empty_like(L) if dL is None else dL
+    if bias and dbias is None:
+        dbias = torch.empty((out_features,), dtype=X.dtype, device=X.device)
+    ld = linear_dims(in_features, out_features, nblocks, rows, X.dtype, bias)
+    need = int(lib().monarch_linear_workspace_bytes(ctypes.byref(ld)))
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=X.device)
+    _require_cuda(dY, X, R, L, dX, dR, dL, dbias, workspace)
+    _check("monarch_linear_bwd", lib().monarch_linear_bwd(
+        _ptr(dY), _ptr(X), _ptr(R), _ptr(L), ctypes.byref(ld), _ptr(dX), _ptr(dR), _ptr(dL),
+        _ptr(dbias if bias else None), _ptr(workspace),
+        ctypes.c_size_t(workspace.numel() * workspace.element_size()), _stream(stream)))
+    return dX, dR, dL, (dbias if bias else None)
 
 
 def kernel_launches() -> int:

@@ -13,13 +13,13 @@ namespace monarch {
 // Device status word: kernels that give up a bounded wait store kStatusTimeout.
 __device__ int g_status;
 
-static int* status_ptr() {
+int* status_ptr() {
   int* p = nullptr;
   if (cudaGetSymbolAddress((void**)&p, g_status) != cudaSuccess) return nullptr;
   return p;
 }
 
-static bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
 
 static int check_dims(const monarch_dims* d) {
   if (d == nullptr) return MONARCH_ERR_NULL;
@@ -88,13 +88,69 @@ cudaError_t debug_wait_timeout(uint64_t timeout_ns, int* status, cudaStream_t st
 // 0 = generic FMA kernels, 1 = tcgen05 group kernel, 2 = tcgen05 row-tile kernel,
 // 3 = tcgen05 row-tile kernel with the L stage in rounds of output columns,
 // 4 = tcgen05 block-diagonal GEMMs and row permutations as separate passes over Y.
-static int fwd_path(const Shape& s, int dtype) {
+int fwd_path(const Shape& s, int dtype) {
   if (dtype != MONARCH_BF16) return 0;
   if (tc_rows_supported(s)) return 2;
   if (tc_wide_supported(s)) return 3;
   if (tc_split_supported(s)) return 4;
   if (tc_fwd_supported(s)) return 1;
   return 0;
+}
+
+// 0 = generic FMA kernels, 1 = row-tile / block-GEMM passes with tcgen05 weight gradients,
+// 2 = tcgen05 GEMM passes (permutation folded into 64-column gathers), 3 = packed
+// block-diagonal tcgen05 GEMM passes with row-transpose passes for the permutations.
+int bwd_path(const Shape& s, int dtype) {
+  if (dtype != MONARCH_BF16) return 0;
+  if (fast_bwd_supported(s)) return 1;
+  if (gemm_bwd_supported(s)) return 2;
+  if (packed_bwd_supported(s)) return 3;
+  return 0;
+}
+
+size_t bwd_workspace(const Shape& s, int dtype) {
+  switch (bwd_path(s, dtype)) {
+    case 1: return fast_bwd_workspace(s);
+    case 2: return gemm_bwd_workspace(s);
+    case 3: return packed_bwd_workspace(s);
+    default: return generic_bwd_workspace(s);
+  }
+}
+
+// Forward on already-checked arguments (rows > 0).
+int fwd_dispatch(const void* X, const void* R, const void* L, void* Y, const Shape& s, int dtype, cudaStream_t st) {
+  cudaError_t e;
+  const int path = fwd_path(s, dtype);
+  if (path != 0) {
+    int* status = status_ptr();
+    if (status == nullptr) return MONARCH_ERR_CUDA;
+    e = path == 2   ? tc_rows_fwd(X, R, L, Y, s, status, st)
+        : path == 3 ? tc_wide_fwd(X, R, L, Y, s, status, st)
+        : path == 4 ? tc_split_fwd(X, R, L, Y, s, status, st)
+                    : tc_fwd(X, R, L, Y, s, status, st);
+  } else {
+    if (!generic_fwd_supported(s)) return MONARCH_ERR_UNSUPPORTED;
+    e = generic_fwd(X, R, L, Y, s, dtype, st);
+  }
+  return e == cudaSuccess ? MONARCH_OK : MONARCH_ERR_CUDA;
+}
+
+// Backward on already-checked arguments (workspace of bwd_workspace(s, dtype) bytes).
+int bwd_dispatch(const void* dY, const void* X, const void* R, const void* L, void* dX, void* dR, void* dL,
+                 void* ws, const Shape& s, int dtype, cudaStream_t st) {
+  cudaError_t e;
+  const int path = bwd_path(s, dtype);
+  if (path != 0) {
+    int* status = status_ptr();
+    if (status == nullptr) return MONARCH_ERR_CUDA;
+    e = path == 1   ? fast_bwd(dY, X, R, L, dX, dR, dL, ws, s, status, st)
+        : path == 2 ? gemm_bwd(dY, X, R, L, dX, dR, dL, ws, s, status, st)
+                    : packed_bwd(dY, X, R, L, dX, dR, dL, ws, s, status, st);
+  } else {
+    if (!generic_bwd_supported(s)) return MONARCH_ERR_UNSUPPORTED;
+    e = generic_bwd(dY, X, R, L, dX, dR, dL, ws, s, dtype, st);
+  }
+  return e == cudaSuccess ? MONARCH_OK : MONARCH_ERR_CUDA;
 }
 
 }  // namespace monarch
@@ -108,26 +164,6 @@ int monarch_validate(const monarch_dims* d) { return check_dims(d); }
 int monarch_fwd_path(const monarch_dims* d) {
   if (check_dims(d) != MONARCH_OK) return -1;
   return fwd_path(to_shape(*d), d->dtype);
-}
-
-// 0 = generic FMA kernels, 1 = row-tile / block-GEMM passes with tcgen05 weight gradients,
-// 2 = tcgen05 GEMM passes (permutation folded into 64-column gathers), 3 = packed
-// block-diagonal tcgen05 GEMM passes with row-transpose passes for the permutations.
-static int bwd_path(const Shape& s, int dtype) {
-  if (dtype != MONARCH_BF16) return 0;
-  if (fast_bwd_supported(s)) return 1;
-  if (gemm_bwd_supported(s)) return 2;
-  if (packed_bwd_supported(s)) return 3;
-  return 0;
-}
-
-static size_t bwd_workspace(const Shape& s, int dtype) {
-  switch (bwd_path(s, dtype)) {
-    case 1: return fast_bwd_workspace(s);
-    case 2: return gemm_bwd_workspace(s);
-    case 3: return packed_bwd_workspace(s);
-    default: return generic_bwd_workspace(s);
-  }
 }
 
 int monarch_bwd_path(const monarch_dims* d) {
@@ -147,21 +183,7 @@ int monarch_fwd(const void* X, const void* R, const void* L, const monarch_dims*
                         {span(X, s.rows * s.n_in(), es), span(R, s.n_R(), es), span(L, s.n_L(), es)})) !=
       MONARCH_OK)
     return rc;
-  cudaStream_t st = (cudaStream_t)stream;
-  cudaError_t e;
-  const int path = fwd_path(s, d->dtype);
-  if (path != 0) {
-    int* status = status_ptr();
-    if (status == nullptr) return MONARCH_ERR_CUDA;
-    e = path == 2   ? tc_rows_fwd(X, R, L, Y, s, status, st)
-        : path == 3 ? tc_wide_fwd(X, R, L, Y, s, status, st)
-        : path == 4 ? tc_split_fwd(X, R, L, Y, s, status, st)
-                    : tc_fwd(X, R, L, Y, s, status, st);
-  } else {
-    if (!generic_fwd_supported(s)) return MONARCH_ERR_UNSUPPORTED;
-    e = generic_fwd(X, R, L, Y, s, d->dtype, st);
-  }
-  return e == cudaSuccess ? MONARCH_OK : MONARCH_ERR_CUDA;
+  return fwd_dispatch(X, R, L, Y, s, d->dtype, (cudaStream_t)stream);
 }
 
 size_t monarch_bwd_workspace_bytes(const monarch_dims* d) {
@@ -186,19 +208,7 @@ int monarch_bwd(const void* dY, const void* X, const void* R, const void* L, con
                         {span(dY, s.rows * s.n_out(), es), span(X, s.rows * s.n_in(), es),
                          span(R, s.n_R(), es), span(L, s.n_L(), es)})) != MONARCH_OK)
     return rc;
-  cudaError_t e;
-  const int path = bwd_path(s, d->dtype);
-  if (path != 0) {
-    int* status = status_ptr();
-    if (status == nullptr) return MONARCH_ERR_CUDA;
-    e = path == 1   ? fast_bwd(dY, X, R, L, dX, dR, dL, workspace, s, status, (cudaStream_t)stream)
-        : path == 2 ? gemm_bwd(dY, X, R, L, dX, dR, dL, workspace, s, status, (cudaStream_t)stream)
-                    : packed_bwd(dY, X, R, L, dX, dR, dL, workspace, s, status, (cudaStream_t)stream);
-  } else {
-    if (!generic_bwd_supported(s)) return MONARCH_ERR_UNSUPPORTED;
-    e = generic_bwd(dY, X, R, L, dX, dR, dL, workspace, s, d->dtype, (cudaStream_t)stream);
-  }
-  return e == cudaSuccess ? MONARCH_OK : MONARCH_ERR_CUDA;
+  return bwd_dispatch(dY, X, R, L, dX, dR, dL, workspace, s, d->dtype, (cudaStream_t)stream);
 }
 
 int monarch_materialise(const void* R, const void* L, const monarch_dims* d, void* M,

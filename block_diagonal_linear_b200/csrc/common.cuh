@@ -6,6 +6,7 @@
 #include <stdint.h>
 
 #include <atomic>
+#include <initializer_list>
 
 #include "../../include/monarch.h"
 
@@ -121,5 +122,15 @@ cudaError_t fast_bwd(const void* dY, const void* X, const void* R, const void* L
                      void* dL, void* ws, const Shape& s, int* status, cudaStream_t st);
 
 cudaError_t debug_wait_timeout(uint64_t timeout_ns, int* status, cudaStream_t st);
+
+// Kernel-family selection and dispatch on already-checked arguments (api.cu).
+int fwd_path(const Shape& s, int dtype);
+int bwd_path(const Shape& s, int dtype);
+size_t bwd_workspace(const Shape& s, int dtype);
+int fwd_dispatch(const void* X, const void* R, const void* L, void* Y, const Shape& s, int dtype, cudaStream_t st);
+int bwd_dispatch(const void* dY, const void* X, const void* R, const void* L, void* dX, void* dR, void* dL,
+                 void* ws, const Shape& s, int dtype, cudaStream_t st);
+int* status_ptr();
+bool aligned16(const void* p);
 
 }  // namespace monarch

@@ -170,6 +170,46 @@ MONARCH_API int monarch_last_device_status(void* stream);
  * monarch_last_device_status(). */
 MONARCH_API int monarch_debug_wait_timeout(uint64_t timeout_ns, void* stream);
 
+/* ---------------------------------------------------------------- MonarchLinear front end
+ * Scatterbrain issue thread, the MonarchLinear __init__ listing: for MonarchLinear(
+ * in_features, out_features, nblocks) the block sizes are in_blksz = ceil(in / nblocks) and
+ * out_blksz = ceil(out / nblocks), the features are extended to in_blksz * nblocks and
+ * out_blksz * nblocks, and the factors are R = blkdiag1 (nblocks, mid, in_blksz) and
+ * L = blkdiag2 (nblocks, out_blksz, mid) with mid = in_blksz when the extended input is
+ * narrower than the extended output and mid = out_blksz otherwise.  The listing shows no
+ * forward; this library reads it as: x zero-padded to the extended width, the Monarch map
+ * of that shape with no output transpose (R on contiguous slices, the transpose, L, flatten),
+ * the result cut to out_features, plus an optional bias (out_features entries). */
+typedef struct {
+  int64_t rows;           /* rows of X                                           */
+  int32_t in_features, out_features, nblocks;
+  int32_t has_bias;       /* 1: bias / dbias arguments are used                  */
+  int32_t dtype;          /* monarch_dtype of every tensor argument              */
+} monarch_linear_dims;
+
+/* The equivalent monarch_dims of a MonarchLinear (host-only; MONARCH_ERR_DIMS / _DTYPE on a
+ * bad size or dtype). */
+MONARCH_API int monarch_linear_shape(const monarch_linear_dims* ld, monarch_dims* d);
+
+/* Device workspace bytes monarch_linear_fwd and monarch_linear_bwd need (0 if ld is bad). */
+MONARCH_API size_t monarch_linear_workspace_bytes(const monarch_linear_dims* ld);
+
+/* Y (rows, out_features) = crop(Monarch(pad(X))) + bias, X (rows, in_features).  R, L have the
+ * shapes monarch_linear_shape gives; bias may be NULL when has_bias is 0.  workspace: device
+ * memory of >= monarch_linear_workspace_bytes(ld) bytes, 256-byte aligned, owned by the
+ * caller.  Y and the workspace must not overlap the inputs or each other (MONARCH_ERR_ALIAS).
+ * Other conventions as monarch_fwd. */
+MONARCH_API int monarch_linear_fwd(const void* X, const void* R, const void* L, const void* bias,
+                                   const monarch_linear_dims* ld, void* Y, void* workspace,
+                                   size_t workspace_bytes, void* stream);
+
+/* Backward of monarch_linear_fwd for the upstream gradient dY (rows, out_features): dX (rows,
+ * in_features), dR, dL (factor shapes), dbias (out_features, the column sums of dY; only when
+ * has_bias), all overwritten.  Same workspace and overlap rules as monarch_linear_fwd. */
+MONARCH_API int monarch_linear_bwd(const void* dY, const void* X, const void* R, const void* L,
+                                   const monarch_linear_dims* ld, void* dX, void* dR, void* dL,
+                                   void* dbias, void* workspace, size_t workspace_bytes, void* stream);
+
 /* Number of kernels this library has launched in this process (every device and
  * stream), counted on the host at each successful launch.  Host-only; a caller
  * reads it before and after a region to count that region's launches. */

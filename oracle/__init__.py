@@ -154,3 +154,52 @@ def normwise_rel_err(got, ref) -> float:
     if den == 0.0:
         return 0.0 if num == 0.0 else float("inf")
     return num / den
+
+
+# ---------------------------------------------------------------- MonarchLinear front end
+# Scatterbrain issue thread, the MonarchLinear __init__ listing: block sizes are the ceilings
+# in_blksz = ceil(in / nblocks) and out_blksz = ceil(out / nblocks); the features are extended
+# to in_blksz * nblocks and out_blksz * nblocks; when the extended input is narrower than the
+# extended output, blkdiag1 is (nblocks, in_blksz, in_blksz) and blkdiag2 (nblocks, out_blksz,
+# in_blksz), otherwise blkdiag1 is (nblocks, out_blksz, in_blksz) and blkdiag2 (nblocks,
+# out_blksz, out_blksz).  The listing shows no forward; the reading taken here: x is
+# zero-padded to the extended width, multiplied as in the nblocks workload (blkdiag1 on
+# contiguous slices, transpose, blkdiag2, flatten), the result is cut to out_features, and an
+# optional bias is added.
+
+def linear_shape(in_features: int, out_features: int, nblocks: int) -> dict:
+    """Monarch shape of MonarchLinear(in_features, out_features, nblocks)."""
+    in_blk = -(-in_features // nblocks)
+    out_blk = -(-out_features // nblocks)
+    mid = in_blk if in_blk * nblocks < out_blk * nblocks else out_blk
+    return dict(nb1=nblocks, in1=in_blk, out1=mid, nb2=nblocks, in2=mid, out2=out_blk, out_transpose=0)
+
+
+def linear_forward(in_features: int, out_features: int, nblocks: int, X, R, L, bias=None,
+                   nthreads: int | None = None) -> np.ndarray:
+    """y = (M x_padded)[:out_features] + bias for every row x, in fp64."""
+    d = linear_shape(in_features, out_features, nblocks)
+    X = _f64(X).reshape(-1, in_features)
+    n_in, _, _ = sizes(d)
+    Xp = np.zeros((X.shape[0], n_in))
+    Xp[:, :in_features] = X
+    Y = forward(d, Xp, R, L, nthreads)[:, :out_features]
+    if bias is not None:
+        Y = Y + _f64(bias)[None, :]
+    return np.ascontiguousarray(Y)
+
+
+def linear_backward(in_features: int, out_features: int, nblocks: int, dY, X, R, L,
+                    nthreads: int | None = None):
+    """(dX, dR, dL, dbias) of linear_forward: the padded output columns get no gradient, the
+    padded input columns' gradient is dropped, dbias sums dY over the rows."""
+    d = linear_shape(in_features, out_features, nblocks)
+    X = _f64(X).reshape(-1, in_features)
+    dY = _f64(dY).reshape(-1, out_features)
+    n_in, _, n_out = sizes(d)
+    Xp = np.zeros((X.shape[0], n_in))
+    Xp[:, :in_features] = X
+    dYp = np.zeros((dY.shape[0], n_out))
+    dYp[:, :out_features] = dY
+    dXp, dR, dL = backward(d, dYp, Xp, R, L, nthreads)
+    return np.ascontiguousarray(dXp[:, :in_features]), dR, dL, dY.sum(axis=0)
