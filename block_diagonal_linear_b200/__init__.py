@@ -43,7 +43,7 @@ EXPORTED = (
     "monarch_materialise", "monarch_status_string", "monarch_last_device_status",
     "monarch_debug_wait_timeout", "monarch_fwd_path", "monarch_bwd_path", "monarch_bwd_noalloc",
     "monarch_kernel_launches", "monarch_linear_shape", "monarch_linear_workspace_bytes",
-    "monarch_linear_fwd", "monarch_linear_bwd",
+    "monarch_linear_fwd", "monarch_linear_bwd", "monarch_project",
 )
 
 
@@ -116,6 +116,8 @@ def lib() -> ctypes.CDLL:
         L.monarch_linear_fwd.restype = ctypes.c_int
         L.monarch_linear_bwd.argtypes = [vp, vp, vp, vp, lp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp]
         L.monarch_linear_bwd.restype = ctypes.c_int
+        L.monarch_project.argtypes = [vp, dp, vp, vp, vp]
+        L.monarch_project.restype = ctypes.c_int
         for name in ("monarch_validate", "monarch_fwd", "monarch_bwd", "monarch_materialise",
                      "monarch_last_device_status", "monarch_debug_wait_timeout",
                      "monarch_fwd_path", "monarch_bwd_path", "monarch_bwd_noalloc"):
@@ -284,6 +286,27 @@ def materialise(R, L, shape: dict, M=None, stream=None):
     _check("monarch_materialise", lib().monarch_materialise(_ptr(R), _ptr(L), ctypes.byref(d),
                                                             _ptr(M), _stream(stream)))
     return M
+
+
+def project(M, shape: dict, dtype="f32", R=None, L=None, stream=None):
+    """(R, L) of the Monarch matrix nearest to the dense float32 M (n_out, n_in), on the GPU."""
+    import torch
+    code = dtype_code(dtype)
+    n_in = shape["nb1"] * shape["in1"]
+    n_out = shape["nb2"] * shape["out2"]
+    if tuple(M.shape) != (n_out, n_in) or M.dtype != torch.float32:
+        raise ValueError("M must be float32 of shape %s" % ((n_out, n_in),))
+    dt = _torch_dtype(code)
+    if R is None:
+        R = torch.empty((shape["nb1"], shape["out1"], shape["in1"]), dtype=dt, device=M.device)
+    if L is None:
+        L = torch.empty((shape["nb2"], shape["out2"], shape["in2"]), dtype=dt, device=M.device)
+    _check_tensors(shape, 0, dt, R=R, L=L)
+    _require_cuda(M, R, L)
+    d = make_dims(shape, 0, code)
+    _check("monarch_project", lib().monarch_project(_ptr(M), ctypes.byref(d), _ptr(R), _ptr(L),
+                                                    _stream(stream)))
+    return R, L
 
 
 def last_device_status(stream=None) -> int:

@@ -170,6 +170,21 @@ MONARCH_API int monarch_last_device_status(void* stream);
  * monarch_last_device_status(). */
 MONARCH_API int monarch_debug_wait_timeout(uint64_t timeout_ns, void* stream);
 
+/* Dense -> Monarch projection (Monarch abstract: projecting onto the Monarch set "has an
+ * analytical optimal solution"; scatterbrain projection question: the dense matrix sliced
+ * with rearrange(M, '(p k) (r s) -> k r p s')).  For the lattice shapes (in2 == nb1,
+ * nb2 == out1, out_transpose = 1) every (j, k) slice A_jk[o][i] = M[o*nb2 + j][k*in1 + i] of
+ * a Monarch matrix is the rank-1 matrix L[j][:, k] R[k][j][:]^T, and the Frobenius-nearest
+ * Monarch matrix takes the best rank-1 approximation s u v^T of every slice:
+ * L[j][o][k] = sqrt(s) u[o], R[k][j][i] = sqrt(s) v[i], with the entry of v largest in
+ * magnitude made positive.
+ * In:  M (n_out, n_in) FLOAT32 row-major (the layout monarch_materialise writes).
+ * Out: R, L in d->dtype, overwritten.  fp32 power iteration per slice on the GPU (results
+ * agree with an SVD to fp32 accuracy when the slice's two leading singular values are well
+ * separated).  MONARCH_ERR_UNSUPPORTED for other shapes or slices wider than 1024 columns.
+ * d->rows is ignored. */
+MONARCH_API int monarch_project(const void* M, const monarch_dims* d, void* R, void* L, void* stream);
+
 /* ---------------------------------------------------------------- MonarchLinear front end
  * Scatterbrain issue thread, the MonarchLinear __init__ listing: for MonarchLinear(
  * in_features, out_features, nblocks) the block sizes are in_blksz = ceil(in / nblocks) and

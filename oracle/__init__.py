@@ -203,3 +203,40 @@ def linear_backward(in_features: int, out_features: int, nblocks: int, dY, X, R,
     dYp[:, :out_features] = dY
     dXp, dR, dL = backward(d, dYp, Xp, R, L, nthreads)
     return np.ascontiguousarray(dXp[:, :in_features]), dR, dL, dY.sum(axis=0)
+
+
+# ---------------------------------------------------------------- dense -> Monarch projection
+# Monarch abstract: projecting a dense matrix onto the Monarch set "has an analytical optimal
+# solution"; the scatterbrain projection question slices the dense matrix with
+# rearrange(M, '(p k) (r s) -> k r p s').  For the lattice shapes (in2 == nb1, nb2 == out1,
+# output transpose) every entry of M is one product, M[o*nb2 + j][k*in1 + i] = L[j][o][k] *
+# R[k][j][i], so the (j, k) slice A_jk[o][i] = M[o*nb2 + j][k*in1 + i] is the rank-1 matrix
+# L[j][:, k] R[k][j][:]^T and the slices cover M without overlap.  The Frobenius-nearest
+# Monarch matrix is therefore the best rank-1 approximation of every slice (Eckart-Young):
+# A_jk ~ s u v^T, L[j][:, k] = sqrt(s) u, R[k][j][:] = sqrt(s) v.  Sign convention (the
+# factors are unique up to a common sign flip): the entry of v largest in magnitude (first
+# one on ties) is made positive.
+
+def projection_supported(d: dict) -> bool:
+    return d["in2"] == d["nb1"] and d["nb2"] == d["out1"] and int(d.get("out_transpose", 1)) == 1
+
+
+def project(d: dict, M) -> tuple[np.ndarray, np.ndarray]:
+    """(R, L) of the Monarch matrix nearest to the dense M (n_out x n_in) in Frobenius norm."""
+    if not projection_supported(d):
+        raise ValueError("projection needs a lattice shape (in2 == nb1, nb2 == out1, out_transpose)")
+    M = _f64(M)
+    nb1, in1, nb2, out2 = d["nb1"], d["in1"], d["nb2"], d["out2"]
+    R = np.zeros((nb1, d["out1"], in1))
+    L = np.zeros((nb2, out2, d["in2"]))
+    for j in range(nb2):
+        for k in range(nb1):
+            A = M[j::nb2, k * in1:(k + 1) * in1]          # rows o*nb2 + j, columns k*in1 + i
+            U, S, Vt = np.linalg.svd(A, full_matrices=False)
+            u, s, v = U[:, 0], S[0], Vt[0]
+            t = int(np.argmax(np.abs(v)))
+            if v[t] < 0:
+                u, v = -u, -v
+            L[j, :, k] = np.sqrt(s) * u
+            R[k, j, :] = np.sqrt(s) * v
+    return R, L
