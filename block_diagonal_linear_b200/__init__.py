@@ -43,7 +43,8 @@ EXPORTED = (
     "monarch_materialise", "monarch_status_string", "monarch_last_device_status",
     "monarch_debug_wait_timeout", "monarch_fwd_path", "monarch_bwd_path", "monarch_bwd_noalloc",
     "monarch_kernel_launches", "monarch_linear_shape", "monarch_linear_workspace_bytes",
-    "monarch_linear_fwd", "monarch_linear_bwd", "monarch_project",
+    "monarch_linear_fwd", "monarch_linear_bwd", "monarch_project", "monarch_dyad_workspace_bytes",
+    "monarch_dyad_path", "monarch_dyad_fwd", "monarch_dyad_bwd",
 )
 
 
@@ -70,6 +71,17 @@ class MonarchLinearDims(ctypes.Structure):
         ("out_features", ctypes.c_int32),
         ("nblocks", ctypes.c_int32),
         ("has_bias", ctypes.c_int32),
+        ("dtype", ctypes.c_int32),
+    ]
+
+
+class MonarchDyadDims(ctypes.Structure):
+    """Mirror of ``monarch_dyad_dims`` in include/monarch.h."""
+    _fields_ = [
+        ("rows", ctypes.c_int64),
+        ("nblocks", ctypes.c_int32),
+        ("in_blk", ctypes.c_int32),
+        ("out_blk", ctypes.c_int32),
         ("dtype", ctypes.c_int32),
     ]
 
@@ -118,6 +130,15 @@ def lib() -> ctypes.CDLL:
         L.monarch_linear_bwd.restype = ctypes.c_int
         L.monarch_project.argtypes = [vp, dp, vp, vp, vp]
         L.monarch_project.restype = ctypes.c_int
+        yp = ctypes.POINTER(MonarchDyadDims)
+        L.monarch_dyad_workspace_bytes.argtypes = [yp]
+        L.monarch_dyad_workspace_bytes.restype = ctypes.c_size_t
+        L.monarch_dyad_path.argtypes = [yp]
+        L.monarch_dyad_path.restype = ctypes.c_int
+        L.monarch_dyad_fwd.argtypes = [vp, vp, vp, yp, vp, vp, ctypes.c_size_t, vp]
+        L.monarch_dyad_fwd.restype = ctypes.c_int
+        L.monarch_dyad_bwd.argtypes = [vp, vp, vp, vp, yp, vp, vp, vp, vp, ctypes.c_size_t, vp]
+        L.monarch_dyad_bwd.restype = ctypes.c_int
         for name in ("monarch_validate", "monarch_fwd", "monarch_bwd", "monarch_materialise",
                      "monarch_last_device_status", "monarch_debug_wait_timeout",
                      "monarch_fwd_path", "monarch_bwd_path", "monarch_bwd_noalloc"):
@@ -398,6 +419,68 @@ def linear_bwd(dY, X, R, L, in_features: int, out_features: int, nblocks: int, b
         _ptr(dbias if bias else None), _ptr(workspace),
         ctypes.c_size_t(workspace.numel() * workspace.element_size()), _stream(stream)))
     return dX, dR, dL, (dbias if bias else None)
+
+
+# ---------------------------------------------------------------- DYAD
+def dyad_dims(nblocks: int, in_blk: int, out_blk: int, rows: int, dtype="bf16") -> MonarchDyadDims:
+    return MonarchDyadDims(int(rows), int(nblocks), int(in_blk), int(out_blk), dtype_code(dtype))
+
+
+def dyad_path(nblocks: int, in_blk: int, out_blk: int, dtype="bf16") -> int:
+    """1 = tcgen05 path, 0 = generic FMA kernels (host-only query)."""
+    return lib().monarch_dyad_path(ctypes.byref(dyad_dims(nblocks, in_blk, out_blk, 1, dtype)))
+
+
+def _dyad_check(W1, W2, rows, **ts):
+    nb, ob, ib = W1.shape
+    want = {"X": (rows, nb * ib), "dX": (rows, nb * ib), "Y": (rows, nb * ob), "dY": (rows, nb * ob),
+            "W1": (nb, ob, ib), "W2": (nb, ob, ib), "dW1": (nb, ob, ib), "dW2": (nb, ob, ib)}
+    for name, t in dict(ts, W1=W1, W2=W2).items():
+        if t is None:
+            continue
+        if tuple(t.shape) != want[name]:
+            raise ValueError("%s has shape %s, DYAD needs %s" % (name, tuple(t.shape), want[name]))
+        if t.dtype != W1.dtype:
+            raise ValueError("%s is %s, W1 is %s: every tensor must have one dtype" % (name, t.dtype, W1.dtype))
+
+
+def dyad_fwd(X, W1, W2, Y=None, workspace=None, stream=None):
+    """DYAD forward on the GPU: Y = BD(W1) x + P_out^T BD(W2) P_in x for every row x."""
+    import torch
+    nb, ob, ib = W1.shape
+    rows = X.shape[0]
+    _dyad_check(W1, W2, rows, X=X, Y=Y)
+    if Y is None:
+        Y = torch.empty((rows, nb * ob), dtype=X.dtype, device=X.device)
+    dd = dyad_dims(nb, ib, ob, rows, X.dtype)
+    need = int(lib().monarch_dyad_workspace_bytes(ctypes.byref(dd)))
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=X.device)
+    _require_cuda(X, W1, W2, Y, workspace)
+    _check("monarch_dyad_fwd", lib().monarch_dyad_fwd(
+        _ptr(X), _ptr(W1), _ptr(W2), ctypes.byref(dd), _ptr(Y), _ptr(workspace),
+        ctypes.c_size_t(workspace.numel() * workspace.element_size()), _stream(stream)))
+    return Y
+
+
+def dyad_bwd(dY, X, W1, W2, dX=None, dW1=None, dW2=None, workspace=None, stream=None):
+    """DYAD backward on the GPU: (dX, dW1, dW2)."""
+    import torch
+    nb, ob, ib = W1.shape
+    rows = X.shape[0]
+    _dyad_check(W1, W2, rows, dY=dY, X=X, dX=dX, dW1=dW1, dW2=dW2)
+    dX = torch.empty_like(X) if dX is None else dX
+    dW1 = torch.empty_like(W1) if dW1 is None else dW1
+    dW2 = torch.empty_like(W2) if dW2 is None else dW2
+    dd = dyad_dims(nb, ib, ob, rows, X.dtype)
+    need = int(lib().monarch_dyad_workspace_bytes(ctypes.byref(dd)))
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=X.device)
+    _require_cuda(dY, X, W1, W2, dX, dW1, dW2, workspace)
+    _check("monarch_dyad_bwd", lib().monarch_dyad_bwd(
+        _ptr(dY), _ptr(X), _ptr(W1), _ptr(W2), ctypes.byref(dd), _ptr(dX), _ptr(dW1), _ptr(dW2), _ptr(workspace),
+        ctypes.c_size_t(workspace.numel() * workspace.element_size()), _stream(stream)))
+    return dX, dW1, dW2
 
 
 def kernel_launches() -> int:

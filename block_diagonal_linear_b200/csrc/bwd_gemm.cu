@@ -216,7 +216,7 @@ cudaError_t gemm_bwd(const void* dY, const void* X, const void* R, const void* L
 // memory-bound shapes).  The permutations are per-row transposes:
 //   dV = P_out^-1 dY,  dZ = packed(L^T) dV,  dU = P^-1 dZ,  dX = packed(R^T) dU,
 //   U = packed(R) X,  Z = P U,  then the weight-gradient GEMMs and the partial sum.
-static int pack_factor(int nblocks, int kw, int nw) {
+int pack_factor(int nblocks, int kw, int nw) {
   for (int g = 1; g <= 8; ++g)
     if (nblocks % g == 0 && (g * kw) % 64 == 0 && (g * nw) % 64 == 0) return g;
   return 0;
@@ -278,6 +278,29 @@ __global__ void pack_weights_kernel(const __nv_bfloat16* __restrict__ R, const _
   }
 }
 
+// Wp[grp][jj*nw + n][jj'*kw + k] = W[grp*g + jj][n][k] if jj == jj' (else 0), from W (nb, nw, kw);
+// with trans, W is read as (nb, kw, nw) and transposed: Wp[...][jj*nw + n][jj*kw + k] = W[b][k][n].
+__global__ void pack_bd_kernel(const __nv_bfloat16* __restrict__ W, __nv_bfloat16* __restrict__ Wp, int nb,
+                               int nw, int kw, int g, int trans) {
+  ptx::griddep_wait();
+  ptx::griddep_launch_dependents();
+  const int64_t n_all = (int64_t)nb * nw * g * kw;
+  const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= n_all) return;
+  const int64_t K = (int64_t)g * kw, row = e / K, col = e % K;
+  const int64_t grp = row / ((int64_t)g * nw), rr = row % ((int64_t)g * nw);
+  const int jj = (int)(rr / nw), n = (int)(rr % nw), jk = (int)(col / kw), k = (int)(col % kw);
+  const int64_t b = grp * g + jj;
+  Wp[e] = jj != jk ? __float2bfloat16_rn(0.f)
+                   : (trans ? W[(b * kw + k) * nw + n] : W[(b * nw + n) * kw + k]);
+}
+
+cudaError_t pack_bd(const void* W, void* Wp, int nb, int nw, int kw, int g, bool trans, cudaStream_t st) {
+  const int64_t n_all = (int64_t)nb * nw * g * kw;
+  return launch_kernel(pack_bd_kernel, dim3((unsigned)((n_all + 255) / 256)), dim3(256), 0, st, true,
+                       (const __nv_bfloat16*)W, (__nv_bfloat16*)Wp, nb, nw, kw, g, trans ? 1 : 0);
+}
+
 struct PackedWs {
   size_t wz, wx, wu, dv, dz, du, u, z, part, total;
   WgradSplit sp;
@@ -312,7 +335,7 @@ static PackedWs packed_layout(const Shape& s) {
 size_t packed_bwd_workspace(const Shape& s) { return packed_layout(s).total; }
 
 // Y (rows x nb*nw) = packed block-diagonal stage of A (rows x nb*kw) with W (nb*nw x g*kw per group).
-static cudaError_t packed_stage(const void* A, int64_t rows, const void* W, void* Y, int nb, int kw, int nw, int g,
+cudaError_t packed_stage(const void* A, int64_t rows, const void* W, void* Y, int nb, int kw, int nw, int g,
                                 int* status, cudaStream_t st) {
   GemmJob j = {};
   const int K = g * kw, N = g * nw;

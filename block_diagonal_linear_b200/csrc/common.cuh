@@ -112,8 +112,10 @@ cudaError_t tc_split_fwd(const void* X, const void* R, const void* L, void* Y, c
 // Y[r][k*64 + n] = sum_i W[k][n][i] X[r][k*64 + i] (bf16, 64 x 64 blocks; Y may equal X).
 cudaError_t bdgemm64(const void* X, const void* W, void* Y, int nb, int64_t rows, int* status,
                      cudaStream_t st, bool pdl);
-// dst[r][b*A + a] = src[r][a*B + b] (bf16; dst may equal src).
+// dst[r][b*A + a] = src[r][a*B + b] (bf16; dst may equal src; A, B multiples of 8).
 cudaError_t permute_rows(const void* src, void* dst, int64_t rows, int A, int B, cudaStream_t st);
+// dst[r][b*A + a] += src[r][a*B + b] (bf16, fp32 add rounded once; dst distinct from src).
+cudaError_t permute_rows_add(const void* src, void* dst, int64_t rows, int A, int B, cudaStream_t st);
 
 // Tensor-core backward of the square small-block shapes (bf16).
 bool fast_bwd_supported(const Shape& s);

@@ -60,6 +60,15 @@ cudaError_t wgrad_tc(const void* A1, int64_t a_cols, int64_t blk_a, const void* 
                      int64_t nblocks, int b_base, int b_grp, int b_gs, int64_t pm_a, int64_t pm_b, int64_t rows,
                      WgradSplit sp, float* partial, int64_t p_stride, int64_t p_off, int* status, cudaStream_t st);
 
+// Smallest g <= 8 dividing nblocks with g*kw and g*nw multiples of 64 (0 if none).
+int pack_factor(int nblocks, int kw, int nw);
+// Packed block-diagonal weights (see bwd_gemm.cu) and the stage that uses them.
+cudaError_t pack_bd(const void* W, void* Wp, int nb, int nw, int kw, int g, bool trans, cudaStream_t st);
+cudaError_t packed_stage(const void* A, int64_t rows, const void* W, void* Y, int nb, int kw, int nw, int g,
+                         int* status, cudaStream_t st);
+__global__ void reduce_partials_kernel(const float* __restrict__ partial, __nv_bfloat16* __restrict__ dR,
+                                       __nv_bfloat16* __restrict__ dL, int64_t nR, int64_t nP, int nsplit);
+
 bool packed_bwd_supported(const Shape& s);
 size_t packed_bwd_workspace(const Shape& s);
 cudaError_t packed_bwd(const void* dY, const void* X, const void* R, const void* L, void* dX, void* dR, void* dL,

@@ -218,7 +218,9 @@ __global__ void __launch_bounds__(kBdThreads, 1)
 // dst[r][b*A + a] = src[r][a*B + b]: per row an (A x B) -> (B x A) transpose.  One warp per
 // row: the whole row is read with 16-byte loads into shared memory (odd word pitch, so the
 // column reads hit 32 banks) before any of it is written, so src may equal dst.
+// With ACC, dst[r][b*A + a] = round(dst[r][b*A + a] + src[r][a*B + b]) (src and dst distinct).
 constexpr int kPermWarps = 8;
+template <bool ACC>
 __global__ void __launch_bounds__(kPermWarps * 32)
     permute_rows_kernel(const __nv_bfloat16* src, __nv_bfloat16* dst, int64_t rows, int A, int B) {
   extern __shared__ __align__(16) uint32_t shw[];
@@ -243,6 +245,16 @@ __global__ void __launch_bounds__(kPermWarps * 32)
 #pragma unroll
       for (int e = 0; e < 4; ++e)
         w[e] = (uint32_t)hb[(a0 + 2 * e) * pitch + b] | ((uint32_t)hb[(a0 + 2 * e + 1) * pitch + b] << 16);
+      if (ACC) {
+        const uint4 o = *(const uint4*)(d + c * 8);
+        const uint32_t ov[4] = {o.x, o.y, o.z, o.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float lo = __uint_as_float(ov[e] << 16) + __uint_as_float(w[e] << 16);
+          const float hi = __uint_as_float(ov[e] & 0xFFFF0000u) + __uint_as_float(w[e] & 0xFFFF0000u);
+          w[e] = ptx::pack_bf16x2(lo, hi);
+        }
+      }
       *(uint4*)(d + c * 8) = make_uint4(w[0], w[1], w[2], w[3]);
     }
     __syncwarp();
@@ -266,14 +278,23 @@ static cudaError_t launch_bdgemm(const void* X, const void* W, void* Y, int nb, 
                        mX, mW, mY, nb, rows, status);
 }
 
-cudaError_t permute_rows(const void* src, void* dst, int64_t rows, int A, int B, cudaStream_t st) {
+template <bool ACC>
+static cudaError_t launch_permute(const void* src, void* dst, int64_t rows, int A, int B, cudaStream_t st) {
   if (rows == 0) return cudaSuccess;
   const size_t smem = (size_t)kPermWarps * (size_t)A * (size_t)(B + 2) * 2;
-  cudaError_t e = cudaFuncSetAttribute(permute_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  cudaError_t e = cudaFuncSetAttribute(permute_rows_kernel<ACC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return e;
-  return launch_kernel(permute_rows_kernel, dim3(2 * 148), dim3(kPermWarps * 32), smem, st, true,
+  return launch_kernel(permute_rows_kernel<ACC>, dim3(2 * 148), dim3(kPermWarps * 32), smem, st, true,
                        (const __nv_bfloat16*)src, (__nv_bfloat16*)dst, rows, A, B);
+}
+
+cudaError_t permute_rows(const void* src, void* dst, int64_t rows, int A, int B, cudaStream_t st) {
+  return launch_permute<false>(src, dst, rows, A, B, st);
+}
+
+cudaError_t permute_rows_add(const void* src, void* dst, int64_t rows, int A, int B, cudaStream_t st) {
+  return launch_permute<true>(src, dst, rows, A, B, st);
 }
 
 using Bd64 = BdCfg<64, 64>;

@@ -225,6 +225,37 @@ MONARCH_API int monarch_linear_bwd(const void* dY, const void* X, const void* R,
                                    const monarch_linear_dims* ld, void* dX, void* dR, void* dL,
                                    void* dbias, void* workspace, size_t workspace_bytes, void* stream);
 
+/* ---------------------------------------------------------------- DYAD
+ * DYAD abstract (mlsanity summary): a weight that is the sum of two matrices, each permutable
+ * to a block-sparse counterpart and stored as a 3-D tensor.  The abstract fixes no
+ * permutation; this library takes the reshape-transpose of the Monarch pages on both sides of
+ * the second term:
+ *   y = BD(W1) x + P_out^T BD(W2) P_in x,
+ *   (P_in x)[i*nb + k] = x[k*in_blk + i],   (P_out^T v)[k*out_blk + a] = v[a*nb + k],
+ * with W1, W2 of shape (nblocks, out_blk, in_blk), X (rows, nblocks*in_blk), Y (rows,
+ * nblocks*out_blk), and BD(W) the block-diagonal product on contiguous slices. */
+typedef struct {
+  int64_t rows;
+  int32_t nblocks, in_blk, out_blk;
+  int32_t dtype;          /* monarch_dtype of every tensor argument */
+} monarch_dyad_dims;
+
+/* Workspace bytes monarch_dyad_fwd / _bwd need (0 if dd is bad).  Host-only. */
+MONARCH_API size_t monarch_dyad_workspace_bytes(const monarch_dyad_dims* dd);
+/* 1 = tcgen05 path (bf16, packable blocks, multiples of 8), 0 = generic FMA kernels, -1 = bad
+ * dims.  Host-only. */
+MONARCH_API int monarch_dyad_path(const monarch_dyad_dims* dd);
+/* Y = DYAD(X).  Caller-owned device memory; the workspace (>= monarch_dyad_workspace_bytes,
+ * 256-byte aligned) may be NULL when that size is the 256-byte minimum of the generic path.
+ * Outputs and workspace must not overlap the inputs or one another (MONARCH_ERR_ALIAS). */
+MONARCH_API int monarch_dyad_fwd(const void* X, const void* W1, const void* W2, const monarch_dyad_dims* dd,
+                                 void* Y, void* workspace, size_t workspace_bytes, void* stream);
+/* (dX, dW1, dW2) of Y = DYAD(X) for the upstream gradient dY (chain rule), all overwritten;
+ * weight gradients are summed over rows in a fixed order.  Same rules as monarch_dyad_fwd. */
+MONARCH_API int monarch_dyad_bwd(const void* dY, const void* X, const void* W1, const void* W2,
+                                 const monarch_dyad_dims* dd, void* dX, void* dW1, void* dW2,
+                                 void* workspace, size_t workspace_bytes, void* stream);
+
 /* Number of kernels this library has launched in this process (every device and
  * stream), counted on the host at each successful launch.  Host-only; a caller
  * reads it before and after a region to count that region's launches. */

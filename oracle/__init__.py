@@ -240,3 +240,64 @@ def project(d: dict, M) -> tuple[np.ndarray, np.ndarray]:
             L[j, :, k] = np.sqrt(s) * u
             R[k, j, :] = np.sqrt(s) * v
     return R, L
+
+
+# ---------------------------------------------------------------- DYAD
+# DYAD abstract (mlsanity summary): the weight is a sum of two matrices, each permutable to a
+# block-sparse counterpart and stored as a 3-D tensor.  The abstract fixes no permutation;
+# the reading taken here uses the reshape-transpose of the Monarch pages on both sides of the
+# second term:
+#   y = BD(W1) x + P_out^T BD(W2) P_in x,
+#   (P_in x)[i*nb + k] = x[k*in_blk + i]          (view (nb, in_blk), transpose, flatten)
+#   (P_out^T v)[k*out_blk + a] = v[a*nb + k]      (the inverse transpose on the output side)
+# with W1, W2 of shape (nb, out_blk, in_blk) and BD the block-diagonal product on contiguous
+# slices: (BD(W) x)[b*out_blk + o] = sum_i W[b][o][i] x[b*in_blk + i].
+
+def _bd(W, x):
+    nb, ob, ib = W.shape
+    out = np.empty((x.shape[0], nb * ob))
+    for b in range(nb):
+        out[:, b * ob:(b + 1) * ob] = x[:, b * ib:(b + 1) * ib] @ W[b].T
+    return out
+
+
+def dyad_forward(W1, W2, X) -> np.ndarray:
+    """y = BD(W1) x + P_out^T BD(W2) P_in x for every row x, in fp64 (steps in that order)."""
+    W1, W2, X = _f64(W1), _f64(W2), _f64(X)
+    nb, ob, ib = W1.shape
+    X = X.reshape(-1, nb * ib)
+    y1 = _bd(W1, X)
+    Px = np.empty_like(X)
+    for k in range(nb):
+        for i in range(ib):
+            Px[:, i * nb + k] = X[:, k * ib + i]
+    v = _bd(W2, Px)
+    y2 = np.empty_like(v)
+    for k in range(nb):
+        for a in range(ob):
+            y2[:, k * ob + a] = v[:, a * nb + k]
+    return y1 + y2
+
+
+def dyad_backward(W1, W2, X, dY):
+    """(dX, dW1, dW2) of dyad_forward by the chain rule, in fp64."""
+    W1, W2, X, dY = _f64(W1), _f64(W2), _f64(X), _f64(dY)
+    nb, ob, ib = W1.shape
+    X = X.reshape(-1, nb * ib)
+    dY = dY.reshape(-1, nb * ob)
+    Px = np.empty_like(X)
+    for k in range(nb):
+        for i in range(ib):
+            Px[:, i * nb + k] = X[:, k * ib + i]
+    dv = np.empty_like(dY)                      # gradient of v: inverse of the output transpose
+    for k in range(nb):
+        for a in range(ob):
+            dv[:, a * nb + k] = dY[:, k * ob + a]
+    dW1 = np.stack([dY[:, b * ob:(b + 1) * ob].T @ X[:, b * ib:(b + 1) * ib] for b in range(nb)])
+    dW2 = np.stack([dv[:, b * ob:(b + 1) * ob].T @ Px[:, b * ib:(b + 1) * ib] for b in range(nb)])
+    dX = _bd(np.transpose(W1, (0, 2, 1)), dY)
+    dPx = _bd(np.transpose(W2, (0, 2, 1)), dv)
+    for k in range(nb):
+        for i in range(ib):
+            dX[:, k * ib + i] += dPx[:, i * nb + k]
+    return dX, dW1, dW2
