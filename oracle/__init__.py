@@ -301,3 +301,78 @@ def dyad_backward(W1, W2, X, dY):
         for i in range(ib):
             dX[:, k * ib + i] += dPx[:, i * nb + k]
     return dX, dW1, dW2
+
+
+# ---------------------------------------------------------------- lattice (hypercube) Monarch
+# Scatterbrain thread, the unofficial-implementation comment: view the n inputs as a lattice
+# (for n = N the 2-D m x m square; for width 12288 the 3-D lattice [16, 24, 32]); one round per
+# dimension applies a separate matrix to every line of the lattice along that dimension
+# (768 matrices of 16 x 16 for the first dimension, 512 of 24 x 24 for the second, 384 for the
+# third).  Readings taken: a row x is the lattice in row-major order (last axis contiguous);
+# the rounds run from the last axis to the first, so that with two axes the map is the
+# two-factor product with the output transpose (R on the contiguous rows of the square, L on
+# its columns); a round may change the length of its axis (n_t -> m_t, the "uneven rectangle"
+# of the same comment); the matrices of round t are indexed by the row-major position of the
+# line in the other axes at that point (axes already done count with their new lengths); the
+# output is the final lattice in row-major order.
+
+def lattice_shapes(n_in: list, n_out: list) -> list:
+    """Weight shapes (lines, m_t, n_t) of every round t (index t = axis)."""
+    d = len(n_in)
+    shapes = [None] * d
+    cur = list(n_in)
+    for t in range(d - 1, -1, -1):
+        lines = int(np.prod([cur[s] for s in range(d) if s != t]))
+        shapes[t] = (lines, n_out[t], n_in[t])
+        cur[t] = n_out[t]
+    return shapes
+
+
+def lattice_forward(n_in: list, n_out: list, Ws: list, X) -> np.ndarray:
+    """Rounds t = d-1 .. 0 over the lattice of every row, in fp64 (plain loops over lines)."""
+    d = len(n_in)
+    X = _f64(X)
+    rows = X.shape[0]
+    cur = list(n_in)
+    A = X.reshape([rows] + cur)
+    for t in range(d - 1, -1, -1):
+        W = _f64(Ws[t])
+        others = [s for s in range(d) if s != t]
+        # move axis t last, lines in row-major order of the other axes
+        At = np.moveaxis(A, 1 + t, -1).reshape(rows, -1, cur[t])
+        Bt = np.empty((rows, At.shape[1], n_out[t]))
+        for line in range(At.shape[1]):
+            Bt[:, line, :] = At[:, line, :] @ W[line].T
+        shape_o = [rows] + [cur[s] for s in others] + [n_out[t]]
+        A = np.moveaxis(Bt.reshape(shape_o), -1, 1 + t)
+        cur[t] = n_out[t]
+    return np.ascontiguousarray(A.reshape(rows, -1))
+
+
+def lattice_backward(n_in: list, n_out: list, Ws: list, X, dY):
+    """(dX, [dW_t]) of lattice_forward by the chain rule (inputs of every round recomputed)."""
+    d = len(n_in)
+    X, dY = _f64(X), _f64(dY)
+    rows = X.shape[0]
+    cur = list(n_in)
+    A = X.reshape([rows] + cur)
+    saved = {}
+    for t in range(d - 1, -1, -1):                     # forward, keeping each round's input
+        W = _f64(Ws[t])
+        others = [s for s in range(d) if s != t]
+        At = np.moveaxis(A, 1 + t, -1).reshape(rows, -1, cur[t])
+        saved[t] = (At, list(cur))
+        Bt = np.einsum("rli,loi->rlo", At, W)
+        A = np.moveaxis(Bt.reshape([rows] + [cur[s] for s in others] + [n_out[t]]), -1, 1 + t)
+        cur[t] = n_out[t]
+    G = dY.reshape([rows] + cur)
+    dWs = [None] * d
+    for t in range(d):                                  # backward, rounds in reverse order
+        W = _f64(Ws[t])
+        At, cin = saved[t]
+        others = [s for s in range(d) if s != t]
+        Gt = np.moveaxis(G, 1 + t, -1).reshape(rows, -1, n_out[t])
+        dWs[t] = np.einsum("rlo,rli->loi", Gt, At)
+        dAt = np.einsum("rlo,loi->rli", Gt, W)
+        G = np.moveaxis(dAt.reshape([rows] + [cin[s] for s in others] + [cin[t]]), -1, 1 + t)
+    return np.ascontiguousarray(G.reshape(rows, -1)), dWs
