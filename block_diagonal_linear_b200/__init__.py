@@ -17,6 +17,8 @@ from __future__ import annotations
 import ctypes
 import os
 
+import numpy as np
+
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libmonarch.so")
 
@@ -44,7 +46,8 @@ EXPORTED = (
     "monarch_debug_wait_timeout", "monarch_fwd_path", "monarch_bwd_path", "monarch_bwd_noalloc",
     "monarch_kernel_launches", "monarch_linear_shape", "monarch_linear_workspace_bytes",
     "monarch_linear_fwd", "monarch_linear_bwd", "monarch_project", "monarch_dyad_workspace_bytes",
-    "monarch_dyad_path", "monarch_dyad_fwd", "monarch_dyad_bwd",
+    "monarch_dyad_path", "monarch_dyad_fwd", "monarch_dyad_bwd", "monarch_lattice_workspace_bytes",
+    "monarch_lattice_path", "monarch_lattice_weight_elems", "monarch_lattice_fwd", "monarch_lattice_bwd",
 )
 
 
@@ -82,6 +85,17 @@ class MonarchDyadDims(ctypes.Structure):
         ("nblocks", ctypes.c_int32),
         ("in_blk", ctypes.c_int32),
         ("out_blk", ctypes.c_int32),
+        ("dtype", ctypes.c_int32),
+    ]
+
+
+class MonarchLatticeDims(ctypes.Structure):
+    """Mirror of ``monarch_lattice_dims`` in include/monarch.h."""
+    _fields_ = [
+        ("rows", ctypes.c_int64),
+        ("naxes", ctypes.c_int32),
+        ("n_in", ctypes.c_int32 * 4),
+        ("n_out", ctypes.c_int32 * 4),
         ("dtype", ctypes.c_int32),
     ]
 
@@ -139,6 +153,18 @@ def lib() -> ctypes.CDLL:
         L.monarch_dyad_fwd.restype = ctypes.c_int
         L.monarch_dyad_bwd.argtypes = [vp, vp, vp, vp, yp, vp, vp, vp, vp, ctypes.c_size_t, vp]
         L.monarch_dyad_bwd.restype = ctypes.c_int
+        tp = ctypes.POINTER(MonarchLatticeDims)
+        pp = ctypes.POINTER(ctypes.c_void_p)
+        L.monarch_lattice_workspace_bytes.argtypes = [tp]
+        L.monarch_lattice_workspace_bytes.restype = ctypes.c_size_t
+        L.monarch_lattice_path.argtypes = [tp]
+        L.monarch_lattice_path.restype = ctypes.c_int
+        L.monarch_lattice_weight_elems.argtypes = [tp, ctypes.c_int32]
+        L.monarch_lattice_weight_elems.restype = ctypes.c_int64
+        L.monarch_lattice_fwd.argtypes = [vp, pp, tp, vp, vp, ctypes.c_size_t, vp]
+        L.monarch_lattice_fwd.restype = ctypes.c_int
+        L.monarch_lattice_bwd.argtypes = [vp, vp, pp, tp, vp, pp, vp, ctypes.c_size_t, vp]
+        L.monarch_lattice_bwd.restype = ctypes.c_int
         for name in ("monarch_validate", "monarch_fwd", "monarch_bwd", "monarch_materialise",
                      "monarch_last_device_status", "monarch_debug_wait_timeout",
                      "monarch_fwd_path", "monarch_bwd_path", "monarch_bwd_noalloc"):
@@ -481,6 +507,69 @@ def dyad_bwd(dY, X, W1, W2, dX=None, dW1=None, dW2=None, workspace=None, stream=
         _ptr(dY), _ptr(X), _ptr(W1), _ptr(W2), ctypes.byref(dd), _ptr(dX), _ptr(dW1), _ptr(dW2), _ptr(workspace),
         ctypes.c_size_t(workspace.numel() * workspace.element_size()), _stream(stream)))
     return dX, dW1, dW2
+
+
+# ---------------------------------------------------------------- lattice (hypercube) Monarch
+def lattice_dims(n_in, n_out, rows: int, dtype="bf16") -> MonarchLatticeDims:
+    if not 1 <= len(n_in) == len(n_out) <= 4:
+        raise ValueError("1 to 4 axes, n_in and n_out of one length")
+    d = MonarchLatticeDims()
+    d.rows, d.naxes, d.dtype = int(rows), len(n_in), dtype_code(dtype)
+    for a, (ni, no) in enumerate(zip(n_in, n_out)):
+        d.n_in[a], d.n_out[a] = int(ni), int(no)
+    return d
+
+
+def lattice_weight_shapes(n_in, n_out) -> list:
+    """(lines, n_out[t], n_in[t]) of every axis t, from the library's host-side rule."""
+    d = lattice_dims(n_in, n_out, 0, "f32")
+    out = []
+    for t in range(len(n_in)):
+        n = int(lib().monarch_lattice_weight_elems(ctypes.byref(d), t))
+        out.append((n // (n_out[t] * n_in[t]), n_out[t], n_in[t]))
+    return out
+
+
+def lattice_path(n_in, n_out, dtype="bf16") -> int:
+    return lib().monarch_lattice_path(ctypes.byref(lattice_dims(n_in, n_out, 1, dtype)))
+
+
+def _ptr_array(ts):
+    return (ctypes.c_void_p * len(ts))(*[t.data_ptr() for t in ts])
+
+
+def lattice_fwd(X, Ws, n_in, n_out, Y=None, workspace=None, stream=None):
+    """Lattice Monarch forward on the GPU; Ws[t] is the weight tensor of axis t."""
+    import torch
+    rows = X.shape[0]
+    if Y is None:
+        Y = torch.empty((rows, int(np.prod(n_out))), dtype=X.dtype, device=X.device)
+    d = lattice_dims(n_in, n_out, rows, X.dtype)
+    need = int(lib().monarch_lattice_workspace_bytes(ctypes.byref(d)))
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=X.device)
+    _require_cuda(X, Y, workspace, *Ws)
+    _check("monarch_lattice_fwd", lib().monarch_lattice_fwd(
+        _ptr(X), _ptr_array(Ws), ctypes.byref(d), _ptr(Y), _ptr(workspace),
+        ctypes.c_size_t(workspace.numel() * workspace.element_size()), _stream(stream)))
+    return Y
+
+
+def lattice_bwd(dY, X, Ws, n_in, n_out, workspace=None, stream=None):
+    """Lattice Monarch backward on the GPU: (dX, [dW_t])."""
+    import torch
+    rows = X.shape[0]
+    dX = torch.empty_like(X)
+    dWs = [torch.empty_like(w) for w in Ws]
+    d = lattice_dims(n_in, n_out, rows, X.dtype)
+    need = int(lib().monarch_lattice_workspace_bytes(ctypes.byref(d)))
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=X.device)
+    _require_cuda(dY, X, dX, workspace, *Ws, *dWs)
+    _check("monarch_lattice_bwd", lib().monarch_lattice_bwd(
+        _ptr(dY), _ptr(X), _ptr_array(Ws), ctypes.byref(d), _ptr(dX), _ptr_array(dWs), _ptr(workspace),
+        ctypes.c_size_t(workspace.numel() * workspace.element_size()), _stream(stream)))
+    return dX, dWs
 
 
 def kernel_launches() -> int:

@@ -242,8 +242,8 @@ bool packed_bwd_supported(const Shape& s) {
   // packed operand widths (K stages of 64, N tiles of 64..256) and the row-transpose passes
   if ((int64_t)p.gz * s.out2 > 4096 || (int64_t)p.gx * s.in1 > 4096 || (int64_t)p.gx * s.out1 > 4096) return false;
   if (s.n_in() > 65536 || s.n_mid() > 65536 || s.n_out() > 65536) return false;
-  if ((int64_t)8 * s.out2 * (s.nb2 + 2) * 2 > 200 * 1024 || (int64_t)8 * s.nb1 * (s.out1 + 2) * 2 > 200 * 1024 ||
-      (int64_t)8 * s.out1 * (s.nb1 + 2) * 2 > 200 * 1024)
+  if ((int64_t)s.out2 * (s.nb2 + 2) * 2 > 200 * 1024 || (int64_t)s.nb1 * (s.out1 + 2) * 2 > 200 * 1024 ||
+      (int64_t)s.out1 * (s.nb1 + 2) * 2 > 200 * 1024)
     return false;
   return true;
 }

@@ -36,8 +36,8 @@ static bool dyad_tc(const DyadShape& s, int dtype) {
   if (pack_factor(s.nb, s.ib, s.ob) == 0 || pack_factor(s.nb, s.ob, s.ib) == 0) return false;
   const int64_t n_in = (int64_t)s.nb * s.ib, n_out = (int64_t)s.nb * s.ob;
   if (n_in > 65536 || n_out > 65536) return false;
-  if ((int64_t)8 * s.nb * (s.ib + 2) * 2 > 200 * 1024 || (int64_t)8 * s.ob * (s.nb + 2) * 2 > 200 * 1024 ||
-      (int64_t)8 * s.nb * (s.ob + 2) * 2 > 200 * 1024 || (int64_t)8 * s.ib * (s.nb + 2) * 2 > 200 * 1024)
+  if ((int64_t)s.nb * (s.ib + 2) * 2 > 200 * 1024 || (int64_t)s.ob * (s.nb + 2) * 2 > 200 * 1024 ||
+      (int64_t)s.nb * (s.ob + 2) * 2 > 200 * 1024 || (int64_t)s.ib * (s.nb + 2) * 2 > 200 * 1024)
     return false;
   return true;
 }

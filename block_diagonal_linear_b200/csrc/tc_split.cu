@@ -12,6 +12,8 @@
 // TMA-friendly), warp 1 issues M = 128, N = 64 MMAs into one of two TMEM slots, warps 2..5
 // drain TMEM (one row per thread), round to bf16 into one of two 128B-swizzled staging tiles
 // and one thread writes the tile with TMA stores.  All waits are bounded (tc_common.cuh).
+#include <algorithm>
+
 #include "tc_common.cuh"
 
 namespace monarch {
@@ -230,7 +232,8 @@ __global__ void __launch_bounds__(kPermWarps * 32)
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   uint32_t* buf = shw + warp * (A * wpitch);
   const uint16_t* hb = (const uint16_t*)buf;
-  for (int64_t r = (int64_t)blockIdx.x * kPermWarps + warp; r < rows; r += (int64_t)gridDim.x * kPermWarps) {
+  const int nwarps = blockDim.x / 32;  // one staged row per warp
+  for (int64_t r = (int64_t)blockIdx.x * nwarps + warp; r < rows; r += (int64_t)gridDim.x * nwarps) {
     const __nv_bfloat16* s = src + r * n;
     for (int c = lane; c < n / 8; c += 32) {  // source chunk: a = 8c / B, b0 = 8c % B
       const uint4 v = *(const uint4*)(s + c * 8);
@@ -281,11 +284,16 @@ static cudaError_t launch_bdgemm(const void* X, const void* W, void* Y, int nb, 
 template <bool ACC>
 static cudaError_t launch_permute(const void* src, void* dst, int64_t rows, int A, int B, cudaStream_t st) {
   if (rows == 0) return cudaSuccess;
-  const size_t smem = (size_t)kPermWarps * (size_t)A * (size_t)(B + 2) * 2;
+  // one staged row per warp: as many warps (up to 8) as shared memory holds rows
+  const size_t row_smem = (size_t)A * (size_t)(B + 2) * 2;
+  const size_t cap = 200 * 1024;
+  if (row_smem > cap) return cudaErrorInvalidValue;
+  const int nwarps = (int)std::min<size_t>(kPermWarps, cap / row_smem);
+  const size_t smem = (size_t)nwarps * row_smem;
   cudaError_t e = cudaFuncSetAttribute(permute_rows_kernel<ACC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return e;
-  return launch_kernel(permute_rows_kernel<ACC>, dim3(2 * 148), dim3(kPermWarps * 32), smem, st, true,
+  return launch_kernel(permute_rows_kernel<ACC>, dim3(2 * 148), dim3(nwarps * 32), smem, st, true,
                        (const __nv_bfloat16*)src, (__nv_bfloat16*)dst, rows, A, B);
 }
 

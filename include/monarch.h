@@ -256,6 +256,39 @@ MONARCH_API int monarch_dyad_bwd(const void* dY, const void* X, const void* W1, 
                                  const monarch_dyad_dims* dd, void* dX, void* dW1, void* dW2,
                                  void* workspace, size_t workspace_bytes, void* stream);
 
+/* ---------------------------------------------------------------- lattice (hypercube) Monarch
+ * Scatterbrain thread, the unofficial-implementation comment: a row viewed as a lattice with
+ * naxes dimensions (row-major, last axis contiguous), one round of per-line matrices per
+ * dimension (for width 12288 = 16 x 24 x 32: 768 matrices of 16 x 16, 512 of 24 x 24, 384 of
+ * 32 x 32).  Readings taken: rounds run from the last axis to the first; round t maps axis t
+ * from n_in[t] to n_out[t]; its weights W[t] have shape (lines_t, n_out[t], n_in[t]), line
+ * index = row-major position in the other axes at that point (axes already done count with
+ * their new lengths; monarch_lattice_weight_elems gives the element count); the output is the
+ * final lattice in row-major order.  Two axes give the two-factor product with the output
+ * transpose (W[1] = R, W[0] = L). */
+typedef struct {
+  int64_t rows;
+  int32_t naxes;          /* 1 .. 4 */
+  int32_t n_in[4], n_out[4];
+  int32_t dtype;          /* monarch_dtype of every tensor argument */
+} monarch_lattice_dims;
+
+MONARCH_API size_t monarch_lattice_workspace_bytes(const monarch_lattice_dims* ld);
+/* 1 = tcgen05 path (bf16, packable lines, lengths multiples of 8), 0 = generic FMA kernels. */
+MONARCH_API int monarch_lattice_path(const monarch_lattice_dims* ld);
+/* Elements of W[axis] (lines * n_out[axis] * n_in[axis]), -1 on bad arguments.  Host-only. */
+MONARCH_API int64_t monarch_lattice_weight_elems(const monarch_lattice_dims* ld, int32_t axis);
+/* Y (rows, prod n_out) = rounds of W over X (rows, prod n_in).  W: host array of naxes device
+ * pointers (W[t] for axis t).  workspace: >= monarch_lattice_workspace_bytes(ld), 256-byte
+ * aligned.  Same conventions as monarch_fwd. */
+MONARCH_API int monarch_lattice_fwd(const void* X, const void* const* W, const monarch_lattice_dims* ld, void* Y,
+                                    void* workspace, size_t workspace_bytes, void* stream);
+/* (dX, dW[t]) for the upstream gradient dY; dW: host array of naxes device pointers; all
+ * outputs overwritten, weight gradients summed over rows in a fixed order. */
+MONARCH_API int monarch_lattice_bwd(const void* dY, const void* X, const void* const* W,
+                                    const monarch_lattice_dims* ld, void* dX, void* const* dW, void* workspace,
+                                    size_t workspace_bytes, void* stream);
+
 /* Number of kernels this library has launched in this process (every device and
  * stream), counted on the host at each successful launch.  Host-only; a caller
  * reads it before and after a region to count that region's launches. */
