@@ -233,7 +233,7 @@ def launches(shape: dict, dtype: str, pname: str) -> int:
     dY = torch.zeros((1, n_out), dtype=dt, device="cuda")
     n0 = bdl.kernel_launches()
     if pname == "fwd":
-        bdl.fwd(X, R, L, shape)
+        bdl.fwd_ws(X, R, L, shape)
     else:
         bdl.bwd(dY, X, R, L, shape)
     torch.cuda.synchronize()
@@ -273,13 +273,16 @@ def time_shape(name, dev, flush, peaks, reps=10, warmup=3, spin_cycles=400000):
     ws = torch.empty(max(bdl.bwd_workspace_bytes(shape, rows, w["dtype"]), 256), dtype=torch.uint8,
                      device=dev)
     stream = torch.cuda.current_stream()
-    runs = {"fwd": lambda: bdl.fwd(X, R, L, shape, Y=Y),
+    # the forward with caller scratch: the two-pass GEMM path where it applies, else monarch_fwd
+    fws = bdl.fwd_workspace_bytes(shape, rows, w["dtype"])
+    fwd_ws = torch.empty(fws, dtype=torch.uint8, device=dev) if fws else None
+    runs = {"fwd": lambda: bdl.fwd_ws(X, R, L, shape, Y=Y, workspace=fwd_ws),
             "bwd": lambda: bdl.bwd(dY, X, R, L, shape, dX=dX, dR=dR, dL=dL, workspace=ws)}
     alg = algorithmic(w, rows)
     hbm, tpk = peaks["hbm_gbs"] * 1e9, peaks["bf16_tflops"] * 1e12
     if w["dtype"] == "f32":
         tpk = FFMA_TFLOPS * 1e12
-    res = {"workload": describe(name, w), "fwd_path": bdl.fwd_path(shape, w["dtype"]),
+    res = {"workload": describe(name, w), "fwd_path": bdl.fwd_ws_path(shape, w["dtype"]),
            "bwd_path": bdl.bwd_path(shape, w["dtype"])}
     for pname, fn in runs.items():
         evs = []
@@ -303,10 +306,11 @@ def time_shape(name, dev, flush, peaks, reps=10, warmup=3, spin_cycles=400000):
             "bound": "hbm" if a["bytes"] / hbm >= a["flops"] / tpk else
                      ("fma" if w["dtype"] == "f32" else "tensor"),
             "launches": launches(shape, w["dtype"], pname),
+            "entry": "monarch_fwd_ws" if pname == "fwd" else "monarch_bwd",
         }
     if bdl.last_device_status() != 0:
         raise SystemExit("device status not OK after timing %s" % name)
-    del X, R, L, dY, Y, dX, dR, dL, ws, d
+    del X, R, L, dY, Y, dX, dR, dL, ws, d, fwd_ws
     torch.cuda.empty_cache()
     return res
 

@@ -44,7 +44,8 @@ EXPORTED = (
     "monarch_validate", "monarch_fwd", "monarch_bwd", "monarch_bwd_workspace_bytes",
     "monarch_materialise", "monarch_status_string", "monarch_last_device_status",
     "monarch_debug_wait_timeout", "monarch_fwd_path", "monarch_bwd_path", "monarch_bwd_noalloc",
-    "monarch_kernel_launches", "monarch_linear_shape", "monarch_linear_workspace_bytes",
+    "monarch_kernel_launches", "monarch_fwd_workspace_bytes", "monarch_fwd_ws_path", "monarch_fwd_ws",
+    "monarch_linear_shape", "monarch_linear_workspace_bytes",
     "monarch_linear_fwd", "monarch_linear_bwd", "monarch_project", "monarch_dyad_workspace_bytes",
     "monarch_dyad_path", "monarch_dyad_fwd", "monarch_dyad_bwd", "monarch_lattice_workspace_bytes",
     "monarch_lattice_path", "monarch_lattice_weight_elems", "monarch_lattice_fwd", "monarch_lattice_bwd",
@@ -131,6 +132,12 @@ def lib() -> ctypes.CDLL:
         L.monarch_bwd_noalloc.argtypes = [vp, vp, vp, vp, dp, vp, vp, vp, vp]
         L.monarch_fwd_path.argtypes = [dp]
         L.monarch_bwd_path.argtypes = [dp]
+        L.monarch_fwd_workspace_bytes.argtypes = [dp]
+        L.monarch_fwd_workspace_bytes.restype = ctypes.c_size_t
+        L.monarch_fwd_ws_path.argtypes = [dp]
+        L.monarch_fwd_ws_path.restype = ctypes.c_int
+        L.monarch_fwd_ws.argtypes = [vp, vp, vp, dp, vp, vp, ctypes.c_size_t, vp]
+        L.monarch_fwd_ws.restype = ctypes.c_int
         L.monarch_kernel_launches.argtypes = []
         L.monarch_kernel_launches.restype = ctypes.c_uint64
         lp = ctypes.POINTER(MonarchLinearDims)
@@ -270,6 +277,34 @@ def fwd(X, R, L, shape: dict, Y=None, stream=None):
     d = make_dims(shape, rows, code)
     _check("monarch_fwd", lib().monarch_fwd(_ptr(X), _ptr(R), _ptr(L), ctypes.byref(d), _ptr(Y),
                                             _stream(stream)))
+    return Y
+
+
+def fwd_workspace_bytes(shape: dict, rows: int, dtype="bf16") -> int:
+    return int(lib().monarch_fwd_workspace_bytes(ctypes.byref(make_dims(shape, rows, dtype))))
+
+
+def fwd_ws_path(shape: dict, dtype="bf16") -> int:
+    """Kernel family of monarch_fwd_ws: 5 = two-pass tcgen05 GEMM forward, else fwd_path's."""
+    return lib().monarch_fwd_ws_path(ctypes.byref(make_dims(shape, 1, dtype)))
+
+
+def fwd_ws(X, R, L, shape: dict, Y=None, workspace=None, stream=None):
+    """Y = X M^T on the GPU with caller scratch (monarch_fwd_ws); same results as fwd()."""
+    import torch
+    code = dtype_code(X.dtype)
+    rows = X.shape[0]
+    _check_tensors(shape, rows, X.dtype, X=X, R=R, L=L, Y=Y)
+    if Y is None:
+        Y = torch.empty((rows, shape["nb2"] * shape["out2"]), dtype=X.dtype, device=X.device)
+    d = make_dims(shape, rows, code)
+    need = int(lib().monarch_fwd_workspace_bytes(ctypes.byref(d)))
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=X.device)
+    _require_cuda(X, R, L, Y, workspace)
+    nbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check("monarch_fwd_ws", lib().monarch_fwd_ws(_ptr(X), _ptr(R), _ptr(L), ctypes.byref(d), _ptr(Y),
+                                                  _ptr(workspace), ctypes.c_size_t(nbytes), _stream(stream)))
     return Y
 
 

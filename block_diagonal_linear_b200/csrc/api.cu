@@ -186,6 +186,45 @@ int monarch_fwd(const void* X, const void* R, const void* L, const monarch_dims*
   return fwd_dispatch(X, R, L, Y, s, d->dtype, (cudaStream_t)stream);
 }
 
+// Forward with caller scratch: the two-pass tcgen05 GEMM forward where it applies (shapes
+// whose permutation moves whole 64-column groups), otherwise the monarch_fwd kernels.
+static size_t fwd_ws_bytes(const Shape& s, int dtype) {
+  return (dtype == MONARCH_BF16 && gemm_bwd_supported(s)) ? gemm_fwd_workspace(s) : 0;
+}
+
+size_t monarch_fwd_workspace_bytes(const monarch_dims* d) {
+  if (check_dims(d) != MONARCH_OK) return 0;
+  return fwd_ws_bytes(to_shape(*d), d->dtype);
+}
+
+int monarch_fwd_ws_path(const monarch_dims* d) {
+  if (check_dims(d) != MONARCH_OK) return -1;
+  const Shape s = to_shape(*d);
+  return fwd_ws_bytes(s, d->dtype) > 0 ? 5 : fwd_path(s, d->dtype);
+}
+
+int monarch_fwd_ws(const void* X, const void* R, const void* L, const monarch_dims* d, void* Y, void* workspace,
+                   size_t workspace_bytes, void* stream) {
+  int rc = check_dims(d);
+  if (rc != MONARCH_OK) return rc;
+  if (d->rows == 0) return MONARCH_OK;
+  if ((rc = check_ptrs({X, R, L, Y})) != MONARCH_OK) return rc;
+  const Shape s = to_shape(*d);
+  const size_t need = fwd_ws_bytes(s, d->dtype);
+  if (need > 0 && (workspace == nullptr || workspace_bytes < need)) return MONARCH_ERR_WORKSPACE;
+  if (need > 0 && ((uintptr_t)workspace & 255u) != 0) return MONARCH_ERR_ALIGN;
+  const int64_t es = d->dtype == MONARCH_BF16 ? 2 : 4;
+  if ((rc = check_alias({span(Y, s.rows * s.n_out(), es), span(workspace, (int64_t)need, 1)},
+                        {span(X, s.rows * s.n_in(), es), span(R, s.n_R(), es), span(L, s.n_L(), es)})) !=
+      MONARCH_OK)
+    return rc;
+  if (need == 0) return fwd_dispatch(X, R, L, Y, s, d->dtype, (cudaStream_t)stream);
+  int* status = status_ptr();
+  if (status == nullptr) return MONARCH_ERR_CUDA;
+  return gemm_fwd(X, R, L, Y, workspace, s, status, (cudaStream_t)stream) == cudaSuccess ? MONARCH_OK
+                                                                                           : MONARCH_ERR_CUDA;
+}
+
 size_t monarch_bwd_workspace_bytes(const monarch_dims* d) {
   if (check_dims(d) != MONARCH_OK) return 0;
   return bwd_workspace(to_shape(*d), d->dtype);

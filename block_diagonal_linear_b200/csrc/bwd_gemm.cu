@@ -209,6 +209,56 @@ cudaError_t gemm_bwd(const void* dY, const void* X, const void* R, const void* L
                        (const float*)part, (__nv_bfloat16*)dR, (__nv_bfloat16*)dL, nR, nP, w.sp.nsplit);
 }
 
+// ================================================================ two-pass forward
+// Y = X M^T for the same shapes as gemm_bwd, with caller scratch:
+//   1. Lp[j][o][kappa] = L[j][o][q(kappa)]   (kappa = k*G + p', q = p'*nb1 + k)
+//   2. U  = blockdiag(R) X                    (GEMM, block-contiguous u[k][p])
+//   3. Y  = blockdiag(Lp) gathered(U)          (GEMM; block j's K stage kb reads the 64 columns
+//                                             of U at k*out1 + j*G + 64*(kb % (G/64)))
+__global__ void gemm_fwd_prep_kernel(const __nv_bfloat16* __restrict__ L, __nv_bfloat16* __restrict__ Lp, Shape s) {
+  ptx::griddep_wait();
+  ptx::griddep_launch_dependents();
+  const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= s.n_L()) return;
+  const int G = s.in2 / s.nb1;
+  const int kappa = (int)(e % s.in2);
+  const int64_t jo = e / s.in2;  // j*out2 + o
+  const int q = (kappa % G) * s.nb1 + kappa / G;
+  Lp[e] = L[jo * s.in2 + q];
+}
+
+size_t gemm_fwd_workspace(const Shape& s) {
+  return al256((size_t)s.n_L() * 2) + al256((size_t)s.rows * (size_t)s.n_mid() * 2);
+}
+
+cudaError_t gemm_fwd(const void* X, const void* R, const void* L, void* Y, void* ws, const Shape& s, int* status,
+                     cudaStream_t st) {
+  if (s.rows == 0) return cudaSuccess;
+  __nv_bfloat16* Lp = (__nv_bfloat16*)ws;
+  __nv_bfloat16* U = (__nv_bfloat16*)((char*)ws + al256((size_t)s.n_L() * 2));
+  const int G = s.in2 / s.nb1;
+  cudaError_t e;
+  if ((e = launch_kernel(gemm_fwd_prep_kernel, dim3((unsigned)((s.n_L() + 255) / 256)), dim3(256), 0, st, false,
+                         (const __nv_bfloat16*)L, Lp, s)) != cudaSuccess)
+    return e;
+  GemmJob j = {};
+  int bn = pick_bn(s.out1);
+  j.nb = s.nb1; j.ntiles = s.out1 / bn; j.kboxes = s.in1 / 64;
+  j.a_b = s.in1; j.a_grp = s.in1 / 64; j.a_gs = 0;
+  j.b_b = s.out1;
+  j.y_b = s.out1; j.y_grp = s.out1 / 64; j.y_gs = 0;
+  if ((e = gemm_bd(X, s.rows, s.n_in(), R, (int64_t)s.nb1 * s.out1, s.in1, U, s.n_mid(), bn, j, status, st, true)) !=
+      cudaSuccess)
+    return e;
+  j = GemmJob{};
+  bn = pick_bn(s.out2);
+  j.nb = s.nb2; j.ntiles = s.out2 / bn; j.kboxes = s.in2 / 64;
+  j.a_b = G; j.a_grp = G / 64; j.a_gs = s.out1;
+  j.b_b = s.out2;
+  j.y_b = s.out2; j.y_grp = s.out2 / 64; j.y_gs = 0;
+  return gemm_bd(U, s.rows, s.n_mid(), Lp, (int64_t)s.nb2 * s.out2, s.in2, Y, s.n_out(), bn, j, status, st, true);
+}
+
 // ================================================================ packed block-diagonal path
 // Any bf16 shape whose small blocks pack into 64-multiples: g consecutive blocks of a
 // block-diagonal stage are one GEMM against a (g*N) x (g*K) block-diagonal weight tile with

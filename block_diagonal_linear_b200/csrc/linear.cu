@@ -5,12 +5,17 @@
 // Forward:  Xp = [X, 0] (rows x in_ext)  ->  Yp = Monarch(Xp)  ->  Y = Yp[:, :out] + bias.
 // Backward: dYp = [dY, 0] -> (dXp, dR, dL) = Monarch backward -> dX = dXp[:, :in];
 //           dbias = sum over rows of dY.
+// Shapes whose permutation moves whole 64-column groups (e.g. 1024 -> 4096 with 4 blocks) run
+// the two-pass tcgen05 GEMM forward with the middle vector in the workspace.
 // The padding passes are skipped when the features already equal the extended widths, and
 // the output goes through a staging buffer only when it is cropped or gets a bias (the crop
 // and the bias add are one pass that rounds once).  The Monarch stages run on the same
 // kernel families as monarch_fwd / monarch_bwd.
+#include <algorithm>
+
 #include "common.cuh"
 #include "ptx.cuh"
+#include "tc_gemm.cuh"
 
 namespace monarch {
 
@@ -90,7 +95,8 @@ static LinWs lin_layout(const monarch_linear_dims& ld, const Shape& s) {
   // forward: cropped / biased output staging; backward: padded dY
   w.dxp = w.yp + ((pad_out || ld.has_bias) ? al256(rows * (size_t)s.n_out() * es) : 0);
   w.core = w.dxp + (pad_in ? al256(rows * (size_t)s.n_in() * es) : 0);
-  w.bias = w.core + al256(bwd_workspace(s, ld.dtype));
+  const bool two_pass = ld.dtype == MONARCH_BF16 && gemm_bwd_supported(s);
+  w.bias = w.core + al256(std::max(bwd_workspace(s, ld.dtype), two_pass ? gemm_fwd_workspace(s) : (size_t)0));
   const size_t nchunks = (rows + kBiasChunk - 1) / kBiasChunk;
   w.total = w.bias + al256((nchunks > 0 ? nchunks : 1) * (size_t)ld.out_features * 4);
   return w;
@@ -184,7 +190,14 @@ int monarch_linear_fwd(const void* X, const void* R, const void* L, const void* 
     if (e != cudaSuccess) return MONARCH_ERR_CUDA;
   }
   void* Yp = stage_out ? (void*)(ws + w.yp) : Y;
-  if ((rc = fwd_dispatch(Xp, R, L, Yp, s, ld->dtype, st)) != MONARCH_OK) return rc;
+  if (ld->dtype == MONARCH_BF16 && gemm_bwd_supported(s)) {
+    // two-pass tcgen05 GEMM forward with the middle vector in the workspace
+    int* status = status_ptr();
+    if (status == nullptr) return MONARCH_ERR_CUDA;
+    if (gemm_fwd(Xp, R, L, Yp, ws + w.core, s, status, st) != cudaSuccess) return MONARCH_ERR_CUDA;
+  } else if ((rc = fwd_dispatch(Xp, R, L, Yp, s, ld->dtype, st)) != MONARCH_OK) {
+    return rc;
+  }
   if (stage_out) {
     const void* b = ld->has_bias ? bias : nullptr;
     cudaError_t e = bf ? launch_crop<__nv_bfloat16>(Yp, s.n_out(), b, Y, ld->out_features, rows, st)

@@ -74,6 +74,10 @@ size_t packed_bwd_workspace(const Shape& s);
 cudaError_t packed_bwd(const void* dY, const void* X, const void* R, const void* L, void* dX, void* dR, void* dL,
                        void* ws, const Shape& s, int* status, cudaStream_t st);
 
+size_t gemm_fwd_workspace(const Shape& s);
+cudaError_t gemm_fwd(const void* X, const void* R, const void* L, void* Y, void* ws, const Shape& s, int* status,
+                     cudaStream_t st);
+
 bool gemm_bwd_supported(const Shape& s);
 size_t gemm_bwd_workspace(const Shape& s);
 cudaError_t gemm_bwd(const void* dY, const void* X, const void* R, const void* L, void* dX, void* dR, void* dL,

@@ -102,6 +102,20 @@ MONARCH_API int monarch_validate(const monarch_dims* d);
 MONARCH_API int monarch_fwd(const void* X, const void* R, const void* L, const monarch_dims* d, void* Y,
                 void* stream);
 
+/* Forward with caller-provided scratch.  Same operation, arguments and results as
+ * monarch_fwd; for shapes whose permutation moves whole 64-column groups (no output
+ * transpose, in2 / nb1 a multiple of 64, e.g. nblocks = 4, 1024 -> 4096; monarch_fwd_ws_path
+ * 5) it runs two tcgen05 GEMM passes: U = blockdiag(R) X into the workspace, then the L stage
+ * reading U through 64-column gathers with L's K index reordered to match (L is reordered
+ * into the workspace too).  For other shapes it runs the monarch_fwd kernels and needs no
+ * workspace (monarch_fwd_workspace_bytes returns 0; workspace may then be NULL).
+ * workspace: >= monarch_fwd_workspace_bytes(d) bytes, 256-byte aligned, caller-owned; it must
+ * not overlap the inputs or Y. */
+MONARCH_API size_t monarch_fwd_workspace_bytes(const monarch_dims* d);
+MONARCH_API int monarch_fwd_ws_path(const monarch_dims* d);
+MONARCH_API int monarch_fwd_ws(const void* X, const void* R, const void* L, const monarch_dims* d, void* Y,
+                               void* workspace, size_t workspace_bytes, void* stream);
+
 /* Backward of Y = X * M^T for a loss with gradient dY (chain rule; the middle
  * vector is recomputed from X rather than stored):
  *   dV[j][o] = dY[idx(j,o)],  dL[j][o][q] = sum_rows dV[j][o] * Z[j][q],

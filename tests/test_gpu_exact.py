@@ -97,3 +97,18 @@ def test_backward_exact(case):
         bad = np.argwhere(g != r)
         assert bad.size == 0, "%s: %d entries differ, first at %s: %r vs %r" % (
             what, len(bad), tuple(bad[0]), g[tuple(bad[0])], r[tuple(bad[0])])
+
+
+@pytest.mark.parametrize("case", [c for c in CASES if c[0] in ("nblk4_group", "nblk2_gemm")], ids=_ids)
+def test_forward_with_workspace_exact(case):
+    """monarch_fwd_ws: the two-pass tcgen05 GEMM forward (U in the workspace, 64-column gathers)."""
+    _, shape, dtype, rows, _, _ = case
+    assert bdl.fwd_ws_path(shape, dtype) == 5
+    inp = synthetic.make_sparse_sign_inputs(dict(shape, rows=rows), seed=23)
+    _check_exact_range(inp)
+    ref = oracle.forward(shape, inp["X"], inp["R"], inp["L"])
+    Y = bdl.fwd_ws(_to_dev(inp["X"], dtype), _to_dev(inp["R"], dtype), _to_dev(inp["L"], dtype), shape)
+    assert bdl.last_device_status() == 0
+    got = _host(Y)
+    bad = np.argwhere(got != ref)
+    assert bad.size == 0, "%d entries differ, first at %s" % (len(bad), tuple(bad[0]))

@@ -220,3 +220,17 @@ def test_workspace_too_small_is_an_error():
     with pytest.raises(bdl.MonarchError) as e:
         bdl.bwd(d["dY"], d["X"], d["R"], d["L"], shape, workspace=ws)
     assert e.value.code == bdl.CODES["MONARCH_ERR_WORKSPACE"]
+
+
+@pytest.mark.parametrize("name", ["nblk4_1024x4096_bf16", "nblk4_1024x4096_bf16_b1000"])
+def test_forward_with_workspace_full_size(name):
+    """monarch_fwd_ws at the full workload size (the launch the benchmark times): every entry
+    against the oracle, normwise."""
+    w = W[name]
+    shape = synthetic.shape_of(w)
+    inp = synthetic.make_inputs(w, seed=13)
+    d = dev_inputs(inp)
+    Y = bdl.fwd_ws(d["X"], d["R"], d["L"], shape)
+    assert bdl.last_device_status() == 0
+    ref = oracle.forward(shape, inp["X"].f64, inp["R"].f64, inp["L"].f64)
+    check(to_f64(Y), ref, "bf16", name + " Y (workspace forward)")
