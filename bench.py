@@ -258,7 +258,7 @@ def device_inputs(w, seed, dev):
     return out
 
 
-def time_shape(name, dev, flush, peaks, reps=10, warmup=3, spin_cycles=400000):
+def time_shape(name, dev, flush, peaks, reps=10, warmup=3, spin_cycles=2000000):
     """Forward and backward of one workload, each pass timed alone with CUDA events on the
     launching stream after an untimed L2 flush and GPU-side spin; averages over `reps`."""
     import torch
@@ -285,16 +285,19 @@ def time_shape(name, dev, flush, peaks, reps=10, warmup=3, spin_cycles=400000):
     res = {"workload": describe(name, w), "fwd_path": bdl.fwd_ws_path(shape, w["dtype"]),
            "bwd_path": bdl.bwd_path(shape, w["dtype"])}
     for pname, fn in runs.items():
-        evs = []
+        evs, host = [], []
         for i in range(warmup + reps):
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             flush.zero_()
             torch.cuda._sleep(spin_cycles)
             e0.record(stream)
+            h0 = time.perf_counter()
             fn()
+            h1 = time.perf_counter()
             e1.record(stream)
             if i >= warmup:
                 evs.append((e0, e1))
+                host.append(h1 - h0)
         torch.cuda.synchronize()
         ms = sum(a.elapsed_time(b) for a, b in evs) / len(evs)
         t = ms / 1e3
@@ -306,6 +309,7 @@ def time_shape(name, dev, flush, peaks, reps=10, warmup=3, spin_cycles=400000):
             "bound": "hbm" if a["bytes"] / hbm >= a["flops"] / tpk else
                      ("fma" if w["dtype"] == "f32" else "tensor"),
             "launches": launches(shape, w["dtype"], pname),
+            "host_enqueue_us": 1e6 * sum(host) / len(host),
             "entry": "monarch_fwd_ws" if pname == "fwd" else "monarch_bwd",
         }
     if bdl.last_device_status() != 0:
@@ -383,9 +387,9 @@ def main():
     do_fwd = args.only in ("step", "fwd")
     do_bwd = args.only in ("step", "bwd")
 
-    # A GPU-side spin after each untimed flush lets the host enqueue the next pass
+    # A GPU-side spin (~1 ms) after each untimed flush lets the host enqueue the next pass
     # before the start event fires, so launch latency on the host is not timed.
-    spin_cycles = 400000
+    spin_cycles = 2000000
 
     def step(ev=None):
         if ev is not None:

@@ -7,6 +7,8 @@
 
 #include <atomic>
 #include <initializer_list>
+#include <mutex>
+#include <unordered_map>
 
 #include "../../include/monarch.h"
 
@@ -72,6 +74,27 @@ inline cudaError_t launch_kernel(void (*kernel)(KArgs...), dim3 grid, dim3 block
   cfg.numAttrs = pdl ? 1 : 0;
   const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, ((KArgs)args)...);
   if (e == cudaSuccess) launch_counter().fetch_add(1, std::memory_order_relaxed);
+  return e;
+}
+
+// cudaFuncSetAttribute(MaxDynamicSharedMemorySize) once per (device, kernel, size): the call
+// costs microseconds of host time, and the multi-kernel paths launch several kernels per call.
+inline cudaError_t ensure_smem_attr(const void* kernel, size_t smem) {
+  static std::mutex mu;
+  static std::unordered_map<const void*, int> done[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    auto it = done[dev].find(kernel);
+    if (it != done[dev].end() && it->second >= (int)smem) return cudaSuccess;
+  }
+  const cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e == cudaSuccess) {
+    std::lock_guard<std::mutex> lock(mu);
+    int& v = done[dev][kernel];
+    if ((int)smem > v) v = (int)smem;
+  }
   return e;
 }
 

@@ -235,8 +235,7 @@ static cudaError_t launch_fwd(const void* X, const void* R, const void* L, void*
   const int rpc = gen_rows_per_cta(s.n_in() + s.n_mid());
   if (rpc < 1) return cudaErrorNotSupported;
   const size_t smem = sizeof(float) * (size_t)rpc * (size_t)(s.n_in() + s.n_mid());
-  cudaError_t e = cudaFuncSetAttribute(gen_fwd_kernel<T>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e = ensure_smem_attr((const void*)gen_fwd_kernel<T>, (int)smem);
   if (e != cudaSuccess) return e;
   const int64_t grid = (s.rows + rpc - 1) / rpc;
   return launch_kernel(gen_fwd_kernel<T>, dim3((unsigned)grid), dim3(kGenThreads), smem, st, false,
@@ -283,8 +282,7 @@ static cudaError_t launch_bwd(const void* dY, const void* X, const void* R, cons
   if (s.rows > 0) {
     const size_t smem =
         sizeof(float) * (size_t)rpc * (size_t)(s.n_in() + s.n_out() + 2 * s.n_mid());
-    e = cudaFuncSetAttribute(gen_bwd_rows_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem);
+    e = ensure_smem_attr((const void*)gen_bwd_rows_kernel<T>, (int)smem);
     if (e != cudaSuccess) return e;
     const int64_t grid = (s.rows + rpc - 1) / rpc;
     if ((e = launch_kernel(gen_bwd_rows_kernel<T>, dim3((unsigned)grid), dim3(kGenThreads), smem, st, false,

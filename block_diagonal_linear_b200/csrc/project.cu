@@ -149,13 +149,12 @@ cudaError_t project(const float* M, void* R, void* L, const Shape& s, int dtype,
   const size_t smem = sizeof(float) * ((size_t)s.out2 * s.in1 + s.in1 + s.out2 + 64);
   const unsigned grid = (unsigned)((int64_t)s.nb1 * s.nb2);
   if (dtype == MONARCH_BF16) {
-    cudaError_t e = cudaFuncSetAttribute(project_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
+    cudaError_t e = ensure_smem_attr((const void*)project_kernel<__nv_bfloat16>, (int)smem);
     if (e != cudaSuccess) return e;
     return launch_kernel(project_kernel<__nv_bfloat16>, dim3(grid), dim3(kProjThreads), smem, st, false, M,
                          (__nv_bfloat16*)R, (__nv_bfloat16*)L, s);
   }
-  cudaError_t e = cudaFuncSetAttribute(project_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e = ensure_smem_attr((const void*)project_kernel<float>, (int)smem);
   if (e != cudaSuccess) return e;
   return launch_kernel(project_kernel<float>, dim3(grid), dim3(kProjThreads), smem, st, false, M, (float*)R,
                        (float*)L, s);

@@ -425,8 +425,7 @@ static cudaError_t launch_tc_fwd(const void* X, const void* R, const void* L, vo
     return cudaErrorInvalidValue;
   static bool attr_set = false;
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(tc_fwd_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         C::SMEM_BYTES);
+    cudaError_t e = ensure_smem_attr((const void*)tc_fwd_kernel<C>, C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }

@@ -289,8 +289,7 @@ static cudaError_t launch_gemm_cfg(const CUtensorMap& mA, const CUtensorMap& mB,
                                    const GemmJob& job, float* partial, int* status, cudaStream_t st,
                                    bool pdl) {
   using C = GemmCfg<BN, KIND>;
-  cudaError_t e = cudaFuncSetAttribute(tc_gemm_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       C::SMEM_BYTES);
+  cudaError_t e = ensure_smem_attr((const void*)tc_gemm_kernel<C>, C::SMEM_BYTES);
   if (e != cudaSuccess) return e;
   int64_t grid = num_sms();
   if (grid > job.units) grid = job.units;

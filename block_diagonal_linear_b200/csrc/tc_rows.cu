@@ -446,8 +446,7 @@ static cudaError_t launch_rows(const void* X, const void* W1, const void* W2, vo
   if (C::MODE != 0 &&
       !make_map_2d(&mZ, Zout, C::N_MID, (uint64_t)rows, 64, C::BM, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
-  cudaError_t e = cudaFuncSetAttribute(tc_rows_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       C::SMEM_BYTES);
+  cudaError_t e = ensure_smem_attr((const void*)tc_rows_kernel<C>, C::SMEM_BYTES);
   if (e != cudaSuccess) return e;
   const int64_t nunits = (rows + C::BM - 1) / C::BM;
   int64_t grid = num_sms();

@@ -272,8 +272,7 @@ static cudaError_t launch_bdgemm(const void* X, const void* W, void* Y, int nb, 
       !make_map_2d(&mW, W, C::KB, (uint64_t)nb * C::NB, 64, C::NB, CU_TENSOR_MAP_SWIZZLE_128B) ||
       !make_map_2d(&mY, Y, (uint64_t)nb * C::NB, (uint64_t)rows, 64, C::BM, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
-  cudaError_t e = cudaFuncSetAttribute(tc_bdgemm_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       C::SMEM_BYTES);
+  cudaError_t e = ensure_smem_attr((const void*)tc_bdgemm_kernel<C>, C::SMEM_BYTES);
   if (e != cudaSuccess) return e;
   const int64_t nunits = (rows + C::BM - 1) / C::BM * nb;
   const int64_t grid = nunits < num_sms() ? nunits : num_sms();
@@ -290,8 +289,7 @@ static cudaError_t launch_permute(const void* src, void* dst, int64_t rows, int 
   if (row_smem > cap) return cudaErrorInvalidValue;
   const int nwarps = (int)std::min<size_t>(kPermWarps, cap / row_smem);
   const size_t smem = (size_t)nwarps * row_smem;
-  cudaError_t e = cudaFuncSetAttribute(permute_rows_kernel<ACC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)smem);
+  cudaError_t e = ensure_smem_attr((const void*)permute_rows_kernel<ACC>, (int)smem);
   if (e != cudaSuccess) return e;
   return launch_kernel(permute_rows_kernel<ACC>, dim3(2 * 148), dim3(nwarps * 32), smem, st, true,
                        (const __nv_bfloat16*)src, (__nv_bfloat16*)dst, rows, A, B);

@@ -375,8 +375,7 @@ static cudaError_t launch_wide(const void* X, const void* R, const void* L, void
   if (!make_map_2d(&mX, X, C::N_IN, (uint64_t)rows, 64, (uint32_t)bm, CU_TENSOR_MAP_SWIZZLE_128B) ||
       !make_map_2d(&mY, Y, C::N_OUT, (uint64_t)rows, 64, (uint32_t)bm, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
-  cudaError_t e = cudaFuncSetAttribute(tc_wide_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       C::SMEM_BYTES);
+  cudaError_t e = ensure_smem_attr((const void*)tc_wide_kernel<C>, C::SMEM_BYTES);
   if (e != cudaSuccess) return e;
   const int64_t nunits = (rows + bm - 1) / bm;
   const int64_t grid = nunits < nsm ? nunits : nsm;
