@@ -60,12 +60,12 @@ __global__ void gemm_bwd_prep_kernel(const __nv_bfloat16* __restrict__ R, const 
 
 // ---------------------------------------------------------------- weight gradient
 // Split of the rows for the weight-gradient GEMMs: chunks of a multiple of 64 rows, enough of
-// them that both launches together give about two units per SM, but at least 512 rows each
+// them that both launches together give about two units per SM, but at least 256 rows each
 // (every chunk costs one fp32 copy of the parameters in partials), and none of them empty
 // (an empty chunk would leave its partials unwritten).
 WgradSplit wgrad_split(int64_t rows, int64_t units_per_split) {
   int64_t n = (2 * 148 + units_per_split - 1) / (units_per_split > 0 ? units_per_split : 1);
-  const int64_t maxs = rows / 512;
+  const int64_t maxs = rows / 256;
   if (n > maxs) n = maxs;
   if (n < 1) n = 1;
   WgradSplit w;
@@ -81,10 +81,10 @@ WgradSplit wgrad_split(int64_t rows, int64_t units_per_split) {
 // A1 is block-contiguous with blocks of blk_a columns; A2's block b occupies the logical
 // columns [b*blk_b, (b+1)*blk_b).  With b_grp = 0, A2 is block-contiguous too; otherwise its
 // 64-column groups are gathered: group g of block b starts at b*b_base + (g / b_grp)*b_gs +
-// (g % b_grp)*64, and the in-block logical column n maps back to (n % pm_a)*pm_b + n / pm_a.
+// (g % b_grp)*64.  Partials are in logical column order.
 cudaError_t wgrad_tc(const void* A1, int64_t a_cols, int64_t blk_a, const void* A2, int64_t b_cols, int64_t blk_b,
-                     int64_t nblocks, int b_base, int b_grp, int b_gs, int64_t pm_a, int64_t pm_b, int64_t rows,
-                     WgradSplit sp, float* partial, int64_t p_stride, int64_t p_off, int* status, cudaStream_t st) {
+                     int64_t nblocks, int b_base, int b_grp, int b_gs, int64_t rows, WgradSplit sp, float* partial,
+                     int64_t p_stride, int64_t p_off, int* status, cudaStream_t st) {
   GemmJob j = {};
   // M side: a group of 128 columns of A1 holding bpg whole blocks, or one block per group in
   // 128-row tiles (rows of a tile beyond the block belong to the next block and are dropped)
@@ -94,6 +94,7 @@ cudaError_t wgrad_tc(const void* A1, int64_t a_cols, int64_t blk_a, const void* 
   const int64_t nw = bpg * blk_b;  // B columns a group needs
   const int BN = nw >= 256 ? 256 : (nw > 64 ? 128 : 64);
   if ((bpg * blk_a) % 8 || (bpg * b_base) % 8 || nw % 8) return cudaErrorInvalidValue;  // 16-byte TMA x
+  if (blk_a % 4 || blk_b % 4 || p_stride % 4 || p_off % 4) return cudaErrorInvalidValue;  // float4 partials
   j.nb = (int)(nblocks / bpg);
   j.ntiles = (int)((nw + BN - 1) / BN);
   j.nsplit = sp.nsplit;
@@ -111,11 +112,32 @@ cudaError_t wgrad_tc(const void* A1, int64_t a_cols, int64_t blk_a, const void* 
   }
   j.blk_a = blk_a;
   j.blk_b = blk_b;
-  j.pm_a = pm_a;
-  j.pm_b = pm_b;
   j.p_stride = p_stride;
   j.p_off = p_off;
   return gemm_wgrad(A1, a_cols, A2, b_cols, rows, BN, j, partial, status, st, true);
+}
+
+// dR = sum of the first nR partials; dL[j][o][q] = sum of the partials at in-block column
+// kappa(q) = (q % nb1)*G + q / nb1 (the order the gathered weight gradient wrote them in).
+__global__ void reduce_partials_gathered_kernel(const float* __restrict__ partial, __nv_bfloat16* __restrict__ dR,
+                                                __nv_bfloat16* __restrict__ dL, int64_t nR, int64_t nP, int nsplit,
+                                                int in2, int nb1, int G) {
+  ptx::griddep_wait();
+  ptx::griddep_launch_dependents();
+  const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= nP) return;
+  int64_t src = e;
+  if (e >= nR) {
+    const int64_t f = e - nR;
+    const int q = (int)(f % in2);
+    src = nR + (f - q) + (int64_t)(q % nb1) * G + q / nb1;
+  }
+  float acc = 0.f;
+  for (int sp = 0; sp < nsplit; ++sp) acc += partial[(int64_t)sp * nP + src];
+  if (e < nR)
+    dR[e] = __float2bfloat16_rn(acc);
+  else
+    dL[e - nR] = __float2bfloat16_rn(acc);
 }
 
 // ---------------------------------------------------------------- host
@@ -196,17 +218,18 @@ cudaError_t gemm_bwd(const void* dY, const void* X, const void* R, const void* L
                      true)) != cudaSuccess)
       return e;
     // 5. weight gradients
-    if ((e = wgrad_tc(dU, s.n_mid(), s.out1, X, s.n_in(), s.in1, s.nb1, 0, 0, 0, s.in1, 1, s.rows,
+    if ((e = wgrad_tc(dU, s.n_mid(), s.out1, X, s.n_in(), s.in1, s.nb1, 0, 0, 0, s.rows,
                       w.sp, part, nP, 0, status, st)) != cudaSuccess)
       return e;
-    if ((e = wgrad_tc(dY, s.n_out(), s.out2, U, s.n_mid(), s.in2, s.nb2, G, G / 64, s.out1, G, s.nb1, s.rows,
+    if ((e = wgrad_tc(dY, s.n_out(), s.out2, U, s.n_mid(), s.in2, s.nb2, G, G / 64, s.out1, s.rows,
                       w.sp, part, nP, nR, status, st)) != cudaSuccess)
       return e;
   } else {
     if ((e = cudaMemsetAsync(part, 0, sizeof(float) * (size_t)w.sp.nsplit * (size_t)nP, st)) != cudaSuccess) return e;
   }
-  return launch_kernel(reduce_partials_kernel, dim3((unsigned)((nP + 255) / 256)), dim3(256), 0, st, true,
-                       (const float*)part, (__nv_bfloat16*)dR, (__nv_bfloat16*)dL, nR, nP, w.sp.nsplit);
+  return launch_kernel(reduce_partials_gathered_kernel, dim3((unsigned)((nP + 255) / 256)), dim3(256), 0, st, true,
+                       (const float*)part, (__nv_bfloat16*)dR, (__nv_bfloat16*)dL, nR, nP, w.sp.nsplit, s.in2, s.nb1,
+                       G);
 }
 
 // ================================================================ two-pass forward
@@ -422,10 +445,10 @@ cudaError_t packed_bwd(const void* dY, const void* X, const void* R, const void*
     if ((e = packed_stage(dU, s.rows, Wx, dX, s.nb1, s.out1, s.in1, pk.gx, status, st)) != cudaSuccess) return e;
     if ((e = packed_stage(X, s.rows, Wu, U, s.nb1, s.in1, s.out1, pk.gx, status, st)) != cudaSuccess) return e;
     if ((e = permute_rows(U, Z, s.rows, s.nb1, s.out1, st)) != cudaSuccess) return e;
-    if ((e = wgrad_tc(dU, s.n_mid(), s.out1, X, s.n_in(), s.in1, s.nb1, 0, 0, 0, s.in1, 1, s.rows, w.sp, part, nP, 0,
+    if ((e = wgrad_tc(dU, s.n_mid(), s.out1, X, s.n_in(), s.in1, s.nb1, 0, 0, 0, s.rows, w.sp, part, nP, 0,
                       status, st)) != cudaSuccess)
       return e;
-    if ((e = wgrad_tc(dV, s.n_out(), s.out2, Z, s.n_mid(), s.in2, s.nb2, 0, 0, 0, s.in2, 1, s.rows, w.sp, part, nP,
+    if ((e = wgrad_tc(dV, s.n_out(), s.out2, Z, s.n_mid(), s.in2, s.nb2, 0, 0, 0, s.rows, w.sp, part, nP,
                       nR, status, st)) != cudaSuccess)
       return e;
   } else if ((e = cudaMemsetAsync(part, 0, sizeof(float) * (size_t)w.sp.nsplit * (size_t)nP, st)) != cudaSuccess) {

@@ -287,9 +287,9 @@ int monarch_dyad_bwd(const void* dY, const void* X, const void* W1, const void* 
         (e = permute_rows_add(PX, dX, s.rows, s.ib, s.nb, st)) != cudaSuccess ||
         (e = permute_rows(X, PX, s.rows, s.nb, s.ib, st)) != cudaSuccess)
       return MONARCH_ERR_CUDA;
-    if ((e = wgrad_tc(dY, n_out, s.ob, X, n_in, s.ib, s.nb, 0, 0, 0, s.ib, 1, s.rows, w.sp, part, 2 * nW, 0, status,
+    if ((e = wgrad_tc(dY, n_out, s.ob, X, n_in, s.ib, s.nb, 0, 0, 0, s.rows, w.sp, part, 2 * nW, 0, status,
                       st)) != cudaSuccess ||
-        (e = wgrad_tc(DV, n_out, s.ob, PX, n_in, s.ib, s.nb, 0, 0, 0, s.ib, 1, s.rows, w.sp, part, 2 * nW, nW, status,
+        (e = wgrad_tc(DV, n_out, s.ob, PX, n_in, s.ib, s.nb, 0, 0, 0, s.rows, w.sp, part, 2 * nW, nW, status,
                       st)) != cudaSuccess)
       return MONARCH_ERR_CUDA;
   } else if ((e = cudaMemsetAsync(part, 0, sizeof(float) * (size_t)w.sp.nsplit * 2 * nW, st)) != cudaSuccess) {

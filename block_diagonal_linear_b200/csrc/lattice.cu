@@ -469,7 +469,7 @@ int monarch_lattice_bwd(const void* dY, const void* X, const void* const* W, con
       if ((e = permute_rows(G, gb, s.rows * P, s.m[t], (int)B, st)) != cudaSuccess) return MONARCH_ERR_CUDA;
       Gt = gb;
     }
-    if ((e = wgrad_tc(Gt, lines * s.m[t], s.m[t], kept[t], lines * s.n[t], s.n[t], lines, 0, 0, 0, s.n[t], 1, s.rows,
+    if ((e = wgrad_tc(Gt, lines * s.m[t], s.m[t], kept[t], lines * s.n[t], s.n[t], lines, 0, 0, 0, s.rows,
                       w.sp, part, w.nparams, poff, status, st)) != cudaSuccess)
       return MONARCH_ERR_CUDA;
     const int g2 = pack_factor((int)lines, s.m[t], s.n[t]);

@@ -244,29 +244,34 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
         }
       } else {
-        // diagonal blocks of D as fp32 partials: row m belongs to block bm = ma / blk_a
-        const int64_t ma = (int64_t)c.b * job.a_b + (int64_t)c.mt * C::BM + r;
-        const int64_t nb0 = (int64_t)c.b * job.b_lb + (int64_t)c.nt * C::BN;
-        const bool row_ok = ma < job.a_cols;
-        const int64_t blk = ma / job.blk_a;
-        // columns of this warp's rows: [first row's block start, last row's block end)
-        const int64_t ma0 = (int64_t)c.b * job.a_b + (int64_t)c.mt * C::BM + quad * 32;
-        int64_t lo = (ma0 / job.blk_a) * job.blk_b - nb0;
-        int64_t hi = ((ma0 + 31) / job.blk_a + 1) * job.blk_b - nb0;
-        lo = lo < 0 ? 0 : (lo / 16) * 16;
-        hi = hi > C::BN ? C::BN : hi;
-        float* prow = partial + (int64_t)c.split * job.p_stride + job.p_off +
-                      blk * job.blk_a * job.blk_b + (ma % job.blk_a) * job.blk_b;
-        for (int c0 = (int)lo; c0 < (int)hi; c0 += 16) {
+        // diagonal blocks of D as fp32 partials: row m belongs to block blk = m_g / blk_a, and
+        // its values go to the columns of that block, in logical column order (any column
+        // permutation is applied when the partials are summed).  32-bit index math, one
+        // division per unit, float4 stores.
+        const int bla = (int)job.blk_a, blb = (int)job.blk_b;
+        const int ma = c.b * job.a_b + c.mt * C::BM + r;
+        const int nb0 = c.b * job.b_lb + c.nt * C::BN;
+        const int blk = ma / bla;
+        const bool row_ok = ma < (int)job.a_cols;
+        const int t_lo = max(0, blk * blb - nb0);
+        const int t_hi = min(C::BN, min((blk + 1) * blb, (int)job.b_cols) - nb0);
+        // the warp's column range: from its first row's block to its last row's block
+        const int ma0 = c.b * job.a_b + c.mt * C::BM + quad * 32;
+        const int w_lo = max(0, (ma0 / bla) * blb - nb0) & ~15;
+        const int w_hi = min(C::BN, ((ma0 + 31) / bla + 1) * blb - nb0);
+        float* prow = partial + (int64_t)c.split * job.p_stride + job.p_off + (int64_t)blk * bla * blb +
+                      (int64_t)(ma - blk * bla) * blb + (nb0 - blk * blb);  // + tile column
+        for (int c0 = w_lo; c0 < w_hi; c0 += 16) {
           uint32_t t16[16];
           ptx::tmem_ld16(tb + c0, t16);
           ptx::tmem_wait_ld();
+          if (row_ok) {
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const int64_t ng = nb0 + c0 + e;
-            if (row_ok && ng < job.b_cols && ng / job.blk_b == blk) {
-              const int64_t nl = ng % job.blk_b;
-              prow[(nl % job.pm_a) * job.pm_b + nl / job.pm_a] = __uint_as_float(t16[e]);
+            for (int e = 0; e < 16; e += 4) {
+              const int cc = c0 + e;
+              if (cc >= t_lo && cc < t_hi)
+                *(float4*)(prow + cc) = make_float4(__uint_as_float(t16[e]), __uint_as_float(t16[e + 1]),
+                                                    __uint_as_float(t16[e + 2]), __uint_as_float(t16[e + 3]));
             }
           }
         }

@@ -16,10 +16,10 @@ namespace monarch {
 // A columns b*a_b + mt*128 (contiguous), B group = nt*(BN/64) + h (b_b, b_grp, b_gs); rows
 // [split*split_rows, +split_rows).  D[m][n] is kept when column m of act1 and the B column
 // n lie in the same block: m_g = b*a_b + mt*128 + m, n_g = b*b_lb + nt*BN + n (the logical
-// position, before gathering); block = m_g / blk_a must equal n_g / blk_b; the in-block column
-// n_l = n_g % blk_b is first mapped to q = (n_l % pm_a)*pm_b + n_l / pm_a (identity with
-// pm_a = blk_b, pm_b = 1), and the value goes to
-// partial[split*p_stride + p_off + block*blk_a*blk_b + (m_g % blk_a)*blk_b + q].
+// position, before gathering); block = m_g / blk_a must equal n_g / blk_b; the value goes to
+// partial[split*p_stride + p_off + block*blk_a*blk_b + (m_g % blk_a)*blk_b + n_g % blk_b]
+// (logical column order: a column permutation of gathered operands is applied by the
+// partial sum).  blk_a, blk_b, p_off, p_stride are multiples of 4 (float4 stores).
 struct GemmJob {
   int kind;
   int nb, mtiles, ntiles, nsplit;
@@ -31,7 +31,6 @@ struct GemmJob {
   int64_t rows, split_rows;   // kind 1
   int64_t a_cols, b_cols;     // kind 1: widths of act1, act2
   int64_t blk_a, blk_b;       // kind 1: block widths (M side, N side, before gathering)
-  int64_t pm_a, pm_b;         // kind 1: in-block column permutation
   int64_t p_stride, p_off;    // kind 1: partial layout
   int64_t units;
 };
@@ -46,7 +45,7 @@ cudaError_t gemm_bd(const void* A, int64_t rows, int64_t a_cols, const void* W, 
                     void* Y, int64_t y_cols, int BN, GemmJob job, int* status, cudaStream_t st, bool pdl);
 // Kind 1: act1 (rows x a_cols), act2 (rows x b_cols); BN in {64, 128, 256}.
 // job: nb, mtiles, ntiles, nsplit, split_rows (multiple of 64), a_b, b_b, b_grp, b_gs, b_lb, blk_a, blk_b,
-// pm_a, pm_b, p_stride, p_off.
+// p_stride, p_off.
 cudaError_t gemm_wgrad(const void* A1, int64_t a_cols, const void* A2, int64_t b_cols, int64_t rows, int BN,
                        GemmJob job, float* partial, int* status, cudaStream_t st, bool pdl);
 
@@ -57,8 +56,8 @@ struct WgradSplit {
 };
 WgradSplit wgrad_split(int64_t rows, int64_t units_per_split);
 cudaError_t wgrad_tc(const void* A1, int64_t a_cols, int64_t blk_a, const void* A2, int64_t b_cols, int64_t blk_b,
-                     int64_t nblocks, int b_base, int b_grp, int b_gs, int64_t pm_a, int64_t pm_b, int64_t rows,
-                     WgradSplit sp, float* partial, int64_t p_stride, int64_t p_off, int* status, cudaStream_t st);
+                     int64_t nblocks, int b_base, int b_grp, int b_gs, int64_t rows, WgradSplit sp, float* partial,
+                     int64_t p_stride, int64_t p_off, int* status, cudaStream_t st);
 
 // Smallest g <= 8 dividing nblocks with g*kw and g*nw multiples of 64 (0 if none).
 int pack_factor(int nblocks, int kw, int nw);
