@@ -23,26 +23,6 @@ cudaError_t tc_rows_dual(const void* dV, const void* Lt, const void* Rt, void* d
                          const Shape& s, int* status, cudaStream_t st);
 
 // ------------------------------------------------------------------ small kernels
-__global__ void transpose_factors_kernel(const __nv_bfloat16* __restrict__ R,
-                                         const __nv_bfloat16* __restrict__ L,
-                                         __nv_bfloat16* __restrict__ Rt,
-                                         __nv_bfloat16* __restrict__ Lt, Shape s) {
-  ptx::griddep_wait();  // Rt, Lt may still be read by the previous backward's kernels
-  ptx::griddep_launch_dependents();
-  const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  const int64_t nR = s.n_R(), nL = s.n_L();
-  if (e < nR) {  // Rt[k][i][p] = R[k][p][i]
-    const int64_t k = e / ((int64_t)s.in1 * s.out1), rem = e % ((int64_t)s.in1 * s.out1);
-    const int i = (int)(rem / s.out1), p = (int)(rem % s.out1);
-    Rt[e] = R[(k * s.out1 + p) * s.in1 + i];
-  } else if (e < nR + nL) {  // Lt[j][q][o] = L[j][o][q]
-    const int64_t f = e - nR;
-    const int64_t j = f / ((int64_t)s.in2 * s.out2), rem = f % ((int64_t)s.in2 * s.out2);
-    const int q = (int)(rem / s.out2), o = (int)(rem % s.out2);
-    Lt[f] = L[(j * s.out2 + o) * s.in2 + q];
-  }
-}
-
 // dV[r][j*out2 + o] = dY[r][o*nb2 + j]: per row an (out2 x nb2) -> (nb2 x out2)
 // transpose.  One warp per row: the row is read with 16-byte coalesced loads, staged in
 // shared memory with an odd word pitch (nb2 + 2 elements, so the column reads of the
@@ -152,9 +132,7 @@ cudaError_t fast_bwd(const void* dY, const void* X, const void* R, const void* L
   // All six launches use programmatic dependent launch: each kernel waits for the previous
   // grid of the stream (griddep_wait) before touching its data, so the next launch and its
   // prologue overlap the tail of the current one.
-  if ((e = launch_kernel(transpose_factors_kernel, dim3((unsigned)((nP + 255) / 256)), dim3(256), 0, st,
-                         true, (const __nv_bfloat16*)R, (const __nv_bfloat16*)L, Rt, Lt, s)) != cudaSuccess)
-    return e;
+  if ((e = factor_transposes(R, Rt, L, Lt, s, 0, st)) != cudaSuccess) return e;
   const WgradSplit sp = wg_split(s);
   const bool split = is_split_square(s);
   if (split && !s.out_transpose) dV = (__nv_bfloat16*)dY;  // dV[j][o] = dy[j*out2 + o]: no copy

@@ -34,27 +34,142 @@ bool gemm_bwd_supported(const Shape& s) {
   const int G = s.in2 / s.nb1;
   if (G % 64) return false;
   if (s.nb1 * s.out1 != s.nb2 * s.in2) return false;
+  if (s.in2 > 65536) return false;  // the forward's column permutation stages one row of L per warp
   return s.n_in() <= (1 << 20) && s.n_out() <= (1 << 20);
 }
 
 // ---------------------------------------------------------------- prep
-__global__ void gemm_bwd_prep_kernel(const __nv_bfloat16* __restrict__ R, const __nv_bfloat16* __restrict__ L,
-                                     __nv_bfloat16* __restrict__ Rt, __nv_bfloat16* __restrict__ Ltp, Shape s) {
+// Block transposes of the factors, with an optional column map:
+//   dst[b][c][r] = src[b][r][cmap(c)],  r < A, c < B,  cmap(c) = (c % G)*nbk + c / G  (G > 0), else c.
+// One CTA per (block b, 32 source rows): the rows are read with coalesced loads into shared
+// memory (row pitch B + 2 elements, so the column reads of the write phase spread over the
+// banks), then every destination row segment of 32 values (64 bytes) is written by four
+// threads with 16-byte stores.  Needs A % 8 == 0 and B % 8 == 0.
+struct FactorT {
+  const __nv_bfloat16* src;
+  __nv_bfloat16* dst;
+  int nblk, A, B, G, nbk;
+  int ctas;  // nblk * ceil(A / 32)
+};
+
+__device__ __forceinline__ void factor_tile(const FactorT& f, int cta, uint16_t* sm) {
+  const int tiles = (f.A + 31) / 32;
+  const int b = cta / tiles, r0 = (cta % tiles) * 32;
+  const int nr = min(32, f.A - r0);
+  const int pitch = f.B + 2;
+  const uint16_t* src = (const uint16_t*)f.src + ((int64_t)b * f.A + r0) * f.B;
+  const int cpr = f.B / 8;
+  for (int c = threadIdx.x; c < nr * cpr; c += blockDim.x) {
+    const int rr = c / cpr, cc = c % cpr;
+    const uint4 v = *(const uint4*)(src + (int64_t)rr * f.B + cc * 8);
+    uint32_t* d = (uint32_t*)(sm + rr * pitch + cc * 8);  // 4-byte aligned: pitch is even
+    d[0] = v.x; d[1] = v.y; d[2] = v.z; d[3] = v.w;
+  }
+  __syncthreads();
+  uint16_t* dst = (uint16_t*)f.dst + (int64_t)b * f.B * f.A + r0;
+  for (int w = threadIdx.x; w < f.B * 4; w += blockDim.x) {
+    const int c = w >> 2, t = w & 3;
+    if (8 * t >= nr) continue;
+    const int q = f.G > 0 ? (c % f.G) * f.nbk + c / f.G : c;
+    uint32_t v[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+      v[e] = (uint32_t)sm[(8 * t + 2 * e) * pitch + q] | ((uint32_t)sm[(8 * t + 2 * e + 1) * pitch + q] << 16);
+    *(uint4*)(dst + (int64_t)c * f.A + 8 * t) = make_uint4(v[0], v[1], v[2], v[3]);
+  }
+}
+
+__global__ void __launch_bounds__(256) factor_transpose_kernel(FactorT f0, FactorT f1) {
+  extern __shared__ __align__(16) uint16_t fsm[];
+  ptx::griddep_wait();  // the outputs may still be read by the previous kernels of the stream
+  ptx::griddep_launch_dependents();
+  const int cta = (int)blockIdx.x;
+  if (cta < f0.ctas)
+    factor_tile(f0, cta, fsm);
+  else
+    factor_tile(f1, cta - f0.ctas, fsm);
+}
+
+static FactorT factor_job(const void* src, void* dst, int nblk, int A, int B, int G, int nbk) {
+  FactorT f;
+  f.src = (const __nv_bfloat16*)src;
+  f.dst = (__nv_bfloat16*)dst;
+  f.nblk = nblk; f.A = A; f.B = B; f.G = G; f.nbk = nbk;
+  f.ctas = nblk * ((A + 31) / 32);
+  return f;
+}
+
+bool factor_transpose_ok(int A, int B) { return A % 8 == 0 && B % 8 == 0 && B <= 2048; }
+
+__global__ void factor_transpose_flat_kernel(const __nv_bfloat16* __restrict__ R, const __nv_bfloat16* __restrict__ L,
+                                             __nv_bfloat16* __restrict__ Rt, __nv_bfloat16* __restrict__ Lt, Shape s,
+                                             int G);
+
+// Rt[k][i][p] = R[k][p][i] and Lt[j][c][o] = L[j][o][cmap(c)] in one launch (G as above).
+cudaError_t factor_transposes(const void* R, void* Rt, const void* L, void* Lt, const Shape& s, int G,
+                              cudaStream_t st) {
+  if (!factor_transpose_ok(s.out1, s.in1) || !factor_transpose_ok(s.out2, s.in2)) {
+    const int64_t n = s.n_R() + s.n_L();
+    return launch_kernel(factor_transpose_flat_kernel, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, st, true,
+                         (const __nv_bfloat16*)R, (const __nv_bfloat16*)L, (__nv_bfloat16*)Rt, (__nv_bfloat16*)Lt, s,
+                         G);
+  }
+  const FactorT f0 = factor_job(R, Rt, s.nb1, s.out1, s.in1, 0, 0);
+  const FactorT f1 = factor_job(L, Lt, s.nb2, s.out2, s.in2, G, s.nb1);
+  const int bmax = s.in1 > s.in2 ? s.in1 : s.in2;
+  const size_t smem = (size_t)32 * (size_t)(bmax + 2) * 2;
+  cudaError_t e = ensure_smem_attr((const void*)factor_transpose_kernel, (int)smem);
+  if (e != cudaSuccess) return e;
+  return launch_kernel(factor_transpose_kernel, dim3((unsigned)(f0.ctas + f1.ctas)), dim3(256), smem, st, true, f0,
+                       f1);
+}
+
+// Elementwise form of the same transposes, for factor widths beyond the staged tile.
+__global__ void factor_transpose_flat_kernel(const __nv_bfloat16* __restrict__ R, const __nv_bfloat16* __restrict__ L,
+                                             __nv_bfloat16* __restrict__ Rt, __nv_bfloat16* __restrict__ Lt, Shape s,
+                                             int G) {
   ptx::griddep_wait();
   ptx::griddep_launch_dependents();
   const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   const int64_t nR = s.n_R(), nL = s.n_L();
-  if (e < nR) {  // Rt[k][i][p] = R[k][p][i]
+  if (e < nR) {
     const int64_t k = e / ((int64_t)s.in1 * s.out1), rem = e % ((int64_t)s.in1 * s.out1);
     const int i = (int)(rem / s.out1), p = (int)(rem % s.out1);
     Rt[e] = R[(k * s.out1 + p) * s.in1 + i];
-  } else if (e < nR + nL) {  // Ltp[j][kappa][o] = L[j][o][q],  kappa = k*G + p',  q = p'*nb1 + k
+  } else if (e < nR + nL) {
     const int64_t f = e - nR;
-    const int G = s.in2 / s.nb1;
     const int64_t j = f / ((int64_t)s.in2 * s.out2), rem = f % ((int64_t)s.in2 * s.out2);
-    const int kappa = (int)(rem / s.out2), o = (int)(rem % s.out2);
-    const int q = (kappa % G) * s.nb1 + kappa / G;
-    Ltp[f] = L[(j * s.out2 + o) * s.in2 + q];
+    const int c = (int)(rem / s.out2), o = (int)(rem % s.out2);
+    const int q = G > 0 ? (c % G) * s.nb1 + c / G : c;
+    Lt[f] = L[(j * s.out2 + o) * s.in2 + q];
+  }
+}
+
+// Lp[row][kappa] = L[row][q(kappa)] for every row of L (one row per warp, staged in shared memory).
+constexpr int kPermColWarps = 8;
+__global__ void __launch_bounds__(kPermColWarps * 32)
+    permute_cols_kernel(const __nv_bfloat16* __restrict__ L, __nv_bfloat16* __restrict__ Lp, int64_t nrows,
+                        int ncols, int G, int nbk) {
+  extern __shared__ __align__(16) uint16_t pcs[];
+  ptx::griddep_wait();
+  ptx::griddep_launch_dependents();
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32, nw = blockDim.x / 32;
+  uint16_t* buf = pcs + warp * ncols;
+  for (int64_t r = (int64_t)blockIdx.x * nw + warp; r < nrows; r += (int64_t)gridDim.x * nw) {
+    const uint16_t* src = (const uint16_t*)L + r * ncols;
+    for (int c = lane; c < ncols / 8; c += 32) *(uint4*)(buf + c * 8) = *(const uint4*)(src + c * 8);
+    __syncwarp();
+    uint16_t* dst = (uint16_t*)Lp + r * ncols;
+    for (int c = lane; c < ncols / 8; c += 32) {
+      uint32_t v[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int k0 = c * 8 + 2 * e, k1 = k0 + 1;
+        v[e] = (uint32_t)buf[(k0 % G) * nbk + k0 / G] | ((uint32_t)buf[(k1 % G) * nbk + k1 / G] << 16);
+      }
+      *(uint4*)(dst + c * 8) = make_uint4(v[0], v[1], v[2], v[3]);
+    }
+    __syncwarp();
   }
 }
 
@@ -183,9 +298,7 @@ cudaError_t gemm_bwd(const void* dY, const void* X, const void* R, const void* L
   const int64_t nR = s.n_R(), nL = s.n_L(), nP = nR + nL;
   const int G = s.in2 / s.nb1;
   cudaError_t e;
-  if ((e = launch_kernel(gemm_bwd_prep_kernel, dim3((unsigned)((nP + 255) / 256)), dim3(256), 0, st, true,
-                         (const __nv_bfloat16*)R, (const __nv_bfloat16*)L, Rt, Ltp, s)) != cudaSuccess)
-    return e;
+  if ((e = factor_transposes(R, Rt, L, Ltp, s, G, st)) != cudaSuccess) return e;
   if (s.rows > 0) {
     // 2. U = blockdiag(R) X
     GemmJob j = {};
@@ -238,18 +351,6 @@ cudaError_t gemm_bwd(const void* dY, const void* X, const void* R, const void* L
 //   2. U  = blockdiag(R) X                    (GEMM, block-contiguous u[k][p])
 //   3. Y  = blockdiag(Lp) gathered(U)          (GEMM; block j's K stage kb reads the 64 columns
 //                                             of U at k*out1 + j*G + 64*(kb % (G/64)))
-__global__ void gemm_fwd_prep_kernel(const __nv_bfloat16* __restrict__ L, __nv_bfloat16* __restrict__ Lp, Shape s) {
-  ptx::griddep_wait();
-  ptx::griddep_launch_dependents();
-  const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (e >= s.n_L()) return;
-  const int G = s.in2 / s.nb1;
-  const int kappa = (int)(e % s.in2);
-  const int64_t jo = e / s.in2;  // j*out2 + o
-  const int q = (kappa % G) * s.nb1 + kappa / G;
-  Lp[e] = L[jo * s.in2 + q];
-}
-
 size_t gemm_fwd_workspace(const Shape& s) {
   return al256((size_t)s.n_L() * 2) + al256((size_t)s.rows * (size_t)s.n_mid() * 2);
 }
@@ -261,8 +362,15 @@ cudaError_t gemm_fwd(const void* X, const void* R, const void* L, void* Y, void*
   __nv_bfloat16* U = (__nv_bfloat16*)((char*)ws + al256((size_t)s.n_L() * 2));
   const int G = s.in2 / s.nb1;
   cudaError_t e;
-  if ((e = launch_kernel(gemm_fwd_prep_kernel, dim3((unsigned)((s.n_L() + 255) / 256)), dim3(256), 0, st, false,
-                         (const __nv_bfloat16*)L, Lp, s)) != cudaSuccess)
+  // one staged row per warp: up to 8 warps, as many as 200 KB of shared memory holds
+  const int64_t lrows = (int64_t)s.nb2 * s.out2;
+  int nw = (int)((200 * 1024) / ((size_t)s.in2 * 2));
+  if (nw > kPermColWarps) nw = kPermColWarps;
+  if (nw < 1) return cudaErrorNotSupported;
+  const size_t psm = (size_t)nw * (size_t)s.in2 * 2;
+  if ((e = ensure_smem_attr((const void*)permute_cols_kernel, (int)psm)) != cudaSuccess) return e;
+  if ((e = launch_kernel(permute_cols_kernel, dim3((unsigned)((lrows + nw - 1) / nw)), dim3(nw * 32), psm, st,
+                         false, (const __nv_bfloat16*)L, Lp, lrows, s.in2, G, s.nb1)) != cudaSuccess)
     return e;
   GemmJob j = {};
   int bn = pick_bn(s.out1);

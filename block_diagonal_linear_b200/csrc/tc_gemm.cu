@@ -15,6 +15,11 @@
 //     D[m][n] = sum_r act1[r][m] act2[r][n]; the rows are split into chunks (split-K) and
 //     each unit writes the diagonal blocks of D (m and n in the same block) as fp32
 //     partials, summed in a fixed order by a separate kernel.
+//   kind 2, block-diagonal stage, weight-stationary: as kind 0, but every CTA owns one
+//     (batch b, n tile) pair and a contiguous range of m tiles; its weight tile W[b] (BN x K)
+//     is loaded once and stays in shared memory, only A streams through the ring.  For
+//     stages whose weight tile is reused by many row tiles (few blocks, many rows) this cuts
+//     the L2 -> SM traffic per output tile roughly in half or better.
 // Roles: warp 0 TMA producer, warp 1 MMA issuer and TMEM owner, warps 2..5 epilogue
 // (one TMEM lane quadrant each: one D row per thread).  Operands move by TMA with 128B
 // swizzle into a ring of stages; two TMEM accumulator slots let the epilogue of one unit
@@ -27,24 +32,27 @@ namespace monarch {
 constexpr int kGemmThreads = 192;
 constexpr int kGemmEpiWarps = 4;
 
-template <int BN_, int KIND_>
+template <int BN_, int KIND_, int KBOX_ = 0>
 struct GemmCfg {
-  static constexpr int BN = BN_, KIND = KIND_;
+  static constexpr int BN = BN_, KIND = KIND_, KBOX = KBOX_;
   static constexpr int BM = 128;
   static constexpr int A_BYTES = BM * 128;          // 128 x 64 bf16 (K-major) or 2 x (64 x 64) (MN-major)
-  static constexpr int B_BYTES = BN * 128;          // BN x 64 (K-major) or BN/64 x (64 x 64) (MN-major)
+  static constexpr int B_BYTES = KIND == 2 ? 0 : BN * 128;  // BN x 64 (K-major) or BN/64 x (64 x 64) (MN-major)
   static constexpr int STAGE = A_BYTES + B_BYTES;
-  static constexpr int STG_BYTES = KIND == 0 ? 2 * BM * 128 : 0;  // two 128 x 64 output chunks
+  static constexpr int STG_BYTES = KIND != 1 ? 2 * BM * 128 : 0;  // two 128 x 64 output chunks
+  static constexpr int W_BYTES = KIND == 2 ? KBOX * BN * 128 : 0;  // kind 2: resident weight tile
   static constexpr int TMEM_COLS = 2 * BN <= 32 ? 32 : (2 * BN <= 64 ? 64 : (2 * BN <= 128 ? 128 : (2 * BN <= 256 ? 256 : 512)));
-  static constexpr int NSTAGE_RAW = (kSmemBudget - STG_BYTES - 1024) / STAGE;
+  static constexpr int NSTAGE_RAW = (kSmemBudget - STG_BYTES - W_BYTES - 1024) / STAGE;
   static constexpr int NSTAGE = NSTAGE_RAW > 8 ? 8 : NSTAGE_RAW;
-  static constexpr int SMEM_BYTES = STG_BYTES + NSTAGE * STAGE + 1024 + 1024;
+  static constexpr int SMEM_BYTES = STG_BYTES + W_BYTES + NSTAGE * STAGE + 1024 + 1024;
   static_assert(BN % 64 == 0 && BN <= 256, "BN");
   static_assert(NSTAGE >= 2, "shared memory");
+  static_assert(KIND != 2 || KBOX >= 1, "kind 2 needs the K extent");
 };
 
 struct GemmBars {
   uint64_t full[8], empty[8];
+  uint64_t wfull;  // kind 2: the resident weight tile
   uint64_t acc_full[2], acc_empty[2];
   uint64_t mma_done;
   uint32_t tmem_base;
@@ -74,9 +82,42 @@ __device__ __forceinline__ UnitCoord unit_coord(const GemmJob& j, int64_t u) {
   return c;
 }
 
+// Units of this CTA: i = 0, 1, ... < unit_count().  Kinds 0 and 1: unit blockIdx.x + i*gridDim.x
+// of the job.  Kind 2: the CTA's (b, n tile) pair is blockIdx.x % (nb*ntiles) and its m tiles a
+// contiguous range (the grid is a multiple of nb*ntiles).
+__device__ __forceinline__ void kind2_range(const GemmJob& j, int* b, int* nt, int* lo, int* hi) {
+  const int nwg = j.nb * j.ntiles;
+  const int wg = (int)(blockIdx.x % nwg), ci = (int)(blockIdx.x / nwg), cpw = (int)(gridDim.x / nwg);
+  *b = wg / j.ntiles;
+  *nt = wg % j.ntiles;
+  *lo = (int)((int64_t)ci * j.mtiles / cpw);
+  *hi = (int)((int64_t)(ci + 1) * j.mtiles / cpw);
+}
+__device__ __forceinline__ int64_t unit_count(const GemmJob& j) {
+  if (j.kind == 2) {
+    int b, nt, lo, hi;
+    kind2_range(j, &b, &nt, &lo, &hi);
+    return hi - lo;
+  }
+  return j.units > (int64_t)blockIdx.x ? (j.units - blockIdx.x + gridDim.x - 1) / gridDim.x : 0;
+}
+__device__ __forceinline__ UnitCoord unit_at(const GemmJob& j, int64_t i) {
+  if (j.kind == 2) {
+    int b, nt, lo, hi;
+    kind2_range(j, &b, &nt, &lo, &hi);
+    UnitCoord c;
+    c.b = b;
+    c.nt = nt;
+    c.mt = lo + (int)i;
+    c.split = 0;
+    return c;
+  }
+  return unit_coord(j, blockIdx.x + i * gridDim.x);
+}
+
 // Number of 64-wide K stages of a unit.
 __device__ __forceinline__ int unit_kstages(const GemmJob& j, const UnitCoord& c) {
-  if (j.kind == 0) return j.kboxes;
+  if (j.kind != 1) return j.kboxes;
   const int64_t r0 = (int64_t)c.split * j.split_rows;
   int64_t n = j.rows - r0;
   if (n > j.split_rows) n = j.split_rows;
@@ -90,12 +131,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                    int* status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  uint8_t* stg = smem;                      // kind 0: two 16 KB output staging chunks
-  uint8_t* ring = smem + C::STG_BYTES;
+  uint8_t* stg = smem;                      // kinds 0, 2: two 16 KB output staging chunks
+  uint8_t* wreg = smem + C::STG_BYTES;      // kind 2: resident weight tile (KBOX boxes of BN x 64)
+  uint8_t* ring = wreg + C::W_BYTES;
   GemmBars* bars = (GemmBars*)(ring + C::NSTAGE * C::STAGE);
   int* abort_flag = &bars->abort_flag;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int64_t nunits = job.units;
+  const int64_t nmine = unit_count(job);  // units of this CTA
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::NSTAGE; ++i) {
@@ -107,6 +149,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       ptx::mbar_init(&bars->acc_empty[i], kGemmEpiWarps);
     }
     ptx::mbar_init(&bars->mma_done, 1);
+    ptx::mbar_init(&bars->wfull, 1);
     bars->abort_flag = 0;
     ptx::fence_mbar_init();
   }
@@ -127,12 +170,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     if (lane == 0) {
       ptx::tma_prefetch_desc(&tmA);
       ptx::tma_prefetch_desc(&tmB);
-      if (C::KIND == 0) ptx::tma_prefetch_desc(&tmY);
+      if (C::KIND != 1) ptx::tma_prefetch_desc(&tmY);
       const uint64_t pol = ptx::policy_evict_normal();
+      if (C::KIND == 2 && nmine > 0) {
+        const UnitCoord c0 = unit_at(job, 0);
+        ptx::mbar_arrive_expect_tx(&bars->wfull, C::W_BYTES);
+        for (int kb = 0; kb < C::KBOX; ++kb)
+          ptx::tma_load_2d(wreg + kb * (C::BN * 128), &tmB, &bars->wfull, kb * 64, c0.b * job.b_b + c0.nt * C::BN,
+                           pol);
+      }
       uint32_t it = 0;
       bool ok = true;
-      for (int64_t u = blockIdx.x; u < nunits && ok; u += gridDim.x) {
-        const UnitCoord c = unit_coord(job, u);
+      for (int64_t i = 0; i < nmine && ok; ++i) {
+        const UnitCoord c = unit_at(job, i);
         const int nk = unit_kstages(job, c);
         for (int kb = 0; kb < nk; ++kb, ++it) {
           const int st = it % C::NSTAGE;
@@ -140,10 +190,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           uint8_t* sa = ring + st * C::STAGE;
           uint8_t* sb = sa + C::A_BYTES;
           ptx::mbar_arrive_expect_tx(&bars->full[st], C::STAGE);
-          if (C::KIND == 0) {
+          if (C::KIND != 1) {
             const int ax = gcol(c.b, job.a_b, kb, job.a_grp, job.a_gs);
             ptx::tma_load_2d(sa, &tmA, &bars->full[st], ax, c.mt * C::BM, pol);
-            ptx::tma_load_2d(sb, &tmB, &bars->full[st], kb * 64, c.b * job.b_b + c.nt * C::BN, pol);
+            if (C::KIND == 0) ptx::tma_load_2d(sb, &tmB, &bars->full[st], kb * 64, c.b * job.b_b + c.nt * C::BN, pol);
           } else {
             const int row = (int)((int64_t)c.split * job.split_rows + (int64_t)kb * 64);
             const int ax = c.b * job.a_b + c.mt * C::BM;
@@ -159,6 +209,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const uint32_t issued = it;
       for (uint32_t k = (issued > (uint32_t)C::NSTAGE ? issued - C::NSTAGE : 0); k < issued; ++k)
         ptx::mbar_wait_bounded(&bars->full[k % C::NSTAGE], (k / C::NSTAGE) & 1, kWaitLimitNs);
+      if (C::KIND == 2 && nmine > 0) ptx::mbar_wait_bounded(&bars->wfull, 0, kWaitLimitNs);
     }
   } else if (warp == 1) {
     // ================================================================ MMA issuer
@@ -169,12 +220,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     // the 64-wide M/N halves), a K step of 16 advances two 8-row groups (2 KB).
     const uint64_t dA = MN ? make_sdesc_lbo(ptx::smem_u32(ring), 8192, 1024, 2) : make_sdesc(ptx::smem_u32(ring), 1024, 2);
     const uint64_t dB = MN ? make_sdesc_lbo(ptx::smem_u32(ring + C::A_BYTES), 8192, 1024, 2)
-                           : make_sdesc(ptx::smem_u32(ring + C::A_BYTES), 1024, 2);
+                           : make_sdesc(ptx::smem_u32(C::KIND == 2 ? wreg : ring + C::A_BYTES), 1024, 2);
     constexpr uint64_t kstep = MN ? (2048 >> 4) : (32 >> 4);
     uint32_t it = 0, n = 0;
     bool ok = true;
-    for (int64_t u = blockIdx.x; u < nunits && ok; u += gridDim.x, ++n) {
-      const UnitCoord c = unit_coord(job, u);
+    if (C::KIND == 2 && nmine > 0) ok = warp_wait_or_abort(lane, &bars->wfull, 0, abort_flag, status);
+    for (int64_t i = 0; i < nmine && ok; ++i, ++n) {
+      const UnitCoord c = unit_at(job, i);
       const int nk = unit_kstages(job, c);
       const int slot = n & 1;
       if (!warp_wait_or_abort(lane, &bars->acc_empty[slot], ((n >> 1) & 1) ^ 1, abort_flag, status)) { ok = false; break; }
@@ -185,9 +237,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         if (!warp_wait_or_abort(lane, &bars->full[st], (it / C::NSTAGE) & 1, abort_flag, status)) { ok = false; break; }
         ptx::tc_fence_after();
         const uint64_t soff = (uint64_t)((st * C::STAGE) >> 4);
+        // kind 2: B is box kb of the resident weight tile
+        const uint64_t boff = C::KIND == 2 ? (uint64_t)((kb * C::BN * 128) >> 4) : soff;
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          ptx::mma_bf16_ss_elect(d, dA + soff + kk * kstep, dB + soff + kk * kstep, idesc,
+          ptx::mma_bf16_ss_elect(d, dA + soff + kk * kstep, dB + boff + kk * kstep, idesc,
                                  (kb > 0 || kk > 0) ? 1u : 0u);
         ptx::mma_commit_elect(&bars->empty[st]);
       }
@@ -206,13 +260,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const uint32_t stg_s = ptx::smem_u32(stg);
     uint32_t n = 0, chunk_n = 0;
     bool ok = true;
-    for (int64_t u = blockIdx.x; u < nunits && ok; u += gridDim.x, ++n) {
-      const UnitCoord c = unit_coord(job, u);
+    for (int64_t i = 0; i < nmine && ok; ++i, ++n) {
+      const UnitCoord c = unit_at(job, i);
       const int slot = n & 1;
       if (!wait_or_abort(&bars->acc_full[slot], (n >> 1) & 1, abort_flag, status)) { ok = false; break; }
       ptx::tc_fence_after();
       const uint32_t tb = tmem + lane_off + slot * C::BN;
-      if (C::KIND == 0) {
+      if (C::KIND != 1) {
         for (int ch = 0; ch < C::BN / 64; ++ch, ++chunk_n) {
           uint32_t v[64];
 #pragma unroll
@@ -280,7 +334,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(&bars->acc_empty[slot]);
     }
-    if (C::KIND == 0 && leader) ptx::bulk_wait_all();
+    if (C::KIND != 1 && leader) ptx::bulk_wait_all();
   }
 
   ptx::tc_fence_before();
@@ -289,15 +343,25 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   if (warp == 1) ptx::tmem_dealloc(tmem, C::TMEM_COLS);
 }
 
-template <int BN, int KIND>
+template <int BN, int KIND, int KBOX = 0>
 static cudaError_t launch_gemm_cfg(const CUtensorMap& mA, const CUtensorMap& mB, const CUtensorMap& mY,
                                    const GemmJob& job, float* partial, int* status, cudaStream_t st,
                                    bool pdl) {
-  using C = GemmCfg<BN, KIND>;
+  using C = GemmCfg<BN, KIND, KBOX>;
   cudaError_t e = ensure_smem_attr((const void*)tc_gemm_kernel<C>, C::SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  int64_t grid = num_sms();
-  if (grid > job.units) grid = job.units;
+  int64_t grid;
+  if (KIND == 2) {
+    // CTAs per (b, n tile) pair: fill the SMs, at most one per m tile
+    const int64_t nwg = (int64_t)job.nb * job.ntiles;
+    int64_t cpw = num_sms() / nwg;
+    if (cpw < 1) cpw = 1;
+    if (cpw > job.mtiles) cpw = job.mtiles;
+    grid = nwg * cpw;
+  } else {
+    grid = num_sms();
+    if (grid > job.units) grid = job.units;
+  }
   return launch_kernel(tc_gemm_kernel<C>, dim3((unsigned)grid), dim3(kGemmThreads), C::SMEM_BYTES, st, pdl,
                        mA, mB, mY, job, partial, status);
 }
@@ -310,9 +374,28 @@ cudaError_t gemm_bd(const void* A, int64_t rows, int64_t a_cols, const void* W, 
       !make_map_2d(&mB, W, (uint64_t)K, (uint64_t)w_rows, 64, (uint32_t)BN, CU_TENSOR_MAP_SWIZZLE_128B) ||
       !make_map_2d(&mY, Y, (uint64_t)y_cols, (uint64_t)rows, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
-  job.kind = 0;
   job.mtiles = (int)((rows + 127) / 128);
   job.units = (int64_t)job.mtiles * job.nb * job.ntiles;
+  // weight-stationary when the (BN x K) weight tile fits the resident region and is reused by
+  // at least two row tiles per CTA
+  const int kbox = job.kboxes;
+  const int64_t nwg = (int64_t)job.nb * job.ntiles;
+  const bool stationary = (int64_t)job.mtiles >= 2 * ((num_sms() / nwg) > 0 ? (num_sms() / nwg) : 1);
+  job.kind = 0;
+  if (stationary) {
+    job.kind = 2;
+    if (BN == 256 && kbox == 4) return launch_gemm_cfg<256, 2, 4>(mA, mB, mY, job, nullptr, status, st, pdl);
+    if (BN == 256 && kbox == 2) return launch_gemm_cfg<256, 2, 2>(mA, mB, mY, job, nullptr, status, st, pdl);
+    if (BN == 128 && kbox == 8) return launch_gemm_cfg<128, 2, 8>(mA, mB, mY, job, nullptr, status, st, pdl);
+    if (BN == 128 && kbox == 4) return launch_gemm_cfg<128, 2, 4>(mA, mB, mY, job, nullptr, status, st, pdl);
+    if (BN == 128 && kbox == 2) return launch_gemm_cfg<128, 2, 2>(mA, mB, mY, job, nullptr, status, st, pdl);
+    if (BN == 64 && kbox == 16) return launch_gemm_cfg<64, 2, 16>(mA, mB, mY, job, nullptr, status, st, pdl);
+    if (BN == 64 && kbox == 4) return launch_gemm_cfg<64, 2, 4>(mA, mB, mY, job, nullptr, status, st, pdl);
+    if (BN == 64 && kbox == 3) return launch_gemm_cfg<64, 2, 3>(mA, mB, mY, job, nullptr, status, st, pdl);
+    if (BN == 64 && kbox == 2) return launch_gemm_cfg<64, 2, 2>(mA, mB, mY, job, nullptr, status, st, pdl);
+    if (BN == 64 && kbox == 1) return launch_gemm_cfg<64, 2, 1>(mA, mB, mY, job, nullptr, status, st, pdl);
+    job.kind = 0;  // no resident configuration for this tile: stream the weights
+  }
   switch (BN) {
     case 64: return launch_gemm_cfg<64, 0>(mA, mB, mY, job, nullptr, status, st, pdl);
     case 128: return launch_gemm_cfg<128, 0>(mA, mB, mY, job, nullptr, status, st, pdl);

@@ -59,6 +59,11 @@ cudaError_t wgrad_tc(const void* A1, int64_t a_cols, int64_t blk_a, const void* 
                      int64_t nblocks, int b_base, int b_grp, int b_gs, int64_t rows, WgradSplit sp, float* partial,
                      int64_t p_stride, int64_t p_off, int* status, cudaStream_t st);
 
+// Rt[k][i][p] = R[k][p][i] and Lt[j][c][o] = L[j][o][cmap(c)] (bf16), one launch;
+// cmap(c) = (c % G)*nb1 + c / G when G > 0, else c.
+cudaError_t factor_transposes(const void* R, void* Rt, const void* L, void* Lt, const Shape& s, int G,
+                              cudaStream_t st);
+
 // Smallest g <= 8 dividing nblocks with g*kw and g*nw multiples of 64 (0 if none).
 int pack_factor(int nblocks, int kw, int nw);
 // Packed block-diagonal weights (see bwd_gemm.cu) and the stage that uses them.

@@ -159,6 +159,10 @@ __global__ void __launch_bounds__(kRowsThreads, 1)
           ptx::mbar_arrive_expect_tx(&bars->full[st], C::XBOX_BYTES);
           ptx::tma_load_2d(ring + st * C::STAGE_BYTES, &tmX, &bars->full[st], b * 64, row0, pol_x);
         }
+        // this unit's X is on its way: pull the next unit's X tile into L2 now, so that HBM
+        // streams it during this unit's L stage and stores instead of after them
+        if (ok && u + gridDim.x < nunits)
+          for (int b = 0; b < C::NXB; ++b) ptx::tma_prefetch_l2_2d(&tmX, b * 64, (int)((u + gridDim.x) * C::BM));
         for (int sp = 0; sp < C::NSTAGE2 && ok; ++sp, ++it) {
           const int st = it % C::NSTAGE;
           if (!wait_or_abort(&bars->empty[st], ((it / C::NSTAGE) & 1) ^ 1, abort_flag, status)) { ok = false; break; }

@@ -145,6 +145,9 @@ __global__ void __launch_bounds__(kWideThreads, 1)
           ptx::mbar_arrive_expect_tx(&bars->xfull[b], xbytes);
           ptx::tma_load_2d(zbuf + b * C::ATOM, &tmX, &bars->xfull[b], b * 64, row0, pol_x);
         }
+        // pull the next unit's X tile into L2 while this unit computes
+        if (u + gridDim.x < nunits)
+          for (int b = 0; b < C::NXB; ++b) ptx::tma_prefetch_l2_2d(&tmX, b * 64, (int)((u + gridDim.x) * bm));
       }
       // no TMA load may still target this CTA's shared memory at exit
       if (unit_n > 0)
