@@ -215,8 +215,19 @@ def run_reference(args, w, name):
 
 # --------------------------------------------------------------------------- kernel paths
 FWD_KERNEL = {2: "tc_rows_kernel", 3: "tc_wide_kernel", 4: "tc_bdgemm_kernel + permute_rows_kernel",
-              1: "tc_fwd_kernel"}
+              1: "tc_fwd_kernel", 5: "tc_gemm_kernel", 6: "tc_stage_kernel"}
 FWD_SOURCE = {2: "tc_rows", 3: "tc_wide", 4: "tc_split", 1: "tc_fwd"}
+
+
+def stage_bytes(w: dict, rows: int) -> float:
+    """Bytes the two streaming stage launches of the workspace forward must move between them:
+    each reads its input rows and factor once and writes its output rows once (the middle
+    vector Z is written by the first and read by the second)."""
+    n_in, n_mid, n_out = synthetic.sizes(w)
+    es = 2 if w["dtype"] == "bf16" else 4
+    p1 = w["nb1"] * w["out1"] * w["in1"]
+    p2 = w["nb2"] * w["out2"] * w["in2"]
+    return float(es * (rows * (n_in + n_mid) + p1 + rows * (n_mid + n_out) + p2))
 
 
 def launches(shape: dict, dtype: str, pname: str) -> int:
@@ -374,6 +385,8 @@ def main():
     dL = torch.empty_like(L)
     ws = torch.empty(max(bdl.bwd_workspace_bytes(shape, rows, w["dtype"]), 256), dtype=torch.uint8,
                      device=dev_)
+    fws_bytes = bdl.fwd_workspace_bytes(shape, rows, w["dtype"])
+    fws = torch.empty(fws_bytes, dtype=torch.uint8, device=dev_) if fws_bytes else None
     l2 = torch.cuda.get_device_properties(dev_).L2_cache_size
     flush = torch.empty(max(2 * l2, 256 << 20), dtype=torch.uint8, device=dev_)
     stream = torch.cuda.current_stream()
@@ -397,7 +410,7 @@ def main():
             torch.cuda._sleep(spin_cycles)
             ev[0].record(stream)
         if do_fwd:
-            bdl.fwd(X, R, L, shape, Y=Y)
+            bdl.fwd_ws(X, R, L, shape, Y=Y, workspace=fws)
         if ev is not None:
             ev[1].record(stream)
             flush.zero_()
@@ -469,7 +482,7 @@ def main():
             s_comp.wait_event(ev_in[b])
             s_comp.wait_event(ev_out[b])     # buffer set b's previous results are copied out
             y, dx, dr, dl = outs_d[b]
-            bdl.fwd(Xe[b], R, L, shape, Y=y)
+            bdl.fwd_ws(Xe[b], R, L, shape, Y=y, workspace=fws)
             bdl.bwd(dYe[b], Xe[b], R, L, shape, dX=dx, dR=dr, dL=dl, workspace=ws)
             if world > 1:
                 dp.allreduce_weight_grads(dr, dl)
@@ -524,7 +537,7 @@ def main():
             "roofline_frac": t_roof / t_s,
             "bound": "hbm" if a["bytes"] / hbm >= a["flops"] / tpk else "tensor",
         }
-    fpath = bdl.fwd_path(shape, w["dtype"])
+    fpath = bdl.fwd_ws_path(shape, w["dtype"])
     bpath = bdl.bwd_path(shape, w["dtype"])
     fwd_launches = launches(shape, w["dtype"], "fwd")
     bwd_launches = launches(shape, w["dtype"], "bwd")
@@ -556,6 +569,15 @@ def main():
                  "block_diagonal_linear_b200/csrc/ptx.cuh", "block_diagonal_linear_b200/csrc/tc_common.cuh"]
                 if fpath in FWD_SOURCE and fwd_launches == 1 else None)
         roof = roof_of("fwd", fwd_avg_s, kname, srcs)
+        if fpath == 6 and roof["bound"] == "hbm":
+            # the dominant kernel is the stage kernel, launched twice per pass: its own bytes
+            # (input, factor and output of each launch) over the two launches' time
+            sb = stage_bytes(w, rows)
+            roof.update({"achieved": sb / fwd_avg_s / 1e9, "algorithmic_bytes_per_launch": sb / 2,
+                         "launches_per_pass": 2,
+                         "note": "stage kernel, Z = P blockdiag(R) X then Y = P_out blockdiag(L) Z; "
+                                 "pass time / 2 per launch"})
+            roof["frac"] = roof["achieved"] / roof["peak"]
     if do_bwd:
         roof_bwd = roof_of("bwd", bwd_avg_s, "monarch_bwd (pass of %d kernels)" % bwd_launches, None)
     if roof is None:

@@ -187,9 +187,21 @@ int monarch_fwd(const void* X, const void* R, const void* L, const monarch_dims*
 }
 
 // Forward with caller scratch: the two-pass tcgen05 GEMM forward where it applies (shapes
-// whose permutation moves whole 64-column groups), otherwise the monarch_fwd kernels.
+// whose permutation moves whole 64-column groups), two streaming stage launches for the
+// square small-block shapes, otherwise the monarch_fwd kernels.
+static int fwd_ws_kind(const Shape& s, int dtype) {
+  if (dtype != MONARCH_BF16) return 0;
+  if (gemm_bwd_supported(s)) return 5;
+  if (tc_stage_supported(s)) return 6;
+  return 0;
+}
+
 static size_t fwd_ws_bytes(const Shape& s, int dtype) {
-  return (dtype == MONARCH_BF16 && gemm_bwd_supported(s)) ? gemm_fwd_workspace(s) : 0;
+  switch (fwd_ws_kind(s, dtype)) {
+    case 5: return gemm_fwd_workspace(s);
+    case 6: return (size_t)s.rows * (size_t)s.n_mid() * 2;
+    default: return 0;
+  }
 }
 
 size_t monarch_fwd_workspace_bytes(const monarch_dims* d) {
@@ -200,7 +212,8 @@ size_t monarch_fwd_workspace_bytes(const monarch_dims* d) {
 int monarch_fwd_ws_path(const monarch_dims* d) {
   if (check_dims(d) != MONARCH_OK) return -1;
   const Shape s = to_shape(*d);
-  return fwd_ws_bytes(s, d->dtype) > 0 ? 5 : fwd_path(s, d->dtype);
+  const int k = fwd_ws_kind(s, d->dtype);
+  return k != 0 ? k : fwd_path(s, d->dtype);
 }
 
 int monarch_fwd_ws(const void* X, const void* R, const void* L, const monarch_dims* d, void* Y, void* workspace,
@@ -221,8 +234,10 @@ int monarch_fwd_ws(const void* X, const void* R, const void* L, const monarch_di
   if (need == 0) return fwd_dispatch(X, R, L, Y, s, d->dtype, (cudaStream_t)stream);
   int* status = status_ptr();
   if (status == nullptr) return MONARCH_ERR_CUDA;
-  return gemm_fwd(X, R, L, Y, workspace, s, status, (cudaStream_t)stream) == cudaSuccess ? MONARCH_OK
-                                                                                           : MONARCH_ERR_CUDA;
+  const cudaError_t e = fwd_ws_kind(s, d->dtype) == 5
+                            ? gemm_fwd(X, R, L, Y, workspace, s, status, (cudaStream_t)stream)
+                            : tc_stage_fwd(X, R, L, Y, workspace, s, status, (cudaStream_t)stream);
+  return e == cudaSuccess ? MONARCH_OK : MONARCH_ERR_CUDA;
 }
 
 size_t monarch_bwd_workspace_bytes(const monarch_dims* d) {

@@ -6,6 +6,8 @@
 //   3. Z = P R x                                                (row-tile kernel, R stage only)
 //   4. dU = P^-1 (L^T dV), dX = R^T dU                          (row-tile kernel on the dual
 //                                                               map, dU stored on the side)
+// For 64 x 64 blocks (n = 4096) steps 3 and 4 are block-diagonal passes: Z and dU come from
+// streaming stages with the permutation folded in (tc_stage.cu), dX from the plain GEMM pass.
 //   5. dL[j] = sum_rows dV_j^T Z_j, dR[k] = sum_rows dU_k^T X_k (split-row weight gradient on
 //                                                               the tcgen05 GEMM, rows as K:
 //                                                               fp32 partials + fixed-order sum)
@@ -140,10 +142,16 @@ cudaError_t fast_bwd(const void* dY, const void* X, const void* R, const void* L
     // dV = P_out^-1 dY;  Z = P (blockdiag(R) X);  dZ = blockdiag(L^T) dV;  dU = P^-1 dZ;
     // dX = blockdiag(R^T) dU.  Z and dZ/dU are permuted in place.
     if (s.out_transpose && (e = permute_rows(dY, dV, s.rows, s.out2, s.nb2, st)) != cudaSuccess) return e;
-    if ((e = bdgemm64(X, R, Z, s.nb1, s.rows, status, st, true)) != cudaSuccess) return e;
-    if ((e = permute_rows(Z, Z, s.rows, s.nb1, s.out1, st)) != cudaSuccess) return e;
-    if ((e = bdgemm64(dV, Lt, dU, s.nb2, s.rows, status, st, true)) != cudaSuccess) return e;
-    if ((e = permute_rows(dU, dU, s.rows, s.out1, s.nb1, st)) != cudaSuccess) return e;
+    if (tc_stage_supported(s)) {
+      // the permutations folded into the stages that produce Z and dU (tc_stage.cu)
+      if ((e = tc_stage(X, R, Z, true, s, status, st, true)) != cudaSuccess) return e;
+      if ((e = tc_stage(dV, Lt, dU, true, s, status, st, true)) != cudaSuccess) return e;
+    } else {
+      if ((e = bdgemm64(X, R, Z, s.nb1, s.rows, status, st, true)) != cudaSuccess) return e;
+      if ((e = permute_rows(Z, Z, s.rows, s.nb1, s.out1, st)) != cudaSuccess) return e;
+      if ((e = bdgemm64(dV, Lt, dU, s.nb2, s.rows, status, st, true)) != cudaSuccess) return e;
+      if ((e = permute_rows(dU, dU, s.rows, s.out1, s.nb1, st)) != cudaSuccess) return e;
+    }
     if ((e = bdgemm64(dU, Rt, dX, s.nb1, s.rows, status, st, true)) != cudaSuccess) return e;
   } else if (s.rows > 0) {
     const size_t gsm = (size_t)kGatherWarps * (size_t)s.out2 * (size_t)(s.nb2 + 2) * 2;

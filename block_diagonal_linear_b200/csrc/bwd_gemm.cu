@@ -232,27 +232,43 @@ cudaError_t wgrad_tc(const void* A1, int64_t a_cols, int64_t blk_a, const void* 
   return gemm_wgrad(A1, a_cols, A2, b_cols, rows, BN, j, partial, status, st, true);
 }
 
-// dR = sum of the first nR partials; dL[j][o][q] = sum of the partials at in-block column
+// Row split for one weight-gradient launch on its own: as many chunks (multiples of 64 rows,
+// at least 256 rows each) as keep the launch to one wave of units on the SMs.
+WgradSplit wgrad_split_wave(int64_t rows, int64_t units_per_split) {
+  int64_t n = 148 / (units_per_split > 0 ? units_per_split : 1);
+  const int64_t maxs = rows / 256;
+  if (n > maxs) n = maxs;
+  if (n < 1) n = 1;
+  WgradSplit w;
+  const int64_t per = (rows + n - 1) / n;
+  w.rows_per_split = ((per + 63) / 64) * 64;
+  if (w.rows_per_split < 64) w.rows_per_split = 64;
+  w.nsplit = (int)((rows + w.rows_per_split - 1) / w.rows_per_split);
+  if (w.nsplit < 1) w.nsplit = 1;
+  return w;
+}
+
+// dR = fixed-order sum of its nsR partials (nR values each, from partial[0]); dL[j][o][q] =
+// fixed-order sum of its nsL partials (nL values each, after dR's) at in-block column
 // kappa(q) = (q % nb1)*G + q / nb1 (the order the gathered weight gradient wrote them in).
 __global__ void reduce_partials_gathered_kernel(const float* __restrict__ partial, __nv_bfloat16* __restrict__ dR,
-                                                __nv_bfloat16* __restrict__ dL, int64_t nR, int64_t nP, int nsplit,
-                                                int in2, int nb1, int G) {
+                                                __nv_bfloat16* __restrict__ dL, int64_t nR, int64_t nL, int nsR,
+                                                int nsL, int in2, int nb1, int G) {
   ptx::griddep_wait();
   ptx::griddep_launch_dependents();
   const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (e >= nP) return;
-  int64_t src = e;
-  if (e >= nR) {
+  if (e >= nR + nL) return;
+  float acc = 0.f;
+  if (e < nR) {
+    for (int sp = 0; sp < nsR; ++sp) acc += partial[(int64_t)sp * nR + e];
+    dR[e] = __float2bfloat16_rn(acc);
+  } else {
     const int64_t f = e - nR;
     const int q = (int)(f % in2);
-    src = nR + (f - q) + (int64_t)(q % nb1) * G + q / nb1;
+    const float* pl = partial + (int64_t)nsR * nR + (f - q) + (int64_t)(q % nb1) * G + q / nb1;
+    for (int sp = 0; sp < nsL; ++sp) acc += pl[(int64_t)sp * nL];
+    dL[f] = __float2bfloat16_rn(acc);
   }
-  float acc = 0.f;
-  for (int sp = 0; sp < nsplit; ++sp) acc += partial[(int64_t)sp * nP + src];
-  if (e < nR)
-    dR[e] = __float2bfloat16_rn(acc);
-  else
-    dL[e - nR] = __float2bfloat16_rn(acc);
 }
 
 // ---------------------------------------------------------------- host
@@ -260,27 +276,26 @@ static size_t al256(size_t b) { return (b + 255) & ~size_t(255); }
 
 struct GemmBwdWs {
   size_t rt, ltp, u, du, part, total;
-  WgradSplit sp;
+  WgradSplit spR, spL;  // each weight-gradient launch has its own row split
 };
 
-static int64_t gemm_bwd_units_per_split(const Shape& s) {
-  // dR: nb1 groups x out1/128 m tiles x in1/BN n tiles; dL: nb2 x out2/128 x in2/BN
-  const int bn1 = s.in1 >= 256 ? 256 : (s.in1 > 64 ? 128 : 64);
-  const int bn2 = s.in2 >= 256 ? 256 : (s.in2 > 64 ? 128 : 64);
-  return (int64_t)s.nb1 * (s.out1 / 128) * ((s.in1 + bn1 - 1) / bn1) +
-         (int64_t)s.nb2 * (s.out2 / 128) * ((s.in2 + bn2 - 1) / bn2);
+// Units of one row chunk of the weight-gradient GEMM: blocks x block/128 m tiles x K/BN n tiles.
+static int64_t wgrad_units_one(int nb, int out, int in) {
+  const int bn = in >= 256 ? 256 : (in > 64 ? 128 : 64);
+  return (int64_t)nb * (out / 128) * ((in + bn - 1) / bn);
 }
 
 static GemmBwdWs gemm_bwd_layout(const Shape& s) {
   GemmBwdWs w;
   const size_t nR = (size_t)s.n_R(), nL = (size_t)s.n_L();
-  w.sp = wgrad_split(s.rows, gemm_bwd_units_per_split(s));
+  w.spR = wgrad_split_wave(s.rows, wgrad_units_one(s.nb1, s.out1, s.in1));
+  w.spL = wgrad_split_wave(s.rows, wgrad_units_one(s.nb2, s.out2, s.in2));
   w.rt = 0;
   w.ltp = w.rt + al256(nR * 2);
   w.u = w.ltp + al256(nL * 2);
   w.du = w.u + al256((size_t)s.rows * (size_t)s.n_mid() * 2);
   w.part = w.du + al256((size_t)s.rows * (size_t)s.n_mid() * 2);
-  w.total = w.part + al256((size_t)w.sp.nsplit * (nR + nL) * 4);
+  w.total = w.part + al256(((size_t)w.spR.nsplit * nR + (size_t)w.spL.nsplit * nL) * 4);
   return w;
 }
 
@@ -332,17 +347,18 @@ cudaError_t gemm_bwd(const void* dY, const void* X, const void* R, const void* L
       return e;
     // 5. weight gradients
     if ((e = wgrad_tc(dU, s.n_mid(), s.out1, X, s.n_in(), s.in1, s.nb1, 0, 0, 0, s.rows,
-                      w.sp, part, nP, 0, status, st)) != cudaSuccess)
+                      w.spR, part, nR, 0, status, st)) != cudaSuccess)
       return e;
     if ((e = wgrad_tc(dY, s.n_out(), s.out2, U, s.n_mid(), s.in2, s.nb2, G, G / 64, s.out1, s.rows,
-                      w.sp, part, nP, nR, status, st)) != cudaSuccess)
+                      w.spL, part + (int64_t)w.spR.nsplit * nR, nL, 0, status, st)) != cudaSuccess)
       return e;
   } else {
-    if ((e = cudaMemsetAsync(part, 0, sizeof(float) * (size_t)w.sp.nsplit * (size_t)nP, st)) != cudaSuccess) return e;
+    const size_t np = (size_t)w.spR.nsplit * (size_t)nR + (size_t)w.spL.nsplit * (size_t)nL;
+    if ((e = cudaMemsetAsync(part, 0, sizeof(float) * np, st)) != cudaSuccess) return e;
   }
   return launch_kernel(reduce_partials_gathered_kernel, dim3((unsigned)((nP + 255) / 256)), dim3(256), 0, st, true,
-                       (const float*)part, (__nv_bfloat16*)dR, (__nv_bfloat16*)dL, nR, nP, w.sp.nsplit, s.in2, s.nb1,
-                       G);
+                       (const float*)part, (__nv_bfloat16*)dR, (__nv_bfloat16*)dL, nR, nL, w.spR.nsplit,
+                       w.spL.nsplit, s.in2, s.nb1, G);
 }
 
 // ================================================================ two-pass forward

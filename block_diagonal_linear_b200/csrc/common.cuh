@@ -129,6 +129,12 @@ cudaError_t tc_wide_fwd(const void* X, const void* R, const void* L, void* Y, co
 
 // Large square blocks (64 x 64, nb1 = nb2): block-diagonal tcgen05 GEMMs and row permutations
 // as four passes over Y (no scratch).
+bool tc_stage_supported(const Shape& s);
+cudaError_t tc_stage(const void* A, const void* W, void* out, bool ot, const Shape& s, int* status,
+                     cudaStream_t st, bool pdl);
+cudaError_t tc_stage_fwd(const void* X, const void* R, const void* L, void* Y, void* Z, const Shape& s,
+                         int* status, cudaStream_t st);
+
 bool tc_split_supported(const Shape& s);
 cudaError_t tc_split_fwd(const void* X, const void* R, const void* L, void* Y, const Shape& s,
                          int* status, cudaStream_t st);

@@ -107,7 +107,11 @@ MONARCH_API int monarch_fwd(const void* X, const void* R, const void* L, const m
  * transpose, in2 / nb1 a multiple of 64, e.g. nblocks = 4, 1024 -> 4096; monarch_fwd_ws_path
  * 5) it runs two tcgen05 GEMM passes: U = blockdiag(R) X into the workspace, then the L stage
  * reading U through 64-column gathers with L's K index reordered to match (L is reordered
- * into the workspace too).  For other shapes it runs the monarch_fwd kernels and needs no
+ * into the workspace too).  For 64 blocks of 64 x 64 per factor (n = 4096,
+ * monarch_fwd_ws_path 6) it runs two streaming stages, each with its permutation folded
+ * into the output stores and its factor's weights resident in shared memory a round of 16
+ * blocks at a time: Z = P blockdiag(R) X into the workspace (rows * n_mid bf16), then
+ * Y = P_out blockdiag(L) Z.  For other shapes it runs the monarch_fwd kernels and needs no
  * workspace (monarch_fwd_workspace_bytes returns 0; workspace may then be NULL).
  * workspace: >= monarch_fwd_workspace_bytes(d) bytes, 256-byte aligned, caller-owned; it must
  * not overlap the inputs or Y. */

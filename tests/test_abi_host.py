@@ -98,6 +98,14 @@ def test_kernel_family_selection():
     assert bdl.bwd_path(synthetic.shape_of(W["n256_fp32"]), "f32") == 0
     assert bdl.bwd_path(synthetic.shape_of(W["n4096_bf16"]), "bf16") == 1
     assert bdl.bwd_path(synthetic.shape_of(W["r768x3072_bf16"]), "bf16") == 3
+    # workspace forward: two-pass GEMM (5), streaming stages (6), else the monarch_fwd family
+    assert bdl.fwd_ws_path(synthetic.shape_of(W["nblk4_1024x4096_bf16"]), "bf16") == 5
+    assert bdl.fwd_ws_path(synthetic.shape_of(W["n4096_bf16"]), "bf16") == 6
+    assert bdl.fwd_ws_path(synthetic.shape_of(W["n4096_bf16"]), "f32") == 0
+    assert bdl.fwd_ws_path(synthetic.shape_of(W["n1024_bf16"]), "bf16") == 2
+    assert bdl.fwd_ws_path(synthetic.shape_of(W["r768x3072_bf16"]), "bf16") == 3
+    n = synthetic.shape_of(W["n4096_bf16"])
+    assert bdl.fwd_workspace_bytes(n, 100, "bf16") == 100 * 4096 * 2
     assert bdl.bwd_path(synthetic.shape_of(W["nblk4_1024x4096_bf16"]), "bf16") == 2
     assert bdl.bwd_path(synthetic.shape_of(W["nblk4_1024x4096_bf16"]), "f32") == 0
 

@@ -99,11 +99,16 @@ def test_backward_exact(case):
             what, len(bad), tuple(bad[0]), g[tuple(bad[0])], r[tuple(bad[0])])
 
 
-@pytest.mark.parametrize("case", [c for c in CASES if c[0] in ("nblk4_group", "nblk2_gemm")], ids=_ids)
+WS_PATHS = {"nblk4_group": 5, "nblk2_gemm": 5, "n4096_split": 6}
+
+
+@pytest.mark.parametrize("case", [c for c in CASES if c[0] in WS_PATHS], ids=_ids)
 def test_forward_with_workspace_exact(case):
-    """monarch_fwd_ws: the two-pass tcgen05 GEMM forward (U in the workspace, 64-column gathers)."""
-    _, shape, dtype, rows, _, _ = case
-    assert bdl.fwd_ws_path(shape, dtype) == 5
+    """monarch_fwd_ws: the two-pass tcgen05 GEMM forward (U in the workspace, 64-column
+    gathers; path 5) or the two streaming stages with folded permutations (Z in the workspace;
+    path 6)."""
+    name, shape, dtype, rows, _, _ = case
+    assert bdl.fwd_ws_path(shape, dtype) == WS_PATHS[name]
     inp = synthetic.make_sparse_sign_inputs(dict(shape, rows=rows), seed=23)
     _check_exact_range(inp)
     ref = oracle.forward(shape, inp["X"], inp["R"], inp["L"])

@@ -222,7 +222,7 @@ def test_workspace_too_small_is_an_error():
     assert e.value.code == bdl.CODES["MONARCH_ERR_WORKSPACE"]
 
 
-@pytest.mark.parametrize("name", ["nblk4_1024x4096_bf16", "nblk4_1024x4096_bf16_b1000"])
+@pytest.mark.parametrize("name", ["nblk4_1024x4096_bf16", "nblk4_1024x4096_bf16_b1000", "n4096_bf16"])
 def test_forward_with_workspace_full_size(name):
     """monarch_fwd_ws at the full workload size (the launch the benchmark times): every entry
     against the oracle, normwise."""
@@ -234,3 +234,19 @@ def test_forward_with_workspace_full_size(name):
     assert bdl.last_device_status() == 0
     ref = oracle.forward(shape, inp["X"].f64, inp["R"].f64, inp["L"].f64)
     check(to_f64(Y), ref, "bf16", name + " Y (workspace forward)")
+
+
+@pytest.mark.parametrize("rows", [1, 63, 64, 65, 129, 1000, 2405])
+def test_stage_forward_tile_edges(rows):
+    """The streaming-stage forward (monarch_fwd_ws, path 6) at 64-row unit edges and with more
+    units than CTAs: Y pre-filled with NaN, so an entry the drain does not write fails."""
+    w = W["n4096_bf16"]
+    shape = synthetic.shape_of(w)
+    assert bdl.fwd_ws_path(shape, "bf16") == 6
+    inp = synthetic.make_inputs(w, seed=9, rows=rows)
+    d = dev_inputs(inp)
+    Y = torch.full((rows, w["nb2"] * w["out2"]), float("nan"), dtype=torch.bfloat16, device="cuda")
+    bdl.fwd_ws(d["X"], d["R"], d["L"], shape, Y=Y)
+    assert bdl.last_device_status() == 0
+    ref = oracle.forward(shape, inp["X"].f64, inp["R"].f64, inp["L"].f64)
+    check(to_f64(Y), ref, "bf16", "Y")
