@@ -192,7 +192,7 @@ int monarch_fwd(const void* X, const void* R, const void* L, const monarch_dims*
 static int fwd_ws_kind(const Shape& s, int dtype) {
   if (dtype != MONARCH_BF16) return 0;
   if (gemm_bwd_supported(s)) return 5;
-  if (tc_stage_supported(s)) return 6;
+  if (tc_stage_fwd_supported(s)) return 6;
   return 0;
 }
 

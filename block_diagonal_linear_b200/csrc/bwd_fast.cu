@@ -144,8 +144,8 @@ cudaError_t fast_bwd(const void* dY, const void* X, const void* R, const void* L
     if (s.out_transpose && (e = permute_rows(dY, dV, s.rows, s.out2, s.nb2, st)) != cudaSuccess) return e;
     if (tc_stage_supported(s)) {
       // the permutations folded into the stages that produce Z and dU (tc_stage.cu)
-      if ((e = tc_stage(X, R, Z, true, s, status, st, true)) != cudaSuccess) return e;
-      if ((e = tc_stage(dV, Lt, dU, true, s, status, st, true)) != cudaSuccess) return e;
+      if ((e = tc_stage(X, R, Z, StageKind::R, s, status, st, true)) != cudaSuccess) return e;
+      if ((e = tc_stage(dV, Lt, dU, StageKind::Lt, s, status, st, true)) != cudaSuccess) return e;
     } else {
       if ((e = bdgemm64(X, R, Z, s.nb1, s.rows, status, st, true)) != cudaSuccess) return e;
       if ((e = permute_rows(Z, Z, s.rows, s.nb1, s.out1, st)) != cudaSuccess) return e;

@@ -562,13 +562,28 @@ cudaError_t packed_bwd(const void* dY, const void* X, const void* R, const void*
                          (const __nv_bfloat16*)R, (const __nv_bfloat16*)L, Wz, Wx, Wu, s, pk.gz, pk.gx)) !=
       cudaSuccess)
     return e;
+  const bool staged = tc_stage_supported(s);
+  if (staged && s.rows > 0) {
+    // the streaming stages take the plain factors: L^T into the (then unused) packed L^T
+    // region, R^T into the packed-R region (the transpose helper writes both)
+    if ((e = factor_transposes(R, Wu, L, Wz, s, 0, st)) != cudaSuccess) return e;
+  }
   if (s.rows > 0) {
     if (s.out_transpose && (e = permute_rows(dY, dV, s.rows, s.out2, s.nb2, st)) != cudaSuccess) return e;
-    if ((e = packed_stage(dV, s.rows, Wz, dZ, s.nb2, s.out2, s.in2, pk.gz, status, st)) != cudaSuccess) return e;
-    if ((e = permute_rows(dZ, dU, s.rows, s.out1, s.nb1, st)) != cudaSuccess) return e;
+    if (staged) {
+      // dU = P^-1 blockdiag(L^T) dV in one streaming stage (no dZ pass, no row transpose)
+      if ((e = tc_stage(dV, Wz, dU, StageKind::Lt, s, status, st, true)) != cudaSuccess) return e;
+    } else {
+      if ((e = packed_stage(dV, s.rows, Wz, dZ, s.nb2, s.out2, s.in2, pk.gz, status, st)) != cudaSuccess) return e;
+      if ((e = permute_rows(dZ, dU, s.rows, s.out1, s.nb1, st)) != cudaSuccess) return e;
+    }
     if ((e = packed_stage(dU, s.rows, Wx, dX, s.nb1, s.out1, s.in1, pk.gx, status, st)) != cudaSuccess) return e;
-    if ((e = packed_stage(X, s.rows, Wu, U, s.nb1, s.in1, s.out1, pk.gx, status, st)) != cudaSuccess) return e;
-    if ((e = permute_rows(U, Z, s.rows, s.nb1, s.out1, st)) != cudaSuccess) return e;
+    if (staged) {
+      if ((e = tc_stage(X, R, Z, StageKind::R, s, status, st, true)) != cudaSuccess) return e;  // Z = P R x
+    } else {
+      if ((e = packed_stage(X, s.rows, Wu, U, s.nb1, s.in1, s.out1, pk.gx, status, st)) != cudaSuccess) return e;
+      if ((e = permute_rows(U, Z, s.rows, s.nb1, s.out1, st)) != cudaSuccess) return e;
+    }
     if ((e = wgrad_tc(dU, s.n_mid(), s.out1, X, s.n_in(), s.in1, s.nb1, 0, 0, 0, s.rows, w.sp, part, nP, 0,
                       status, st)) != cudaSuccess)
       return e;

@@ -129,8 +129,13 @@ cudaError_t tc_wide_fwd(const void* X, const void* R, const void* L, void* Y, co
 
 // Large square blocks (64 x 64, nb1 = nb2): block-diagonal tcgen05 GEMMs and row permutations
 // as four passes over Y (no scratch).
+// Streaming block-diagonal stages with the row permutation folded into the stores (tc_stage.cu):
+//   R:  Z  = P blockdiag(R) X          L:  Y  = P_out blockdiag(L) Z
+//   Lt: dU = P^-1 blockdiag(L^T) dV     Rt: dX = blockdiag(R^T) dU
+enum class StageKind { R, L, Lt, Rt };
 bool tc_stage_supported(const Shape& s);
-cudaError_t tc_stage(const void* A, const void* W, void* out, bool ot, const Shape& s, int* status,
+bool tc_stage_fwd_supported(const Shape& s);
+cudaError_t tc_stage(const void* A, const void* W, void* out, StageKind k, const Shape& s, int* status,
                      cudaStream_t st, bool pdl);
 cudaError_t tc_stage_fwd(const void* X, const void* R, const void* L, void* Y, void* Z, const Shape& s,
                          int* status, cudaStream_t st);

@@ -307,27 +307,51 @@ static cudaError_t launch_stage(const void* A, const void* W, void* out, int64_t
                        pdl, mA, mO, (const __nv_bfloat16*)W, (__nv_bfloat16*)out, rows, status);
 }
 
+// ---------------------------------------------------------------- shapes
 // 64 blocks of 64 x 64 per factor (n = 4096): one round per CTA group, 128 KB of weights each.
 using Stage64T = StageCfg<64, 64, 64, 1, 1>;
 using Stage64N = StageCfg<64, 64, 64, 0, 1>;
+// 768 -> 3072 (R: 16 blocks of 48 x 48; L: 48 blocks of 64 x 16): every factor fits resident.
+// Its backward's Z and dU passes use stages; its forward stays the fused row-tile kernel, which
+// measured faster than two stages (32.8 vs 35.8 us for 8192 rows).
+using StageR768 = StageCfg<16, 48, 48, 1, 1>;   // Z = P blockdiag(R) X
+using StageLt768 = StageCfg<48, 64, 16, 1, 3>;  // dU = P^-1 blockdiag(L^T) dV
 
-bool tc_stage_supported(const Shape& s) { return tc_split_supported(s) && s.nb1 == 64; }
-
-// out = (OT ? P : identity) blockdiag(W) A for one stage of a tc_stage_supported shape
-// (W: nb1 blocks of 64 x 64).
-cudaError_t tc_stage(const void* A, const void* W, void* out, bool ot, const Shape& s, int* status,
-                     cudaStream_t st, bool pdl) {
-  if (!tc_stage_supported(s)) return cudaErrorNotSupported;
-  return ot ? launch_stage<Stage64T>(A, W, out, s.rows, status, st, pdl)
-            : launch_stage<Stage64N>(A, W, out, s.rows, status, st, pdl);
+static bool is_sq64(const Shape& s) { return tc_split_supported(s) && s.nb1 == 64; }
+static bool is_r768(const Shape& s) {
+  return s.nb1 == 16 && s.in1 == 48 && s.out1 == 48 && s.nb2 == 48 && s.in2 == 16 && s.out2 == 64 &&
+         s.out_transpose == 1;
 }
 
-// Y = X M^T as two stages through the caller's middle buffer Z (rows x n_mid bf16).
+bool tc_stage_supported(const Shape& s) { return is_sq64(s) || is_r768(s); }
+// Shapes whose workspace forward is the two stages (R, then L).
+bool tc_stage_fwd_supported(const Shape& s) { return is_sq64(s); }
+
+// One stage of a tc_stage_supported shape (see StageKind in common.cuh).
+cudaError_t tc_stage(const void* A, const void* W, void* out, StageKind k, const Shape& s, int* status,
+                     cudaStream_t st, bool pdl) {
+  if (is_sq64(s)) {
+    const bool ot = k == StageKind::R || k == StageKind::Lt || (k == StageKind::L && s.out_transpose == 1);
+    return ot ? launch_stage<Stage64T>(A, W, out, s.rows, status, st, pdl)
+              : launch_stage<Stage64N>(A, W, out, s.rows, status, st, pdl);
+  }
+  if (is_r768(s)) {
+    switch (k) {
+      case StageKind::R: return launch_stage<StageR768>(A, W, out, s.rows, status, st, pdl);
+      case StageKind::Lt: return launch_stage<StageLt768>(A, W, out, s.rows, status, st, pdl);
+      default: return cudaErrorNotSupported;
+    }
+  }
+  return cudaErrorNotSupported;
+}
+
+// Y = X M^T as two stages through the caller's middle buffer Z (rows x n_mid bf16), for the
+// tc_stage_fwd_supported shapes.
 cudaError_t tc_stage_fwd(const void* X, const void* R, const void* L, void* Y, void* Z, const Shape& s,
                          int* status, cudaStream_t st) {
-  cudaError_t e = tc_stage(X, R, Z, true, s, status, st, false);
+  cudaError_t e = tc_stage(X, R, Z, StageKind::R, s, status, st, false);
   if (e != cudaSuccess) return e;
-  return tc_stage(Z, L, Y, s.out_transpose == 1, s, status, st, true);
+  return tc_stage(Z, L, Y, StageKind::L, s, status, st, true);
 }
 
 }  // namespace monarch

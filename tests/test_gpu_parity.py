@@ -236,11 +236,11 @@ def test_forward_with_workspace_full_size(name):
     check(to_f64(Y), ref, "bf16", name + " Y (workspace forward)")
 
 
-@pytest.mark.parametrize("rows", [1, 63, 64, 65, 129, 1000, 2405])
-def test_stage_forward_tile_edges(rows):
+@pytest.mark.parametrize("name,rows", [("n4096_bf16", r) for r in (1, 63, 64, 65, 129, 1000, 2405)])
+def test_stage_forward_tile_edges(name, rows):
     """The streaming-stage forward (monarch_fwd_ws, path 6) at 64-row unit edges and with more
     units than CTAs: Y pre-filled with NaN, so an entry the drain does not write fails."""
-    w = W["n4096_bf16"]
+    w = W[name]
     shape = synthetic.shape_of(w)
     assert bdl.fwd_ws_path(shape, "bf16") == 6
     inp = synthetic.make_inputs(w, seed=9, rows=rows)
