@@ -131,10 +131,10 @@ cudaError_t fast_bwd(const void* dY, const void* X, const void* R, const void* L
   float* part = (float*)(base + w.part);
   const int64_t nR = s.n_R(), nP = s.n_R() + s.n_L();
   cudaError_t e;
-  // All six launches use programmatic dependent launch: each kernel waits for the previous
-  // grid of the stream (griddep_wait) before touching its data, so the next launch and its
-  // prologue overlap the tail of the current one.
-  if ((e = factor_transposes(R, Rt, L, Lt, s, 0, st)) != cudaSuccess) return e;
+  // All launches use programmatic dependent launch: each kernel waits for the previous grid of
+  // the stream (griddep_wait) before touching its data, so the next launch and its prologue
+  // overlap the tail of the current one.  The factor transposes (Rt, Lt) are needed only from the
+  // dual stage on: they are launched right after the Z pass and run concurrently with it.
   const WgradSplit sp = wg_split(s);
   const bool split = is_split_square(s);
   if (split && !s.out_transpose) dV = (__nv_bfloat16*)dY;  // dV[j][o] = dy[j*out2 + o]: no copy
@@ -144,11 +144,14 @@ cudaError_t fast_bwd(const void* dY, const void* X, const void* R, const void* L
     if (s.out_transpose && (e = permute_rows(dY, dV, s.rows, s.out2, s.nb2, st)) != cudaSuccess) return e;
     if (tc_stage_supported(s)) {
       // the permutations folded into the stages that produce Z and dU (tc_stage.cu)
-      if ((e = tc_stage(X, R, Z, StageKind::R, s, status, st, true)) != cudaSuccess) return e;
-      if ((e = tc_stage(dV, Lt, dU, StageKind::Lt, s, status, st, true)) != cudaSuccess) return e;
+      if ((e = tc_stage(X, R, Z, StageKind::R, s, status, st, true, true)) != cudaSuccess) return e;
+      if ((e = factor_transposes(R, Rt, L, Lt, s, 0, st, true)) != cudaSuccess) return e;
+      // Lt comes from the launch just before: read it after the wait
+      if ((e = tc_stage(dV, Lt, dU, StageKind::Lt, s, status, st, true, false)) != cudaSuccess) return e;
     } else {
       if ((e = bdgemm64(X, R, Z, s.nb1, s.rows, status, st, true)) != cudaSuccess) return e;
       if ((e = permute_rows(Z, Z, s.rows, s.nb1, s.out1, st)) != cudaSuccess) return e;
+      if ((e = factor_transposes(R, Rt, L, Lt, s, 0, st, true)) != cudaSuccess) return e;
       if ((e = bdgemm64(dV, Lt, dU, s.nb2, s.rows, status, st, true)) != cudaSuccess) return e;
       if ((e = permute_rows(dU, dU, s.rows, s.out1, s.nb1, st)) != cudaSuccess) return e;
     }
@@ -159,6 +162,7 @@ cudaError_t fast_bwd(const void* dY, const void* X, const void* R, const void* L
                            (const __nv_bfloat16*)dY, dV, s)) != cudaSuccess)
       return e;
     if ((e = tc_rows_middle(X, R, Z, s, status, st)) != cudaSuccess) return e;
+    if ((e = factor_transposes(R, Rt, L, Lt, s, 0, st, true)) != cudaSuccess) return e;
     if ((e = tc_rows_dual(dV, Lt, Rt, dX, dU, s, status, st)) != cudaSuccess) return e;
   }
   if (s.rows > 0) {

@@ -79,15 +79,21 @@ __device__ __forceinline__ void factor_tile(const FactorT& f, int cta, uint16_t*
   }
 }
 
-__global__ void __launch_bounds__(256) factor_transpose_kernel(FactorT f0, FactorT f1) {
+// after_reader: launched (with programmatic dependent launch) right behind a kernel that neither
+// reads nor writes Rt / Lt and that passed its own grid-dependency wait before letting this grid
+// start; then every earlier reader of Rt / Lt has finished, so the transposes run concurrently
+// with that kernel and wait for it only at the end (so that the kernels after this one, which
+// wait for this grid, also see that kernel's results).  Otherwise: the usual wait first.
+__global__ void __launch_bounds__(256) factor_transpose_kernel(FactorT f0, FactorT f1, int after_reader) {
   extern __shared__ __align__(16) uint16_t fsm[];
-  ptx::griddep_wait();  // the outputs may still be read by the previous kernels of the stream
+  if (!after_reader) ptx::griddep_wait();  // the outputs may still be read by the previous kernels
   ptx::griddep_launch_dependents();
   const int cta = (int)blockIdx.x;
   if (cta < f0.ctas)
     factor_tile(f0, cta, fsm);
   else
     factor_tile(f1, cta - f0.ctas, fsm);
+  if (after_reader) ptx::griddep_wait();
 }
 
 static FactorT factor_job(const void* src, void* dst, int nblk, int A, int B, int G, int nbk) {
@@ -107,7 +113,7 @@ __global__ void factor_transpose_flat_kernel(const __nv_bfloat16* __restrict__ R
 
 // Rt[k][i][p] = R[k][p][i] and Lt[j][c][o] = L[j][o][cmap(c)] in one launch (G as above).
 cudaError_t factor_transposes(const void* R, void* Rt, const void* L, void* Lt, const Shape& s, int G,
-                              cudaStream_t st) {
+                              cudaStream_t st, bool after_reader) {
   if (!factor_transpose_ok(s.out1, s.in1) || !factor_transpose_ok(s.out2, s.in2)) {
     const int64_t n = s.n_R() + s.n_L();
     return launch_kernel(factor_transpose_flat_kernel, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, st, true,
@@ -121,7 +127,7 @@ cudaError_t factor_transposes(const void* R, void* Rt, const void* L, void* Lt, 
   cudaError_t e = ensure_smem_attr((const void*)factor_transpose_kernel, (int)smem);
   if (e != cudaSuccess) return e;
   return launch_kernel(factor_transpose_kernel, dim3((unsigned)(f0.ctas + f1.ctas)), dim3(256), smem, st, true, f0,
-                       f1);
+                       f1, after_reader ? 1 : 0);
 }
 
 // Elementwise form of the same transposes, for factor widths beyond the staged tile.
@@ -151,7 +157,9 @@ __global__ void __launch_bounds__(kPermColWarps * 32)
     permute_cols_kernel(const __nv_bfloat16* __restrict__ L, __nv_bfloat16* __restrict__ Lp, int64_t nrows,
                         int ncols, int G, int nbk) {
   extern __shared__ __align__(16) uint16_t pcs[];
-  ptx::griddep_wait();
+  // launched right behind the R-stage GEMM, which does not touch Lp and passed its own
+  // grid-dependency wait before this grid could start: run concurrently with it, and wait for
+  // it at the end only (the L-stage GEMM after this grid needs both)
   ptx::griddep_launch_dependents();
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32, nw = blockDim.x / 32;
   uint16_t* buf = pcs + warp * ncols;
@@ -171,6 +179,7 @@ __global__ void __launch_bounds__(kPermColWarps * 32)
     }
     __syncwarp();
   }
+  ptx::griddep_wait();
 }
 
 // ---------------------------------------------------------------- weight gradient
@@ -248,9 +257,10 @@ WgradSplit wgrad_split_wave(int64_t rows, int64_t units_per_split) {
   return w;
 }
 
-// dR = fixed-order sum of its nsR partials (nR values each, from partial[0]); dL[j][o][q] =
-// fixed-order sum of its nsL partials (nL values each, after dR's) at in-block column
-// kappa(q) = (q % nb1)*G + q / nb1 (the order the gathered weight gradient wrote them in).
+// dR = fixed-order sum of its nsR partials (nR values each, from partial[0]); dL = fixed-order
+// sum of its nsL partials (nL values each, after dR's).  The dL partials are in gathered order:
+// in-block column kappa holds dL[j][o][q] with q = (kappa % G)*nb1 + kappa / G.  Threads walk
+// the partials in their own order (coalesced reads) and scatter the bf16 results.
 __global__ void reduce_partials_gathered_kernel(const float* __restrict__ partial, __nv_bfloat16* __restrict__ dR,
                                                 __nv_bfloat16* __restrict__ dL, int64_t nR, int64_t nL, int nsR,
                                                 int nsL, int in2, int nb1, int G) {
@@ -263,11 +273,11 @@ __global__ void reduce_partials_gathered_kernel(const float* __restrict__ partia
     for (int sp = 0; sp < nsR; ++sp) acc += partial[(int64_t)sp * nR + e];
     dR[e] = __float2bfloat16_rn(acc);
   } else {
-    const int64_t f = e - nR;
-    const int q = (int)(f % in2);
-    const float* pl = partial + (int64_t)nsR * nR + (f - q) + (int64_t)(q % nb1) * G + q / nb1;
+    const int64_t f = e - nR;  // position in the gathered partial layout
+    const float* pl = partial + (int64_t)nsR * nR + f;
     for (int sp = 0; sp < nsL; ++sp) acc += pl[(int64_t)sp * nL];
-    dL[f] = __float2bfloat16_rn(acc);
+    const int kappa = (int)(f % in2);
+    dL[f - kappa + (int64_t)(kappa % G) * nb1 + kappa / G] = __float2bfloat16_rn(acc);
   }
 }
 
@@ -313,7 +323,6 @@ cudaError_t gemm_bwd(const void* dY, const void* X, const void* R, const void* L
   const int64_t nR = s.n_R(), nL = s.n_L(), nP = nR + nL;
   const int G = s.in2 / s.nb1;
   cudaError_t e;
-  if ((e = factor_transposes(R, Rt, L, Ltp, s, G, st)) != cudaSuccess) return e;
   if (s.rows > 0) {
     // 2. U = blockdiag(R) X
     GemmJob j = {};
@@ -325,6 +334,8 @@ cudaError_t gemm_bwd(const void* dY, const void* X, const void* R, const void* L
     if ((e = gemm_bd(X, s.rows, s.n_in(), R, (int64_t)s.nb1 * s.out1, s.in1, U, s.n_mid(), bn, j, status, st,
                      true)) != cudaSuccess)
       return e;
+    // 1. the factor prep overlaps the U pass (which reads neither Rt nor Ltp)
+    if ((e = factor_transposes(R, Rt, L, Ltp, s, G, st, true)) != cudaSuccess) return e;
     // 3. dU = blockdiag(Ltp) dY, output group g of block j -> u[k][j*G + 64*(g % (G/64))], k = g / (G/64)
     j = GemmJob{};
     bn = pick_bn(s.in2);
@@ -378,16 +389,6 @@ cudaError_t gemm_fwd(const void* X, const void* R, const void* L, void* Y, void*
   __nv_bfloat16* U = (__nv_bfloat16*)((char*)ws + al256((size_t)s.n_L() * 2));
   const int G = s.in2 / s.nb1;
   cudaError_t e;
-  // one staged row per warp: up to 8 warps, as many as 200 KB of shared memory holds
-  const int64_t lrows = (int64_t)s.nb2 * s.out2;
-  int nw = (int)((200 * 1024) / ((size_t)s.in2 * 2));
-  if (nw > kPermColWarps) nw = kPermColWarps;
-  if (nw < 1) return cudaErrorNotSupported;
-  const size_t psm = (size_t)nw * (size_t)s.in2 * 2;
-  if ((e = ensure_smem_attr((const void*)permute_cols_kernel, (int)psm)) != cudaSuccess) return e;
-  if ((e = launch_kernel(permute_cols_kernel, dim3((unsigned)((lrows + nw - 1) / nw)), dim3(nw * 32), psm, st,
-                         false, (const __nv_bfloat16*)L, Lp, lrows, s.in2, G, s.nb1)) != cudaSuccess)
-    return e;
   GemmJob j = {};
   int bn = pick_bn(s.out1);
   j.nb = s.nb1; j.ntiles = s.out1 / bn; j.kboxes = s.in1 / 64;
@@ -396,6 +397,17 @@ cudaError_t gemm_fwd(const void* X, const void* R, const void* L, void* Y, void*
   j.y_b = s.out1; j.y_grp = s.out1 / 64; j.y_gs = 0;
   if ((e = gemm_bd(X, s.rows, s.n_in(), R, (int64_t)s.nb1 * s.out1, s.in1, U, s.n_mid(), bn, j, status, st, true)) !=
       cudaSuccess)
+    return e;
+  // the column permutation of L overlaps the R-stage pass; one staged row per warp, up to 8
+  // warps, as many as 200 KB of shared memory holds
+  const int64_t lrows = (int64_t)s.nb2 * s.out2;
+  int nw = (int)((200 * 1024) / ((size_t)s.in2 * 2));
+  if (nw > kPermColWarps) nw = kPermColWarps;
+  if (nw < 1) return cudaErrorNotSupported;
+  const size_t psm = (size_t)nw * (size_t)s.in2 * 2;
+  if ((e = ensure_smem_attr((const void*)permute_cols_kernel, (int)psm)) != cudaSuccess) return e;
+  if ((e = launch_kernel(permute_cols_kernel, dim3((unsigned)((lrows + nw - 1) / nw)), dim3(nw * 32), psm, st,
+                         true, (const __nv_bfloat16*)L, Lp, lrows, s.in2, G, s.nb1)) != cudaSuccess)
     return e;
   j = GemmJob{};
   bn = pick_bn(s.out2);
@@ -566,20 +578,22 @@ cudaError_t packed_bwd(const void* dY, const void* X, const void* R, const void*
   if (staged && s.rows > 0) {
     // the streaming stages take the plain factors: L^T into the (then unused) packed L^T
     // region, R^T into the packed-R region (the transpose helper writes both)
-    if ((e = factor_transposes(R, Wu, L, Wz, s, 0, st)) != cudaSuccess) return e;
+    if ((e = factor_transposes(R, Wu, L, Wz, s, 0, st, false)) != cudaSuccess) return e;
   }
   if (s.rows > 0) {
     if (s.out_transpose && (e = permute_rows(dY, dV, s.rows, s.out2, s.nb2, st)) != cudaSuccess) return e;
     if (staged) {
-      // dU = P^-1 blockdiag(L^T) dV in one streaming stage (no dZ pass, no row transpose)
-      if ((e = tc_stage(dV, Wz, dU, StageKind::Lt, s, status, st, true)) != cudaSuccess) return e;
+      // dU = P^-1 blockdiag(L^T) dV in one streaming stage (no dZ pass, no row transpose); L^T
+      // was written two launches back when the dY permutation sits in between
+      if ((e = tc_stage(dV, Wz, dU, StageKind::Lt, s, status, st, true, s.out_transpose == 1)) != cudaSuccess)
+        return e;
     } else {
       if ((e = packed_stage(dV, s.rows, Wz, dZ, s.nb2, s.out2, s.in2, pk.gz, status, st)) != cudaSuccess) return e;
       if ((e = permute_rows(dZ, dU, s.rows, s.out1, s.nb1, st)) != cudaSuccess) return e;
     }
     if ((e = packed_stage(dU, s.rows, Wx, dX, s.nb1, s.out1, s.in1, pk.gx, status, st)) != cudaSuccess) return e;
     if (staged) {
-      if ((e = tc_stage(X, R, Z, StageKind::R, s, status, st, true)) != cudaSuccess) return e;  // Z = P R x
+      if ((e = tc_stage(X, R, Z, StageKind::R, s, status, st, true, true)) != cudaSuccess) return e;  // Z = P R x
     } else {
       if ((e = packed_stage(X, s.rows, Wu, U, s.nb1, s.in1, s.out1, pk.gx, status, st)) != cudaSuccess) return e;
       if ((e = permute_rows(U, Z, s.rows, s.nb1, s.out1, st)) != cudaSuccess) return e;

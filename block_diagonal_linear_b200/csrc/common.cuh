@@ -132,11 +132,13 @@ cudaError_t tc_wide_fwd(const void* X, const void* R, const void* L, void* Y, co
 // Streaming block-diagonal stages with the row permutation folded into the stores (tc_stage.cu):
 //   R:  Z  = P blockdiag(R) X          L:  Y  = P_out blockdiag(L) Z
 //   Lt: dU = P^-1 blockdiag(L^T) dV     Rt: dX = blockdiag(R^T) dU
+// w_early: W may be read before the kernel's grid-dependency wait -- it is the caller's factor, or
+// it was written at least two launches earlier on the stream (that kernel has finished by then).
 enum class StageKind { R, L, Lt, Rt };
 bool tc_stage_supported(const Shape& s);
 bool tc_stage_fwd_supported(const Shape& s);
 cudaError_t tc_stage(const void* A, const void* W, void* out, StageKind k, const Shape& s, int* status,
-                     cudaStream_t st, bool pdl);
+                     cudaStream_t st, bool pdl, bool w_early);
 cudaError_t tc_stage_fwd(const void* X, const void* R, const void* L, void* Y, void* Z, const Shape& s,
                          int* status, cudaStream_t st);
 

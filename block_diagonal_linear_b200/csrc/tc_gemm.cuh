@@ -61,8 +61,10 @@ cudaError_t wgrad_tc(const void* A1, int64_t a_cols, int64_t blk_a, const void* 
 
 // Rt[k][i][p] = R[k][p][i] and Lt[j][c][o] = L[j][o][cmap(c)] (bf16), one launch;
 // cmap(c) = (c % G)*nb1 + c / G when G > 0, else c.
+// after_reader: the launch directly follows (on stream st) one of this library's kernels that does
+// not touch Rt / Lt; the transposes then overlap it (see factor_transpose_kernel).
 cudaError_t factor_transposes(const void* R, void* Rt, const void* L, void* Lt, const Shape& s, int G,
-                              cudaStream_t st);
+                              cudaStream_t st, bool after_reader);
 
 // Smallest g <= 8 dividing nblocks with g*kw and g*nw multiples of 64 (0 if none).
 int pack_factor(int nblocks, int kw, int nw);

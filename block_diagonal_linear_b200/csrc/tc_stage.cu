@@ -95,7 +95,7 @@ template <class C>
 __global__ void __launch_bounds__(kStageThreads, 1)
     tc_stage_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmO,
                     const __nv_bfloat16* __restrict__ W, __nv_bfloat16* __restrict__ out, int64_t rows,
-                    int* status) {
+                    int w_is_input, int* status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t* wsm = smem;                        // resident weights
@@ -123,9 +123,12 @@ __global__ void __launch_bounds__(kStageThreads, 1)
     ptx::tmem_alloc(&bars->tmem_base, C::TMEM_COLS);
     ptx::tmem_relinquish();
   }
-  // The weights do not depend on the previous kernel of the stream: copy them in before the
-  // grid-dependency wait.  Piece (b, s) holds rows p < OUT of W[b], K values [16 s, 16 s + 16),
-  // 32B-swizzled K-major: chunk c of row n lands at n*32 + ((c ^ ((n >> 2) & 1)) << 4).
+  // Weights that are a caller input (R, L) do not depend on the previous kernel of the stream:
+  // they are copied in before the grid-dependency wait.  Weights made by an earlier kernel of
+  // the same call (the transposed factors) only after it.  Piece (b, s) holds rows p < OUT of
+  // W[b], K values [16 s, 16 s + 16), 32B-swizzled K-major: chunk c of row n lands at
+  // n*32 + ((c ^ ((n >> 2) & 1)) << 4).
+  if (!w_is_input) ptx::griddep_wait();
   {
     const uint32_t w_s = ptx::smem_u32(wsm);
     const int b_first = stage_group<C>() * C::RG * 16;  // first block of this CTA's group
@@ -282,8 +285,8 @@ __global__ void __launch_bounds__(kStageThreads, 1)
 }
 
 template <class C>
-static cudaError_t launch_stage(const void* A, const void* W, void* out, int64_t rows, int* status,
-                                cudaStream_t st, bool pdl) {
+static cudaError_t launch_stage(const void* A, const void* W, bool w_is_input, void* out, int64_t rows,
+                                int* status, cudaStream_t st, bool pdl) {
   if (rows == 0) return cudaSuccess;
   CUtensorMap mA, mO;
   if (!make_map_2d(&mA, A, C::N_IN, (uint64_t)rows, 64, C::BM, CU_TENSOR_MAP_SWIZZLE_128B))
@@ -304,7 +307,8 @@ static cudaError_t launch_stage(const void* A, const void* W, void* out, int64_t
   if (per < 1) per = 1;
   if (per > nunits) per = nunits;
   return launch_kernel(tc_stage_kernel<C>, dim3((unsigned)(per * C::NG)), dim3(kStageThreads), C::SMEM_BYTES, st,
-                       pdl, mA, mO, (const __nv_bfloat16*)W, (__nv_bfloat16*)out, rows, status);
+                       pdl, mA, mO, (const __nv_bfloat16*)W, (__nv_bfloat16*)out, rows, w_is_input ? 1 : 0,
+                       status);
 }
 
 // ---------------------------------------------------------------- shapes
@@ -329,16 +333,17 @@ bool tc_stage_fwd_supported(const Shape& s) { return is_sq64(s); }
 
 // One stage of a tc_stage_supported shape (see StageKind in common.cuh).
 cudaError_t tc_stage(const void* A, const void* W, void* out, StageKind k, const Shape& s, int* status,
-                     cudaStream_t st, bool pdl) {
+                     cudaStream_t st, bool pdl, bool w_early) {
+  const bool input = w_early;
   if (is_sq64(s)) {
     const bool ot = k == StageKind::R || k == StageKind::Lt || (k == StageKind::L && s.out_transpose == 1);
-    return ot ? launch_stage<Stage64T>(A, W, out, s.rows, status, st, pdl)
-              : launch_stage<Stage64N>(A, W, out, s.rows, status, st, pdl);
+    return ot ? launch_stage<Stage64T>(A, W, input, out, s.rows, status, st, pdl)
+              : launch_stage<Stage64N>(A, W, input, out, s.rows, status, st, pdl);
   }
   if (is_r768(s)) {
     switch (k) {
-      case StageKind::R: return launch_stage<StageR768>(A, W, out, s.rows, status, st, pdl);
-      case StageKind::Lt: return launch_stage<StageLt768>(A, W, out, s.rows, status, st, pdl);
+      case StageKind::R: return launch_stage<StageR768>(A, W, input, out, s.rows, status, st, pdl);
+      case StageKind::Lt: return launch_stage<StageLt768>(A, W, input, out, s.rows, status, st, pdl);
       default: return cudaErrorNotSupported;
     }
   }
@@ -349,9 +354,9 @@ cudaError_t tc_stage(const void* A, const void* W, void* out, StageKind k, const
 // tc_stage_fwd_supported shapes.
 cudaError_t tc_stage_fwd(const void* X, const void* R, const void* L, void* Y, void* Z, const Shape& s,
                          int* status, cudaStream_t st) {
-  cudaError_t e = tc_stage(X, R, Z, StageKind::R, s, status, st, false);
+  cudaError_t e = tc_stage(X, R, Z, StageKind::R, s, status, st, false, true);
   if (e != cudaSuccess) return e;
-  return tc_stage(Z, L, Y, StageKind::L, s, status, st, true);
+  return tc_stage(Z, L, Y, StageKind::L, s, status, st, true, true);
 }
 
 }  // namespace monarch
