@@ -242,11 +242,14 @@ def launches(shape: dict, dtype: str, pname: str) -> int:
     R = torch.zeros((shape["nb1"], shape["out1"], shape["in1"]), dtype=dt, device="cuda")
     L = torch.zeros((shape["nb2"], shape["out2"], shape["in2"]), dtype=dt, device="cuda")
     dY = torch.zeros((1, n_out), dtype=dt, device="cuda")
-    n0 = bdl.kernel_launches()
     if pname == "fwd":
-        bdl.fwd_ws(X, R, L, shape)
+        n0 = bdl.kernel_launches()
+        bdl.fwd_train(X, R, L, shape)
     else:
-        bdl.bwd(dY, X, R, L, shape)
+        _, saved = bdl.fwd_train(X, R, L, shape)
+        torch.cuda.synchronize()
+        n0 = bdl.kernel_launches()
+        bdl.bwd_saved(dY, X, R, L, shape, saved)
     torch.cuda.synchronize()
     return bdl.kernel_launches() - n0
 
@@ -284,11 +287,12 @@ def time_shape(name, dev, flush, peaks, reps=10, warmup=3, spin_cycles=2000000):
     ws = torch.empty(max(bdl.bwd_workspace_bytes(shape, rows, w["dtype"]), 256), dtype=torch.uint8,
                      device=dev)
     stream = torch.cuda.current_stream()
-    # the forward with caller scratch: the two-pass GEMM path where it applies, else monarch_fwd
-    fws = bdl.fwd_workspace_bytes(shape, rows, w["dtype"])
-    fwd_ws = torch.empty(fws, dtype=torch.uint8, device=dev) if fws else None
-    runs = {"fwd": lambda: bdl.fwd_ws(X, R, L, shape, Y=Y, workspace=fwd_ws),
-            "bwd": lambda: bdl.bwd(dY, X, R, L, shape, dX=dX, dR=dR, dL=dL, workspace=ws)}
+    # the training pair: the forward keeps the middle vector, the backward reuses it
+    sb = bdl.saved_bytes(shape, rows, w["dtype"])
+    saved = torch.empty(sb, dtype=torch.uint8, device=dev) if sb else None
+    bdl.fwd_train(X, R, L, shape, Y=Y, saved=saved)  # the backward timings read this saved buffer
+    runs = {"fwd": lambda: bdl.fwd_train(X, R, L, shape, Y=Y, saved=saved),
+            "bwd": lambda: bdl.bwd_saved(dY, X, R, L, shape, saved, dX=dX, dR=dR, dL=dL, workspace=ws)}
     alg = algorithmic(w, rows)
     hbm, tpk = peaks["hbm_gbs"] * 1e9, peaks["bf16_tflops"] * 1e12
     if w["dtype"] == "f32":
@@ -321,11 +325,11 @@ def time_shape(name, dev, flush, peaks, reps=10, warmup=3, spin_cycles=2000000):
                      ("fma" if w["dtype"] == "f32" else "tensor"),
             "launches": launches(shape, w["dtype"], pname),
             "host_enqueue_us": 1e6 * sum(host) / len(host),
-            "entry": "monarch_fwd_ws" if pname == "fwd" else "monarch_bwd",
+            "entry": "monarch_fwd_train" if pname == "fwd" else "monarch_bwd_saved",
         }
     if bdl.last_device_status() != 0:
         raise SystemExit("device status not OK after timing %s" % name)
-    del X, R, L, dY, Y, dX, dR, dL, ws, d, fwd_ws
+    del X, R, L, dY, Y, dX, dR, dL, ws, d, saved
     torch.cuda.empty_cache()
     return res
 
@@ -385,8 +389,9 @@ def main():
     dL = torch.empty_like(L)
     ws = torch.empty(max(bdl.bwd_workspace_bytes(shape, rows, w["dtype"]), 256), dtype=torch.uint8,
                      device=dev_)
-    fws_bytes = bdl.fwd_workspace_bytes(shape, rows, w["dtype"])
-    fws = torch.empty(fws_bytes, dtype=torch.uint8, device=dev_) if fws_bytes else None
+    sb = bdl.saved_bytes(shape, rows, w["dtype"])  # the forward's saved middle vector
+    saved = torch.empty(sb, dtype=torch.uint8, device=dev_) if sb else None
+    bdl.fwd_train(X, R, L, shape, Y=Y, saved=saved)  # a backward-only run reads this
     l2 = torch.cuda.get_device_properties(dev_).L2_cache_size
     flush = torch.empty(max(2 * l2, 256 << 20), dtype=torch.uint8, device=dev_)
     stream = torch.cuda.current_stream()
@@ -410,14 +415,14 @@ def main():
             torch.cuda._sleep(spin_cycles)
             ev[0].record(stream)
         if do_fwd:
-            bdl.fwd_ws(X, R, L, shape, Y=Y, workspace=fws)
+            bdl.fwd_train(X, R, L, shape, Y=Y, saved=saved)
         if ev is not None:
             ev[1].record(stream)
             flush.zero_()
             torch.cuda._sleep(spin_cycles)
             ev[2].record(stream)
         if do_bwd:
-            bdl.bwd(dY, X, R, L, shape, dX=dX, dR=dR, dL=dL, workspace=ws)
+            bdl.bwd_saved(dY, X, R, L, shape, saved, dX=dX, dR=dR, dL=dL, workspace=ws)
             allreduce_grads()
         if ev is not None:
             ev[3].record(stream)
@@ -482,8 +487,8 @@ def main():
             s_comp.wait_event(ev_in[b])
             s_comp.wait_event(ev_out[b])     # buffer set b's previous results are copied out
             y, dx, dr, dl = outs_d[b]
-            bdl.fwd_ws(Xe[b], R, L, shape, Y=y, workspace=fws)
-            bdl.bwd(dYe[b], Xe[b], R, L, shape, dX=dx, dR=dr, dL=dl, workspace=ws)
+            bdl.fwd_train(Xe[b], R, L, shape, Y=y, saved=saved)
+            bdl.bwd_saved(dYe[b], Xe[b], R, L, shape, saved, dX=dx, dR=dr, dL=dl, workspace=ws)
             if world > 1:
                 dp.allreduce_weight_grads(dr, dl)
             ev_comp[b].record(s_comp)
@@ -595,7 +600,8 @@ def main():
         "warmup": args.warmup, "ms_per_step": tot_ms / K, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": w["dtype"], "data": "synthetic",
         "config": {"workload": describe(name, w), "rows_per_gpu": rows,
-                   "step": "forward + backward (dX, dR, dL)" +
+                   "step": "forward keeping the middle vector (monarch_fwd_train) + backward reusing it "
+                           "(monarch_bwd_saved: dX, dR, dL)" +
                            (" + NCCL all-reduce of dR, dL" if world > 1 else ""),
                    "l2": "flushed before every timed pass (%d MiB write, untimed), then a "
                          "GPU-side spin so host launch latency is outside the timed pass"

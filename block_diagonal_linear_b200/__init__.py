@@ -45,6 +45,7 @@ EXPORTED = (
     "monarch_materialise", "monarch_status_string", "monarch_last_device_status",
     "monarch_debug_wait_timeout", "monarch_fwd_path", "monarch_bwd_path", "monarch_bwd_noalloc",
     "monarch_kernel_launches", "monarch_fwd_workspace_bytes", "monarch_fwd_ws_path", "monarch_fwd_ws",
+    "monarch_saved_bytes", "monarch_fwd_train", "monarch_bwd_saved",
     "monarch_linear_shape", "monarch_linear_workspace_bytes",
     "monarch_linear_fwd", "monarch_linear_bwd", "monarch_project", "monarch_dyad_workspace_bytes",
     "monarch_dyad_path", "monarch_dyad_fwd", "monarch_dyad_bwd", "monarch_lattice_workspace_bytes",
@@ -138,6 +139,12 @@ def lib() -> ctypes.CDLL:
         L.monarch_fwd_ws_path.restype = ctypes.c_int
         L.monarch_fwd_ws.argtypes = [vp, vp, vp, dp, vp, vp, ctypes.c_size_t, vp]
         L.monarch_fwd_ws.restype = ctypes.c_int
+        L.monarch_saved_bytes.argtypes = [dp]
+        L.monarch_saved_bytes.restype = ctypes.c_size_t
+        L.monarch_fwd_train.argtypes = [vp, vp, vp, dp, vp, vp, ctypes.c_size_t, vp]
+        L.monarch_fwd_train.restype = ctypes.c_int
+        L.monarch_bwd_saved.argtypes = [vp, vp, vp, vp, dp, vp, ctypes.c_size_t, vp, vp, vp, vp, ctypes.c_size_t, vp]
+        L.monarch_bwd_saved.restype = ctypes.c_int
         L.monarch_kernel_launches.argtypes = []
         L.monarch_kernel_launches.restype = ctypes.c_uint64
         lp = ctypes.POINTER(MonarchLinearDims)
@@ -306,6 +313,55 @@ def fwd_ws(X, R, L, shape: dict, Y=None, workspace=None, stream=None):
     _check("monarch_fwd_ws", lib().monarch_fwd_ws(_ptr(X), _ptr(R), _ptr(L), ctypes.byref(d), _ptr(Y),
                                                   _ptr(workspace), ctypes.c_size_t(nbytes), _stream(stream)))
     return Y
+
+
+def saved_bytes(shape: dict, rows: int, dtype="bf16") -> int:
+    """Bytes of the buffer monarch_fwd_train fills for monarch_bwd_saved (0: nothing is saved)."""
+    return int(lib().monarch_saved_bytes(ctypes.byref(make_dims(shape, rows, dtype))))
+
+
+def fwd_train(X, R, L, shape: dict, Y=None, saved=None, stream=None):
+    """Training forward (monarch_fwd_train): returns (Y, saved); pass `saved` to bwd_saved."""
+    import torch
+    code = dtype_code(X.dtype)
+    rows = X.shape[0]
+    _check_tensors(shape, rows, X.dtype, X=X, R=R, L=L, Y=Y)
+    if Y is None:
+        Y = torch.empty((rows, shape["nb2"] * shape["out2"]), dtype=X.dtype, device=X.device)
+    d = make_dims(shape, rows, code)
+    need = int(lib().monarch_saved_bytes(ctypes.byref(d)))
+    if saved is None and need > 0:
+        saved = torch.empty(need, dtype=torch.uint8, device=X.device)
+    _require_cuda(X, R, L, Y, saved)
+    nbytes = 0 if saved is None else saved.numel() * saved.element_size()
+    _check("monarch_fwd_train", lib().monarch_fwd_train(_ptr(X), _ptr(R), _ptr(L), ctypes.byref(d), _ptr(Y),
+                                                        _ptr(saved), ctypes.c_size_t(nbytes), _stream(stream)))
+    return Y, saved
+
+
+def bwd_saved(dY, X, R, L, shape: dict, saved, dX=None, dR=None, dL=None, workspace=None, stream=None):
+    """(dX, dR, dL) like bwd(), reusing the middle vector fwd_train saved (monarch_bwd_saved)."""
+    import torch
+    code = dtype_code(X.dtype)
+    rows = X.shape[0]
+    _check_tensors(shape, rows, X.dtype, dY=dY, X=X, R=R, L=L, dX=dX, dR=dR, dL=dL)
+    if dX is None:
+        dX = torch.empty_like(X)
+    if dR is None:
+        dR = torch.empty_like(R)
+    if dL is None:
+        dL = torch.empty_like(L)
+    d = make_dims(shape, rows, code)
+    need = int(lib().monarch_bwd_workspace_bytes(ctypes.byref(d)))
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=X.device)
+    _require_cuda(dY, X, R, L, dX, dR, dL, workspace, saved)
+    sbytes = 0 if saved is None else saved.numel() * saved.element_size()
+    _check("monarch_bwd_saved",
+           lib().monarch_bwd_saved(_ptr(dY), _ptr(X), _ptr(R), _ptr(L), ctypes.byref(d), _ptr(saved),
+                                   ctypes.c_size_t(sbytes), _ptr(dX), _ptr(dR), _ptr(dL), _ptr(workspace),
+                                   ctypes.c_size_t(workspace.numel() * workspace.element_size()), _stream(stream)))
+    return dX, dR, dL
 
 
 def bwd(dY, X, R, L, shape: dict, dX=None, dR=None, dL=None, workspace=None, stream=None):

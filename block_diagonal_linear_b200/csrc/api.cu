@@ -137,14 +137,14 @@ int fwd_dispatch(const void* X, const void* R, const void* L, void* Y, const Sha
 
 // Backward on already-checked arguments (workspace of bwd_workspace(s, dtype) bytes).
 int bwd_dispatch(const void* dY, const void* X, const void* R, const void* L, void* dX, void* dR, void* dL,
-                 void* ws, const Shape& s, int dtype, cudaStream_t st) {
+                 void* ws, const Shape& s, int dtype, cudaStream_t st, const void* saved) {
   cudaError_t e;
   const int path = bwd_path(s, dtype);
   if (path != 0) {
     int* status = status_ptr();
     if (status == nullptr) return MONARCH_ERR_CUDA;
-    e = path == 1   ? fast_bwd(dY, X, R, L, dX, dR, dL, ws, s, status, st)
-        : path == 2 ? gemm_bwd(dY, X, R, L, dX, dR, dL, ws, s, status, st)
+    e = path == 1   ? fast_bwd(dY, X, R, L, dX, dR, dL, ws, s, status, st, saved)
+        : path == 2 ? gemm_bwd(dY, X, R, L, dX, dR, dL, ws, s, status, st, saved)
                     : packed_bwd(dY, X, R, L, dX, dR, dL, ws, s, status, st);
   } else {
     if (!generic_bwd_supported(s)) return MONARCH_ERR_UNSUPPORTED;
@@ -238,6 +238,82 @@ int monarch_fwd_ws(const void* X, const void* R, const void* L, const monarch_di
                             ? gemm_fwd(X, R, L, Y, workspace, s, status, (cudaStream_t)stream)
                             : tc_stage_fwd(X, R, L, Y, workspace, s, status, (cudaStream_t)stream);
   return e == cudaSuccess ? MONARCH_OK : MONARCH_ERR_CUDA;
+}
+
+// What the training forward leaves for the backward: 2 = Z from the fused row-tile forward,
+// 5 = the two-pass GEMM forward's workspace (U), 6 = the streaming stages' Z; 0 = nothing (the
+// backward recomputes the middle vector).
+static int saved_kind(const Shape& s, int dtype) {
+  if (dtype != MONARCH_BF16) return 0;
+  const int k = fwd_ws_kind(s, dtype);
+  if (k == 5 || k == 6) return k;
+  if (fwd_path(s, dtype) == 2 && bwd_path(s, dtype) == 1) return 2;
+  return 0;
+}
+
+static size_t saved_bytes(const Shape& s, int dtype) {
+  switch (saved_kind(s, dtype)) {
+    case 2:
+    case 6: return (size_t)s.rows * (size_t)s.n_mid() * 2;
+    case 5: return gemm_fwd_workspace(s);
+    default: return 0;
+  }
+}
+
+size_t monarch_saved_bytes(const monarch_dims* d) {
+  if (check_dims(d) != MONARCH_OK) return 0;
+  return saved_bytes(to_shape(*d), d->dtype);
+}
+
+int monarch_fwd_train(const void* X, const void* R, const void* L, const monarch_dims* d, void* Y, void* saved,
+                      size_t saved_bytes_, void* stream) {
+  int rc = check_dims(d);
+  if (rc != MONARCH_OK) return rc;
+  if (d->rows == 0) return MONARCH_OK;
+  if ((rc = check_ptrs({X, R, L, Y})) != MONARCH_OK) return rc;
+  const Shape s = to_shape(*d);
+  const size_t need = saved_bytes(s, d->dtype);
+  if (need > 0 && (saved == nullptr || saved_bytes_ < need)) return MONARCH_ERR_WORKSPACE;
+  if (need > 0 && ((uintptr_t)saved & 255u) != 0) return MONARCH_ERR_ALIGN;
+  const int64_t es = d->dtype == MONARCH_BF16 ? 2 : 4;
+  if ((rc = check_alias({span(Y, s.rows * s.n_out(), es), span(saved, (int64_t)need, 1)},
+                        {span(X, s.rows * s.n_in(), es), span(R, s.n_R(), es), span(L, s.n_L(), es)})) !=
+      MONARCH_OK)
+    return rc;
+  const cudaStream_t st = (cudaStream_t)stream;
+  const int kind = saved_kind(s, d->dtype);
+  if (kind == 0) return fwd_dispatch(X, R, L, Y, s, d->dtype, st);
+  int* status = status_ptr();
+  if (status == nullptr) return MONARCH_ERR_CUDA;
+  const cudaError_t e = kind == 2   ? tc_rows_fwd_save(X, R, L, Y, saved, s, status, st)
+                        : kind == 5 ? gemm_fwd(X, R, L, Y, saved, s, status, st)
+                                    : tc_stage_fwd(X, R, L, Y, saved, s, status, st);
+  return e == cudaSuccess ? MONARCH_OK : MONARCH_ERR_CUDA;
+}
+
+int monarch_bwd_saved(const void* dY, const void* X, const void* R, const void* L, const monarch_dims* d,
+                      const void* saved, size_t saved_bytes_, void* dX, void* dR, void* dL, void* workspace,
+                      size_t workspace_bytes, void* stream) {
+  int rc = check_dims(d);
+  if (rc != MONARCH_OK) return rc;
+  if ((rc = check_ptrs({R, L, dR, dL})) != MONARCH_OK) return rc;
+  if (d->rows > 0 && (rc = check_ptrs({dY, X, dX})) != MONARCH_OK) return rc;
+  const Shape s = to_shape(*d);
+  const size_t need_saved = saved_bytes(s, d->dtype);
+  if (need_saved > 0 && (saved == nullptr || saved_bytes_ < need_saved)) return MONARCH_ERR_WORKSPACE;
+  if (need_saved > 0 && ((uintptr_t)saved & 255u) != 0) return MONARCH_ERR_ALIGN;
+  const size_t need = bwd_workspace(s, d->dtype);
+  if (workspace == nullptr || workspace_bytes < need) return MONARCH_ERR_WORKSPACE;
+  if (((uintptr_t)workspace & 255u) != 0) return MONARCH_ERR_ALIGN;
+  const int64_t es = d->dtype == MONARCH_BF16 ? 2 : 4;
+  if ((rc = check_alias({span(dX, s.rows * s.n_in(), es), span(dR, s.n_R(), es), span(dL, s.n_L(), es),
+                         span(workspace, (int64_t)need, 1)},
+                        {span(dY, s.rows * s.n_out(), es), span(X, s.rows * s.n_in(), es),
+                         span(R, s.n_R(), es), span(L, s.n_L(), es), span(saved, (int64_t)need_saved, 1)})) !=
+      MONARCH_OK)
+    return rc;
+  return bwd_dispatch(dY, X, R, L, dX, dR, dL, workspace, s, d->dtype, (cudaStream_t)stream,
+                      need_saved > 0 ? saved : nullptr);
 }
 
 size_t monarch_bwd_workspace_bytes(const monarch_dims* d) {

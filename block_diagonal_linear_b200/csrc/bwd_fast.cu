@@ -120,7 +120,7 @@ static FastWs fast_layout(const Shape& s) {
 size_t fast_bwd_workspace(const Shape& s) { return fast_layout(s).total; }
 
 cudaError_t fast_bwd(const void* dY, const void* X, const void* R, const void* L, void* dX, void* dR,
-                     void* dL, void* ws, const Shape& s, int* status, cudaStream_t st) {
+                     void* dL, void* ws, const Shape& s, int* status, cudaStream_t st, const void* saved) {
   const FastWs w = fast_layout(s);
   char* base = (char*)ws;
   __nv_bfloat16* Rt = (__nv_bfloat16*)(base + w.rt);
@@ -138,20 +138,31 @@ cudaError_t fast_bwd(const void* dY, const void* X, const void* R, const void* L
   const WgradSplit sp = wg_split(s);
   const bool split = is_split_square(s);
   if (split && !s.out_transpose) dV = (__nv_bfloat16*)dY;  // dV[j][o] = dy[j*out2 + o]: no copy
+  if (saved != nullptr) Z = (__nv_bfloat16*)saved;  // the training forward's Z: no recompute
   if (s.rows > 0 && split) {
     // dV = P_out^-1 dY;  Z = P (blockdiag(R) X);  dZ = blockdiag(L^T) dV;  dU = P^-1 dZ;
     // dX = blockdiag(R^T) dU.  Z and dZ/dU are permuted in place.
-    if (s.out_transpose && (e = permute_rows(dY, dV, s.rows, s.out2, s.nb2, st)) != cudaSuccess) return e;
+    bool prev = false;  // a kernel of this call precedes (the transposes may then overlap it)
+    if (s.out_transpose) {
+      if ((e = permute_rows(dY, dV, s.rows, s.out2, s.nb2, st)) != cudaSuccess) return e;
+      prev = true;
+    }
     if (tc_stage_supported(s)) {
       // the permutations folded into the stages that produce Z and dU (tc_stage.cu)
-      if ((e = tc_stage(X, R, Z, StageKind::R, s, status, st, true, true)) != cudaSuccess) return e;
-      if ((e = factor_transposes(R, Rt, L, Lt, s, 0, st, true)) != cudaSuccess) return e;
+      if (saved == nullptr) {
+        if ((e = tc_stage(X, R, Z, StageKind::R, s, status, st, true, true)) != cudaSuccess) return e;
+        prev = true;
+      }
+      if ((e = factor_transposes(R, Rt, L, Lt, s, 0, st, prev)) != cudaSuccess) return e;
       // Lt comes from the launch just before: read it after the wait
       if ((e = tc_stage(dV, Lt, dU, StageKind::Lt, s, status, st, true, false)) != cudaSuccess) return e;
     } else {
-      if ((e = bdgemm64(X, R, Z, s.nb1, s.rows, status, st, true)) != cudaSuccess) return e;
-      if ((e = permute_rows(Z, Z, s.rows, s.nb1, s.out1, st)) != cudaSuccess) return e;
-      if ((e = factor_transposes(R, Rt, L, Lt, s, 0, st, true)) != cudaSuccess) return e;
+      if (saved == nullptr) {
+        if ((e = bdgemm64(X, R, Z, s.nb1, s.rows, status, st, true)) != cudaSuccess) return e;
+        if ((e = permute_rows(Z, Z, s.rows, s.nb1, s.out1, st)) != cudaSuccess) return e;
+        prev = true;
+      }
+      if ((e = factor_transposes(R, Rt, L, Lt, s, 0, st, prev)) != cudaSuccess) return e;
       if ((e = bdgemm64(dV, Lt, dU, s.nb2, s.rows, status, st, true)) != cudaSuccess) return e;
       if ((e = permute_rows(dU, dU, s.rows, s.out1, s.nb1, st)) != cudaSuccess) return e;
     }
@@ -161,7 +172,7 @@ cudaError_t fast_bwd(const void* dY, const void* X, const void* R, const void* L
     if ((e = launch_kernel(gather_dv_kernel, dim3(2 * 148), dim3(kGatherWarps * 32), gsm, st, true,
                            (const __nv_bfloat16*)dY, dV, s)) != cudaSuccess)
       return e;
-    if ((e = tc_rows_middle(X, R, Z, s, status, st)) != cudaSuccess) return e;
+    if (saved == nullptr && (e = tc_rows_middle(X, R, Z, s, status, st)) != cudaSuccess) return e;
     if ((e = factor_transposes(R, Rt, L, Lt, s, 0, st, true)) != cudaSuccess) return e;
     if ((e = tc_rows_dual(dV, Lt, Rt, dX, dU, s, status, st)) != cudaSuccess) return e;
   }

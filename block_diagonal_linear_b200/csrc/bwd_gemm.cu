@@ -312,7 +312,7 @@ static GemmBwdWs gemm_bwd_layout(const Shape& s) {
 size_t gemm_bwd_workspace(const Shape& s) { return gemm_bwd_layout(s).total; }
 
 cudaError_t gemm_bwd(const void* dY, const void* X, const void* R, const void* L, void* dX, void* dR, void* dL,
-                     void* ws, const Shape& s, int* status, cudaStream_t st) {
+                     void* ws, const Shape& s, int* status, cudaStream_t st, const void* saved) {
   const GemmBwdWs w = gemm_bwd_layout(s);
   char* base = (char*)ws;
   __nv_bfloat16* Rt = (__nv_bfloat16*)(base + w.rt);
@@ -324,18 +324,25 @@ cudaError_t gemm_bwd(const void* dY, const void* X, const void* R, const void* L
   const int G = s.in2 / s.nb1;
   cudaError_t e;
   if (s.rows > 0) {
-    // 2. U = blockdiag(R) X
     GemmJob j = {};
-    int bn = pick_bn(s.out1);
-    j.nb = s.nb1; j.ntiles = s.out1 / bn; j.kboxes = s.in1 / 64;
-    j.a_b = s.in1; j.a_grp = s.in1 / 64; j.a_gs = 0;
-    j.b_b = s.out1;
-    j.y_b = s.out1; j.y_grp = s.out1 / 64; j.y_gs = 0;
-    if ((e = gemm_bd(X, s.rows, s.n_in(), R, (int64_t)s.nb1 * s.out1, s.in1, U, s.n_mid(), bn, j, status, st,
-                     true)) != cudaSuccess)
-      return e;
-    // 1. the factor prep overlaps the U pass (which reads neither Rt nor Ltp)
-    if ((e = factor_transposes(R, Rt, L, Ltp, s, G, st, true)) != cudaSuccess) return e;
+    int bn;
+    if (saved != nullptr) {
+      // U from the training forward's workspace: no recompute, and the prep is the first launch
+      U = (__nv_bfloat16*)((const char*)saved + gemm_fwd_u_offset(s));
+      if ((e = factor_transposes(R, Rt, L, Ltp, s, G, st, false)) != cudaSuccess) return e;
+    } else {
+      // 2. U = blockdiag(R) X
+      bn = pick_bn(s.out1);
+      j.nb = s.nb1; j.ntiles = s.out1 / bn; j.kboxes = s.in1 / 64;
+      j.a_b = s.in1; j.a_grp = s.in1 / 64; j.a_gs = 0;
+      j.b_b = s.out1;
+      j.y_b = s.out1; j.y_grp = s.out1 / 64; j.y_gs = 0;
+      if ((e = gemm_bd(X, s.rows, s.n_in(), R, (int64_t)s.nb1 * s.out1, s.in1, U, s.n_mid(), bn, j, status, st,
+                       true)) != cudaSuccess)
+        return e;
+      // 1. the factor prep overlaps the U pass (which reads neither Rt nor Ltp)
+      if ((e = factor_transposes(R, Rt, L, Ltp, s, G, st, true)) != cudaSuccess) return e;
+    }
     // 3. dU = blockdiag(Ltp) dY, output group g of block j -> u[k][j*G + 64*(g % (G/64))], k = g / (G/64)
     j = GemmJob{};
     bn = pick_bn(s.in2);
@@ -378,6 +385,8 @@ cudaError_t gemm_bwd(const void* dY, const void* X, const void* R, const void* L
 //   2. U  = blockdiag(R) X                    (GEMM, block-contiguous u[k][p])
 //   3. Y  = blockdiag(Lp) gathered(U)          (GEMM; block j's K stage kb reads the 64 columns
 //                                             of U at k*out1 + j*G + 64*(kb % (G/64)))
+size_t gemm_fwd_u_offset(const Shape& s) { return al256((size_t)s.n_L() * 2); }
+
 size_t gemm_fwd_workspace(const Shape& s) {
   return al256((size_t)s.n_L() * 2) + al256((size_t)s.rows * (size_t)s.n_mid() * 2);
 }

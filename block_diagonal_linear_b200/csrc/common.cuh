@@ -119,6 +119,8 @@ cudaError_t tc_fwd(const void* X, const void* R, const void* L, void* Y, const S
 
 // tcgen05 fused forward with 64-row tiles and the whole middle vector on chip (small blocks).
 bool tc_rows_supported(const Shape& s);
+cudaError_t tc_rows_fwd_save(const void* X, const void* R, const void* L, void* Y, void* Z, const Shape& s,
+                             int* status, cudaStream_t st);
 cudaError_t tc_rows_fwd(const void* X, const void* R, const void* L, void* Y, const Shape& s,
                         int* status, cudaStream_t st);
 
@@ -156,8 +158,10 @@ cudaError_t permute_rows_add(const void* src, void* dst, int64_t rows, int A, in
 // Tensor-core backward of the square small-block shapes (bf16).
 bool fast_bwd_supported(const Shape& s);
 size_t fast_bwd_workspace(const Shape& s);
+// saved: the middle vector Z of this call's rows as the training forward left it (nullptr: recompute)
 cudaError_t fast_bwd(const void* dY, const void* X, const void* R, const void* L, void* dX, void* dR,
-                     void* dL, void* ws, const Shape& s, int* status, cudaStream_t st);
+                     void* dL, void* ws, const Shape& s, int* status, cudaStream_t st,
+                     const void* saved = nullptr);
 
 cudaError_t debug_wait_timeout(uint64_t timeout_ns, int* status, cudaStream_t st);
 
@@ -167,7 +171,7 @@ int bwd_path(const Shape& s, int dtype);
 size_t bwd_workspace(const Shape& s, int dtype);
 int fwd_dispatch(const void* X, const void* R, const void* L, void* Y, const Shape& s, int dtype, cudaStream_t st);
 int bwd_dispatch(const void* dY, const void* X, const void* R, const void* L, void* dX, void* dR, void* dL,
-                 void* ws, const Shape& s, int dtype, cudaStream_t st);
+                 void* ws, const Shape& s, int dtype, cudaStream_t st, const void* saved = nullptr);
 int* status_ptr();
 bool aligned16(const void* p);
 

@@ -86,7 +86,10 @@ cudaError_t gemm_fwd(const void* X, const void* R, const void* L, void* Y, void*
 
 bool gemm_bwd_supported(const Shape& s);
 size_t gemm_bwd_workspace(const Shape& s);
+// saved: the workspace of the two-pass forward of the same rows (its U is reused; nullptr: recompute U)
 cudaError_t gemm_bwd(const void* dY, const void* X, const void* R, const void* L, void* dX, void* dR, void* dL,
-                     void* ws, const Shape& s, int* status, cudaStream_t st);
+                     void* ws, const Shape& s, int* status, cudaStream_t st, const void* saved = nullptr);
+// Offset of U in the two-pass forward's workspace.
+size_t gemm_fwd_u_offset(const Shape& s);
 
 }  // namespace monarch

@@ -466,6 +466,9 @@ using RowsSq32 = RowsCfg<32, 32, 32, 32, 32, 32, 1>;  // n = 1024 = 32^2
 // transposed factors and no output transpose; MODE 1 also stores dU.
 using RowsSq16Bwd = RowsCfg<16, 16, 16, 16, 16, 16, 0, 1>;
 using RowsSq32Bwd = RowsCfg<32, 32, 32, 32, 32, 32, 0, 1>;
+// Training forward: Y, and the middle tile Z (block-contiguous by L block) stored for the backward.
+using RowsSq16Save = RowsCfg<16, 16, 16, 16, 16, 16, 1, 1>;
+using RowsSq32Save = RowsCfg<32, 32, 32, 32, 32, 32, 1, 1>;
 // R stage and permutation only (Z = P R x), for the weight gradient of L.
 using RowsSq16Z = RowsCfg<16, 16, 16, 16, 16, 16, 1, 2>;
 using RowsSq32Z = RowsCfg<32, 32, 32, 32, 32, 32, 1, 2>;
@@ -484,6 +487,14 @@ cudaError_t tc_rows_fwd(const void* X, const void* R, const void* L, void* Y, co
                         int* status, cudaStream_t st) {
   if (rows_shape_is<RowsSq16>(s)) return launch_rows<RowsSq16>(X, R, L, Y, nullptr, s.rows, status, st);
   if (rows_shape_is<RowsSq32>(s)) return launch_rows<RowsSq32>(X, R, L, Y, nullptr, s.rows, status, st);
+  return cudaErrorNotSupported;
+}
+
+// Y = X M^T and, on the side, Z = P R x (what the middle-only pass of the backward computes).
+cudaError_t tc_rows_fwd_save(const void* X, const void* R, const void* L, void* Y, void* Z, const Shape& s,
+                             int* status, cudaStream_t st) {
+  if (rows_shape_is<RowsSq16>(s)) return launch_rows<RowsSq16Save>(X, R, L, Y, Z, s.rows, status, st);
+  if (rows_shape_is<RowsSq32>(s)) return launch_rows<RowsSq32Save>(X, R, L, Y, Z, s.rows, status, st);
   return cudaErrorNotSupported;
 }
 

@@ -120,6 +120,35 @@ MONARCH_API int monarch_fwd_ws_path(const monarch_dims* d);
 MONARCH_API int monarch_fwd_ws(const void* X, const void* R, const void* L, const monarch_dims* d, void* Y,
                                void* workspace, size_t workspace_bytes, void* stream);
 
+/* Training pair: a forward that keeps what its backward needs, and that backward.
+ *
+ * monarch_fwd_train computes Y = X * M^T exactly as monarch_fwd_ws does (same kernels, same
+ * results) and leaves the middle vector of these rows in `saved`, in the layout the backward's
+ * own recompute would produce: for the fused small-block forward (monarch_fwd_path 2) and the
+ * streaming-stage forward (monarch_fwd_ws_path 6) the permuted middle vector Z (rows x n_mid
+ * bf16, Z[r][j*in2 + q]); for the two-pass GEMM forward (monarch_fwd_ws_path 5) that
+ * forward's whole workspace (the reordered L, then U = blockdiag(R) X).  This is what an
+ * autograd framework saves for the backward of a product of factors; it trades a write and a
+ * read of rows x n_mid bf16 for the backward's recompute pass (a read of X, a write of the
+ * middle vector, and its flops).
+ *
+ * monarch_bwd_saved computes the same dX, dR, dL as monarch_bwd (bit for bit: the saved middle
+ * vector equals the recomputed one) from dY, X, R, L and that `saved` buffer, skipping the
+ * recompute.  For shapes and dtypes with nothing to save monarch_saved_bytes returns 0, `saved`
+ * may be NULL, monarch_fwd_train runs monarch_fwd and monarch_bwd_saved runs monarch_bwd.
+ *
+ * saved: >= monarch_saved_bytes(d) bytes, 256-byte aligned, caller-owned; written by
+ * monarch_fwd_train, read by monarch_bwd_saved with the same dims and the same X, R, L, and
+ * not modified in between.  It must not overlap the other arguments.  workspace (backward):
+ * >= monarch_bwd_workspace_bytes(d) bytes, as for monarch_bwd.  Errors as for monarch_fwd_ws
+ * and monarch_bwd (MONARCH_ERR_WORKSPACE for a missing or short `saved`). */
+MONARCH_API size_t monarch_saved_bytes(const monarch_dims* d);
+MONARCH_API int monarch_fwd_train(const void* X, const void* R, const void* L, const monarch_dims* d, void* Y,
+                                  void* saved, size_t saved_bytes, void* stream);
+MONARCH_API int monarch_bwd_saved(const void* dY, const void* X, const void* R, const void* L,
+                                  const monarch_dims* d, const void* saved, size_t saved_bytes, void* dX,
+                                  void* dR, void* dL, void* workspace, size_t workspace_bytes, void* stream);
+
 /* Backward of Y = X * M^T for a loss with gradient dY (chain rule; the middle
  * vector is recomputed from X rather than stored):
  *   dV[j][o] = dY[idx(j,o)],  dL[j][o][q] = sum_rows dV[j][o] * Z[j][q],

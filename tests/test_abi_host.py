@@ -83,6 +83,41 @@ def test_bwd_workspace_checks_before_device_work():
     assert bdl.bwd_workspace_bytes(dict(shape, out1=5), 10, "bf16") == 0
 
 
+def test_training_pair_sizes_and_checks_before_device_work():
+    """monarch_saved_bytes per forward family, and the training pair's argument checks (fake
+    device pointers: every call must fail before any device work)."""
+    W = synthetic.WORKLOADS
+    n1024, n4096 = synthetic.shape_of(W["n1024_bf16"]), synthetic.shape_of(W["n4096_bf16"])
+    nblk4, r768 = synthetic.shape_of(W["nblk4_1024x4096_bf16"]), synthetic.shape_of(W["r768x3072_bf16"])
+    assert bdl.saved_bytes(n1024, 100, "bf16") == 100 * 1024 * 2  # Z of the fused forward
+    assert bdl.saved_bytes(n4096, 100, "bf16") == 100 * 4096 * 2  # Z of the streaming stages
+    assert bdl.saved_bytes(nblk4, 100, "bf16") == bdl.fwd_workspace_bytes(nblk4, 100, "bf16")  # L reordered, U
+    assert bdl.saved_bytes(r768, 100, "bf16") == 0                # the backward recomputes
+    assert bdl.saved_bytes(n1024, 100, "f32") == 0
+    lib = bdl.lib()
+    d = bdl.make_dims(n1024, 1000, "bf16")
+    need = bdl.saved_bytes(n1024, 1000, "bf16")
+    p, sz = ctypes.c_void_p(1 << 40), ctypes.c_size_t
+    assert lib.monarch_fwd_train(p, p, p, ctypes.byref(d), p, None, sz(need), None) == \
+        bdl.CODES["MONARCH_ERR_WORKSPACE"]
+    assert lib.monarch_fwd_train(p, p, p, ctypes.byref(d), p, p, sz(need - 1), None) == \
+        bdl.CODES["MONARCH_ERR_WORKSPACE"]
+    assert lib.monarch_fwd_train(p, p, p, ctypes.byref(d), p, ctypes.c_void_p((1 << 40) + 16), sz(need), None) == \
+        bdl.CODES["MONARCH_ERR_ALIGN"]
+    # saved overlapping X
+    assert lib.monarch_fwd_train(p, ctypes.c_void_p(1 << 41), ctypes.c_void_p(1 << 42), ctypes.byref(d),
+                                 ctypes.c_void_p(1 << 43), p, sz(need), None) == bdl.CODES["MONARCH_ERR_ALIAS"]
+    wneed = bdl.bwd_workspace_bytes(n1024, 1000, "bf16")
+    q = [ctypes.c_void_p(k << 36) for k in range(1, 10)]
+    assert lib.monarch_bwd_saved(q[0], q[1], q[2], q[3], ctypes.byref(d), None, sz(need), q[4], q[5], q[6], q[7],
+                                 sz(wneed), None) == bdl.CODES["MONARCH_ERR_WORKSPACE"]
+    assert lib.monarch_bwd_saved(q[0], q[1], q[2], q[3], ctypes.byref(d), q[8], sz(need), q[4], q[5], q[6], q[7],
+                                 sz(wneed - 1), None) == bdl.CODES["MONARCH_ERR_WORKSPACE"]
+    # an output (dX) overlapping the saved buffer
+    assert lib.monarch_bwd_saved(q[0], q[1], q[2], q[3], ctypes.byref(d), q[8], sz(need), q[8], q[5], q[6], q[7],
+                                 sz(wneed), None) == bdl.CODES["MONARCH_ERR_ALIAS"]
+
+
 def test_kernel_family_selection():
     W = synthetic.WORKLOADS
     assert bdl.fwd_path(synthetic.shape_of(W["n1024_bf16"]), "bf16") == 2

@@ -117,3 +117,27 @@ def test_forward_with_workspace_exact(case):
     got = _host(Y)
     bad = np.argwhere(got != ref)
     assert bad.size == 0, "%d entries differ, first at %s" % (len(bad), tuple(bad[0]))
+
+
+TRAIN_CASES = [c for c in CASES if c[0] in ("sq16_rows", "n1024_rows", "n4096_split", "nblk4_group", "nblk2_gemm",
+                                          "r768x3072_wide")]
+
+
+@pytest.mark.parametrize("case", TRAIN_CASES, ids=_ids)
+def test_training_pair_exact(case):
+    """monarch_fwd_train + monarch_bwd_saved: Y, dX, dR, dL equal the oracle entry by entry, with
+    the middle vector taken from the forward (or recomputed where nothing is saved: 768 -> 3072)."""
+    name, shape, dtype, rows, _, _ = case
+    inp = synthetic.make_sparse_sign_inputs(dict(shape, rows=rows), seed=24)
+    _check_exact_range(inp)
+    X, R, L, dY = (_to_dev(inp[k], dtype) for k in ("X", "R", "L", "dY"))
+    Y, saved = bdl.fwd_train(X, R, L, shape)
+    assert (saved is None) == (name == "r768x3072_wide")
+    got = bdl.bwd_saved(dY, X, R, L, shape, saved)
+    assert bdl.last_device_status() == 0
+    refs = (oracle.forward(shape, inp["X"], inp["R"], inp["L"]),) + \
+        tuple(oracle.backward(shape, inp["dY"], inp["X"], inp["R"], inp["L"]))
+    for g, r, what in zip((Y,) + tuple(got), refs, ("Y", "dX", "dR", "dL")):
+        g = _host(g)
+        bad = np.argwhere(g != r)
+        assert bad.size == 0, "%s: %d entries differ, first at %s" % (what, len(bad), tuple(bad[0]))

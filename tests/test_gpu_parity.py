@@ -250,3 +250,22 @@ def test_stage_forward_tile_edges(name, rows):
     assert bdl.last_device_status() == 0
     ref = oracle.forward(shape, inp["X"].f64, inp["R"].f64, inp["L"].f64)
     check(to_f64(Y), ref, "bf16", "Y")
+
+
+@pytest.mark.parametrize("name", ["n1024_bf16", "n4096_bf16", "nblk4_1024x4096_bf16"])
+def test_training_pair_matches_forward_and_backward_bitwise(name):
+    """Full workload size: the training forward's Y equals monarch_fwd_ws's and the saved backward's
+    dX, dR, dL equal monarch_bwd's bit for bit (the saved middle vector is the recomputed one)."""
+    w = W[name]
+    shape = synthetic.shape_of(w)
+    inp = synthetic.make_inputs(w, seed=14)
+    d = dev_inputs(inp)
+    assert bdl.saved_bytes(shape, w["rows"], "bf16") > 0
+    Y1 = bdl.fwd_ws(d["X"], d["R"], d["L"], shape)
+    Y2, saved = bdl.fwd_train(d["X"], d["R"], d["L"], shape)
+    g1 = bdl.bwd(d["dY"], d["X"], d["R"], d["L"], shape)
+    g2 = bdl.bwd_saved(d["dY"], d["X"], d["R"], d["L"], shape, saved)
+    assert bdl.last_device_status() == 0
+    assert torch.equal(Y1, Y2)
+    for a, b, what in zip(g1, g2, ("dX", "dR", "dL")):
+        assert torch.equal(a, b), what
