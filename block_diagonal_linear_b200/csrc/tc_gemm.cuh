@@ -33,6 +33,8 @@ struct GemmJob {
   int64_t blk_a, blk_b;       // kind 1: block widths (M side, N side, before gathering)
   int64_t p_stride, p_off;    // kind 1: partial layout
   int64_t units;
+  int ab3d;                   // kind 1: A and B maps are 3-D (64 columns, rows, 64-column chunks)
+                              // and a stage fetches each operand with one multi-chunk box
 };
 
 __host__ __device__ __forceinline__ int gcol(int b, int base, int g, int grp, int gs) {
