@@ -11,7 +11,9 @@ data-parallel training.
 
 Inputs are seeded synthetic tensors with the workload's shapes and value
 distributions.  Timing: CUDA events on the launching stream around each pass;
-L2 is flushed (256 MiB write, untimed) before every timed pass; max over ranks.
+L2 is flushed before every timed pass (untimed): a 256 MiB write, then a read of the same
+buffer, so the pass starts with no useful line in L2 and without the flush's dirty lines to
+write back; max over ranks.
 Rank 0 prints one JSON line.
 """
 from __future__ import annotations
@@ -272,6 +274,25 @@ def device_inputs(w, seed, dev):
     return out
 
 
+class L2Flush:
+    """Untimed L2 flush before a timed pass: write a buffer of at least twice the L2 size, then
+    read it back.  The write evicts every line a pass could reuse; the read evicts the flush's
+    own dirty lines (their write-back happens here, not inside the timed pass)."""
+
+    def __init__(self, dev):
+        import torch
+        l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+        self.buf = torch.empty(max(2 * l2, 256 << 20), dtype=torch.uint8, device=dev)
+
+    def __call__(self):
+        import torch
+        self.buf.zero_()
+        torch.amax(self.buf.view(torch.int32))
+
+    def mib(self):
+        return self.buf.numel() >> 20
+
+
 def time_shape(name, dev, flush, peaks, reps=10, warmup=3, spin_cycles=2000000):
     """Forward and backward of one workload, each pass timed alone with CUDA events on the
     launching stream after an untimed L2 flush and GPU-side spin; averages over `reps`."""
@@ -303,7 +324,7 @@ def time_shape(name, dev, flush, peaks, reps=10, warmup=3, spin_cycles=2000000):
         evs, host = [], []
         for i in range(warmup + reps):
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            flush.zero_()
+            flush()
             torch.cuda._sleep(spin_cycles)
             e0.record(stream)
             h0 = time.perf_counter()
@@ -392,8 +413,7 @@ def main():
     sb = bdl.saved_bytes(shape, rows, w["dtype"])  # the forward's saved middle vector
     saved = torch.empty(sb, dtype=torch.uint8, device=dev_) if sb else None
     bdl.fwd_train(X, R, L, shape, Y=Y, saved=saved)  # a backward-only run reads this
-    l2 = torch.cuda.get_device_properties(dev_).L2_cache_size
-    flush = torch.empty(max(2 * l2, 256 << 20), dtype=torch.uint8, device=dev_)
+    flush = L2Flush(dev_)
     stream = torch.cuda.current_stream()
 
     from block_diagonal_linear_b200 import dp
@@ -411,14 +431,14 @@ def main():
 
     def step(ev=None):
         if ev is not None:
-            flush.zero_()
+            flush()
             torch.cuda._sleep(spin_cycles)
             ev[0].record(stream)
         if do_fwd:
             bdl.fwd_train(X, R, L, shape, Y=Y, saved=saved)
         if ev is not None:
             ev[1].record(stream)
-            flush.zero_()
+            flush()
             torch.cuda._sleep(spin_cycles)
             ev[2].record(stream)
         if do_bwd:
@@ -603,9 +623,10 @@ def main():
                    "step": "forward keeping the middle vector (monarch_fwd_train) + backward reusing it "
                            "(monarch_bwd_saved: dX, dR, dL)" +
                            (" + NCCL all-reduce of dR, dL" if world > 1 else ""),
-                   "l2": "flushed before every timed pass (%d MiB write, untimed), then a "
-                         "GPU-side spin so host launch latency is outside the timed pass"
-                         % (flush.numel() >> 20),
+                   "l2": "flushed before every timed pass (untimed: %d MiB write, then a read of "
+                         "the same buffer so no dirty flush line is written back inside the pass), "
+                         "then a GPU-side spin so host launch latency is outside the timed pass"
+                         % flush.mib(),
                    "parallelism": "dp%d" % world, "timed": args.only},
         "tflops": (alg["fwd"]["flops"] + alg["bwd"]["flops"]) * world * K / (tot_ms / 1e3) / 1e12,
         "passes": passes,

@@ -145,7 +145,7 @@ int bwd_dispatch(const void* dY, const void* X, const void* R, const void* L, vo
     if (status == nullptr) return MONARCH_ERR_CUDA;
     e = path == 1   ? fast_bwd(dY, X, R, L, dX, dR, dL, ws, s, status, st, saved)
         : path == 2 ? gemm_bwd(dY, X, R, L, dX, dR, dL, ws, s, status, st, saved)
-                    : packed_bwd(dY, X, R, L, dX, dR, dL, ws, s, status, st);
+                    : packed_bwd(dY, X, R, L, dX, dR, dL, ws, s, status, st, saved);
   } else {
     if (!generic_bwd_supported(s)) return MONARCH_ERR_UNSUPPORTED;
     e = generic_bwd(dY, X, R, L, dX, dR, dL, ws, s, dtype, st);
@@ -241,19 +241,22 @@ int monarch_fwd_ws(const void* X, const void* R, const void* L, const monarch_di
 }
 
 // What the training forward leaves for the backward: 2 = Z from the fused row-tile forward,
-// 5 = the two-pass GEMM forward's workspace (U), 6 = the streaming stages' Z; 0 = nothing (the
-// backward recomputes the middle vector).
+// 3 = Z from the wide-output forward (for the packed backward's streaming stages), 5 = the
+// two-pass GEMM forward's workspace (U), 6 = the streaming stages' Z; 0 = nothing (the backward
+// recomputes the middle vector).
 static int saved_kind(const Shape& s, int dtype) {
   if (dtype != MONARCH_BF16) return 0;
   const int k = fwd_ws_kind(s, dtype);
   if (k == 5 || k == 6) return k;
   if (fwd_path(s, dtype) == 2 && bwd_path(s, dtype) == 1) return 2;
+  if (fwd_path(s, dtype) == 3 && bwd_path(s, dtype) == 3 && tc_stage_supported(s)) return 3;
   return 0;
 }
 
 static size_t saved_bytes(const Shape& s, int dtype) {
   switch (saved_kind(s, dtype)) {
     case 2:
+    case 3:
     case 6: return (size_t)s.rows * (size_t)s.n_mid() * 2;
     case 5: return gemm_fwd_workspace(s);
     default: return 0;
@@ -286,6 +289,7 @@ int monarch_fwd_train(const void* X, const void* R, const void* L, const monarch
   int* status = status_ptr();
   if (status == nullptr) return MONARCH_ERR_CUDA;
   const cudaError_t e = kind == 2   ? tc_rows_fwd_save(X, R, L, Y, saved, s, status, st)
+                        : kind == 3 ? tc_wide_fwd_save(X, R, L, Y, saved, s, status, st)
                         : kind == 5 ? gemm_fwd(X, R, L, Y, saved, s, status, st)
                                     : tc_stage_fwd(X, R, L, Y, saved, s, status, st);
   return e == cudaSuccess ? MONARCH_OK : MONARCH_ERR_CUDA;

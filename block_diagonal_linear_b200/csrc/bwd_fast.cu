@@ -178,12 +178,9 @@ cudaError_t fast_bwd(const void* dY, const void* X, const void* R, const void* L
   }
   if (s.rows > 0) {
     // dR[k] = sum_rows dU_k^T X_k;  dL[j] = sum_rows dV_j^T Z_j  (all operands block-contiguous)
-    if ((e = wgrad_tc(dU, s.n_mid(), s.out1, X, s.n_in(), s.in1, s.nb1, 0, 0, 0, s.rows, sp, part, nP, 0,
-                      status, st)) != cudaSuccess)
-      return e;
-    if ((e = wgrad_tc(dV, s.n_out(), s.out2, Z, s.n_mid(), s.in2, s.nb2, 0, 0, 0, s.rows, sp, part, nP,
-                      nR, status, st)) != cudaSuccess)
-      return e;
+    const WgradArgs gR = {dU, s.n_mid(), s.out1, X, s.n_in(), s.in1, s.nb1, 0, 0, 0, sp, nP, 0};
+    const WgradArgs gL = {dV, s.n_out(), s.out2, Z, s.n_mid(), s.in2, s.nb2, 0, 0, 0, sp, nP, nR};
+    if ((e = wgrad_tc2(gR, gL, s.rows, part, status, st)) != cudaSuccess) return e;
   } else if ((e = cudaMemsetAsync(part, 0, sizeof(float) * (size_t)sp.nsplit * (size_t)nP, st)) != cudaSuccess) {
     return e;
   }

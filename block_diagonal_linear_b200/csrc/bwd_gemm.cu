@@ -184,9 +184,9 @@ __global__ void __launch_bounds__(kPermColWarps * 32)
 
 // ---------------------------------------------------------------- weight gradient
 // Split of the rows for the weight-gradient GEMMs: chunks of a multiple of 64 rows, enough of
-// them that both launches together give about two units per SM, but at least 256 rows each
-// (every chunk costs one fp32 copy of the parameters in partials), and none of them empty
-// (an empty chunk would leave its partials unwritten).
+// them that the two products (dR and dL, one launch) give about two units per SM, but at least
+// 256 rows each (every chunk costs one fp32 copy of the parameters in partials), and none of
+// them empty (an empty chunk would leave its partials unwritten).
 WgradSplit wgrad_split(int64_t rows, int64_t units_per_split) {
   int64_t n = (2 * 148 + units_per_split - 1) / (units_per_split > 0 ? units_per_split : 1);
   const int64_t maxs = rows / 256;
@@ -206,39 +206,62 @@ WgradSplit wgrad_split(int64_t rows, int64_t units_per_split) {
 // columns [b*blk_b, (b+1)*blk_b).  With b_grp = 0, A2 is block-contiguous too; otherwise its
 // 64-column groups are gathered: group g of block b starts at b*b_base + (g / b_grp)*b_gs +
 // (g % b_grp)*64.  Partials are in logical column order.
-cudaError_t wgrad_tc(const void* A1, int64_t a_cols, int64_t blk_a, const void* A2, int64_t b_cols, int64_t blk_b,
-                     int64_t nblocks, int b_base, int b_grp, int b_gs, int64_t rows, WgradSplit sp, float* partial,
-                     int64_t p_stride, int64_t p_off, int* status, cudaStream_t st) {
+static int wgrad_job(const WgradArgs& w, GemmJob* jp) {
   GemmJob j = {};
   // M side: a group of 128 columns of A1 holding bpg whole blocks, or one block per group in
   // 128-row tiles (rows of a tile beyond the block belong to the next block and are dropped)
   int64_t bpg = 1;  // blocks per group
-  if (blk_a <= 128 && 128 % blk_a == 0 && nblocks % (128 / blk_a) == 0) bpg = 128 / blk_a;
-  j.mtiles = (int)((blk_a + 127) / 128);
-  const int64_t nw = bpg * blk_b;  // B columns a group needs
+  if (w.blk_a <= 128 && 128 % w.blk_a == 0 && w.nblocks % (128 / w.blk_a) == 0) bpg = 128 / w.blk_a;
+  j.mtiles = (int)((w.blk_a + 127) / 128);
+  const int64_t nw = bpg * w.blk_b;  // B columns a group needs
   const int BN = nw >= 256 ? 256 : (nw > 64 ? 128 : 64);
-  if ((bpg * blk_a) % 8 || (bpg * b_base) % 8 || nw % 8) return cudaErrorInvalidValue;  // 16-byte TMA x
-  if (blk_a % 4 || blk_b % 4 || p_stride % 4 || p_off % 4) return cudaErrorInvalidValue;  // float4 partials
-  j.nb = (int)(nblocks / bpg);
+  if ((bpg * w.blk_a) % 8 || (bpg * w.b_base) % 8 || nw % 8) return 0;  // 16-byte TMA x
+  if (w.blk_a % 4 || w.blk_b % 4 || w.p_stride % 4 || w.p_off % 4) return 0;  // float4 partials
+  j.nb = (int)(w.nblocks / bpg);
   j.ntiles = (int)((nw + BN - 1) / BN);
-  j.nsplit = sp.nsplit;
-  j.split_rows = sp.rows_per_split;
-  j.a_b = (int)(bpg * blk_a);
+  j.nsplit = w.sp.nsplit;
+  j.split_rows = w.sp.rows_per_split;
+  j.a_b = (int)(bpg * w.blk_a);
   j.b_lb = (int)nw;
-  if (b_grp == 0) {  // contiguous
+  if (w.b_grp == 0) {  // contiguous
     j.b_b = (int)nw;
     j.b_grp = 1 << 30;
     j.b_gs = 0;
   } else {
-    j.b_b = (int)(bpg * b_base);
-    j.b_grp = b_grp;
-    j.b_gs = b_gs;
+    j.b_b = (int)(bpg * w.b_base);
+    j.b_grp = w.b_grp;
+    j.b_gs = w.b_gs;
   }
-  j.blk_a = blk_a;
-  j.blk_b = blk_b;
-  j.p_stride = p_stride;
-  j.p_off = p_off;
+  j.blk_a = w.blk_a;
+  j.blk_b = w.blk_b;
+  j.p_stride = w.p_stride;
+  j.p_off = w.p_off;
+  *jp = j;
+  return BN;
+}
+
+cudaError_t wgrad_tc(const void* A1, int64_t a_cols, int64_t blk_a, const void* A2, int64_t b_cols, int64_t blk_b,
+                     int64_t nblocks, int b_base, int b_grp, int b_gs, int64_t rows, WgradSplit sp, float* partial,
+                     int64_t p_stride, int64_t p_off, int* status, cudaStream_t st) {
+  const WgradArgs w = {A1, a_cols, blk_a, A2, b_cols, blk_b, nblocks, b_base, b_grp, b_gs, sp, p_stride, p_off};
+  GemmJob j;
+  const int BN = wgrad_job(w, &j);
+  if (BN == 0) return cudaErrorInvalidValue;
   return gemm_wgrad(A1, a_cols, A2, b_cols, rows, BN, j, partial, status, st, true);
+}
+
+cudaError_t wgrad_tc2(const WgradArgs& w1, const WgradArgs& w2, int64_t rows, float* partial, int* status,
+                      cudaStream_t st) {
+  GemmJob j1, j2;
+  const int bn1 = wgrad_job(w1, &j1), bn2 = wgrad_job(w2, &j2);
+  if (bn1 == 0 || bn2 == 0) return cudaErrorInvalidValue;
+  if (bn1 != bn2) {
+    cudaError_t e = gemm_wgrad(w1.A1, w1.a_cols, w1.A2, w1.b_cols, rows, bn1, j1, partial, status, st, true);
+    if (e != cudaSuccess) return e;
+    return gemm_wgrad(w2.A1, w2.a_cols, w2.A2, w2.b_cols, rows, bn2, j2, partial, status, st, true);
+  }
+  const WgradOperands o1 = {w1.A1, w1.a_cols, w1.A2, w1.b_cols}, o2 = {w2.A1, w2.a_cols, w2.A2, w2.b_cols};
+  return gemm_wgrad2(o1, j1, o2, j2, rows, bn1, partial, status, st, true);
 }
 
 // Row split for one weight-gradient launch on its own: as many chunks (multiples of 64 rows,
@@ -286,7 +309,7 @@ static size_t al256(size_t b) { return (b + 255) & ~size_t(255); }
 
 struct GemmBwdWs {
   size_t rt, ltp, u, du, part, total;
-  WgradSplit spR, spL;  // each weight-gradient launch has its own row split
+  WgradSplit spR, spL;  // each weight-gradient job has its own row split
 };
 
 // Units of one row chunk of the weight-gradient GEMM: blocks x block/128 m tiles x K/BN n tiles.
@@ -364,12 +387,10 @@ cudaError_t gemm_bwd(const void* dY, const void* X, const void* R, const void* L
                      true)) != cudaSuccess)
       return e;
     // 5. weight gradients
-    if ((e = wgrad_tc(dU, s.n_mid(), s.out1, X, s.n_in(), s.in1, s.nb1, 0, 0, 0, s.rows,
-                      w.spR, part, nR, 0, status, st)) != cudaSuccess)
-      return e;
-    if ((e = wgrad_tc(dY, s.n_out(), s.out2, U, s.n_mid(), s.in2, s.nb2, G, G / 64, s.out1, s.rows,
-                      w.spL, part + (int64_t)w.spR.nsplit * nR, nL, 0, status, st)) != cudaSuccess)
-      return e;
+    const WgradArgs gR = {dU, s.n_mid(), s.out1, X, s.n_in(), s.in1, s.nb1, 0, 0, 0, w.spR, nR, 0};
+    const WgradArgs gL = {dY, s.n_out(), s.out2, U, s.n_mid(), s.in2, s.nb2, G, G / 64, s.out1, w.spL, nL,
+                          (int64_t)w.spR.nsplit * nR};
+    if ((e = wgrad_tc2(gR, gL, s.rows, part, status, st)) != cudaSuccess) return e;
   } else {
     const size_t np = (size_t)w.spR.nsplit * (size_t)nR + (size_t)w.spL.nsplit * (size_t)nL;
     if ((e = cudaMemsetAsync(part, 0, sizeof(float) * np, st)) != cudaSuccess) return e;
@@ -566,7 +587,7 @@ cudaError_t packed_stage(const void* A, int64_t rows, const void* W, void* Y, in
 }
 
 cudaError_t packed_bwd(const void* dY, const void* X, const void* R, const void* L, void* dX, void* dR, void* dL,
-                       void* ws, const Shape& s, int* status, cudaStream_t st) {
+                       void* ws, const Shape& s, int* status, cudaStream_t st, const void* saved) {
   const PackInfo pk = pack_info(s);
   const PackedWs w = packed_layout(s);
   char* base = (char*)ws;
@@ -584,6 +605,8 @@ cudaError_t packed_bwd(const void* dY, const void* X, const void* R, const void*
       cudaSuccess)
     return e;
   const bool staged = tc_stage_supported(s);
+  if (saved != nullptr && staged) Z = (__nv_bfloat16*)saved;  // kept by the training forward
+  const bool need_z = saved == nullptr || !staged;
   if (staged && s.rows > 0) {
     // the streaming stages take the plain factors: L^T into the (then unused) packed L^T
     // region, R^T into the packed-R region (the transpose helper writes both)
@@ -602,17 +625,15 @@ cudaError_t packed_bwd(const void* dY, const void* X, const void* R, const void*
     }
     if ((e = packed_stage(dU, s.rows, Wx, dX, s.nb1, s.out1, s.in1, pk.gx, status, st)) != cudaSuccess) return e;
     if (staged) {
-      if ((e = tc_stage(X, R, Z, StageKind::R, s, status, st, true, true)) != cudaSuccess) return e;  // Z = P R x
+      // Z = P R x (R is the caller's: its weights may load before the wait)
+      if (need_z && (e = tc_stage(X, R, Z, StageKind::R, s, status, st, true, true)) != cudaSuccess) return e;
     } else {
       if ((e = packed_stage(X, s.rows, Wu, U, s.nb1, s.in1, s.out1, pk.gx, status, st)) != cudaSuccess) return e;
       if ((e = permute_rows(U, Z, s.rows, s.nb1, s.out1, st)) != cudaSuccess) return e;
     }
-    if ((e = wgrad_tc(dU, s.n_mid(), s.out1, X, s.n_in(), s.in1, s.nb1, 0, 0, 0, s.rows, w.sp, part, nP, 0,
-                      status, st)) != cudaSuccess)
-      return e;
-    if ((e = wgrad_tc(dV, s.n_out(), s.out2, Z, s.n_mid(), s.in2, s.nb2, 0, 0, 0, s.rows, w.sp, part, nP,
-                      nR, status, st)) != cudaSuccess)
-      return e;
+    const WgradArgs gR = {dU, s.n_mid(), s.out1, X, s.n_in(), s.in1, s.nb1, 0, 0, 0, w.sp, nP, 0};
+    const WgradArgs gL = {dV, s.n_out(), s.out2, Z, s.n_mid(), s.in2, s.nb2, 0, 0, 0, w.sp, nP, nR};
+    if ((e = wgrad_tc2(gR, gL, s.rows, part, status, st)) != cudaSuccess) return e;
   } else if ((e = cudaMemsetAsync(part, 0, sizeof(float) * (size_t)w.sp.nsplit * (size_t)nP, st)) != cudaSuccess) {
     return e;
   }

@@ -128,6 +128,9 @@ cudaError_t tc_rows_fwd(const void* X, const void* R, const void* L, void* Y, co
 bool tc_wide_supported(const Shape& s);
 cudaError_t tc_wide_fwd(const void* X, const void* R, const void* L, void* Y, const Shape& s,
                         int* status, cudaStream_t st);
+// The same forward also writing the middle vector Z (rows x n_mid, the L stage's input order).
+cudaError_t tc_wide_fwd_save(const void* X, const void* R, const void* L, void* Y, void* Z, const Shape& s,
+                             int* status, cudaStream_t st);
 
 // Large square blocks (64 x 64, nb1 = nb2): block-diagonal tcgen05 GEMMs and row permutations
 // as four passes over Y (no scratch).

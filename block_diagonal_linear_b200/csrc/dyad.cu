@@ -287,11 +287,9 @@ int monarch_dyad_bwd(const void* dY, const void* X, const void* W1, const void* 
         (e = permute_rows_add(PX, dX, s.rows, s.ib, s.nb, st)) != cudaSuccess ||
         (e = permute_rows(X, PX, s.rows, s.nb, s.ib, st)) != cudaSuccess)
       return MONARCH_ERR_CUDA;
-    if ((e = wgrad_tc(dY, n_out, s.ob, X, n_in, s.ib, s.nb, 0, 0, 0, s.rows, w.sp, part, 2 * nW, 0, status,
-                      st)) != cudaSuccess ||
-        (e = wgrad_tc(DV, n_out, s.ob, PX, n_in, s.ib, s.nb, 0, 0, 0, s.rows, w.sp, part, 2 * nW, nW, status,
-                      st)) != cudaSuccess)
-      return MONARCH_ERR_CUDA;
+    const WgradArgs g1 = {dY, n_out, s.ob, X, n_in, s.ib, s.nb, 0, 0, 0, w.sp, 2 * nW, 0};
+    const WgradArgs g2 = {DV, n_out, s.ob, PX, n_in, s.ib, s.nb, 0, 0, 0, w.sp, 2 * nW, nW};
+    if ((e = wgrad_tc2(g1, g2, s.rows, part, status, st)) != cudaSuccess) return MONARCH_ERR_CUDA;
   } else if ((e = cudaMemsetAsync(part, 0, sizeof(float) * (size_t)w.sp.nsplit * 2 * nW, st)) != cudaSuccess) {
     return MONARCH_ERR_CUDA;
   }

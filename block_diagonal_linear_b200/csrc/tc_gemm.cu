@@ -14,7 +14,9 @@
 //     group of blocks, A = act1[rows][cols] and B = act2[rows][cols], so
 //     D[m][n] = sum_r act1[r][m] act2[r][n]; the rows are split into chunks (split-K) and
 //     each unit writes the diagonal blocks of D (m and n in the same block) as fp32
-//     partials, summed in a fixed order by a separate kernel.
+//     partials, summed in a fixed order by a separate kernel.  One launch may carry two
+//     such jobs (dR and dL of a backward): the units of the second follow those of the
+//     first, with their own operand maps.
 //   kind 2, block-diagonal stage, weight-stationary: as kind 0, but every CTA owns one
 //     (batch b, n tile) pair and a contiguous range of m tiles; its weight tile W[b] (BN x K)
 //     is loaded once and stays in shared memory, only A streams through the ring.  For
@@ -64,6 +66,7 @@ struct GemmBars {
 // group, then split.
 struct UnitCoord {
   int b, mt, nt, split;
+  int second;  // kind 1: the unit belongs to the launch's second job
 };
 __device__ __forceinline__ UnitCoord unit_coord(const GemmJob& j, int64_t u) {
   UnitCoord c;
@@ -79,11 +82,12 @@ __device__ __forceinline__ UnitCoord unit_coord(const GemmJob& j, int64_t u) {
     c.b = (int)(u % j.nb);
     c.split = (int)(u / j.nb);
   }
+  c.second = 0;
   return c;
 }
 
 // Units of this CTA: i = 0, 1, ... < unit_count().  Kinds 0 and 1: unit blockIdx.x + i*gridDim.x
-// of the job.  Kind 2: the CTA's (b, n tile) pair is blockIdx.x % (nb*ntiles) and its m tiles a
+// of the job (kind 1: of the two jobs' units, the second job's after the first's).  Kind 2: the CTA's (b, n tile) pair is blockIdx.x % (nb*ntiles) and its m tiles a
 // contiguous range (the grid is a multiple of nb*ntiles).
 __device__ __forceinline__ void kind2_range(const GemmJob& j, int* b, int* nt, int* lo, int* hi) {
   const int nwg = j.nb * j.ntiles;
@@ -93,15 +97,16 @@ __device__ __forceinline__ void kind2_range(const GemmJob& j, int* b, int* nt, i
   *lo = (int)((int64_t)ci * j.mtiles / cpw);
   *hi = (int)((int64_t)(ci + 1) * j.mtiles / cpw);
 }
-__device__ __forceinline__ int64_t unit_count(const GemmJob& j) {
+__device__ __forceinline__ int64_t unit_count(const GemmJob& j, const GemmJob& j2) {
   if (j.kind == 2) {
     int b, nt, lo, hi;
     kind2_range(j, &b, &nt, &lo, &hi);
     return hi - lo;
   }
-  return j.units > (int64_t)blockIdx.x ? (j.units - blockIdx.x + gridDim.x - 1) / gridDim.x : 0;
+  const int64_t total = j.units + (j.kind == 1 ? j2.units : 0);
+  return total > (int64_t)blockIdx.x ? (total - blockIdx.x + gridDim.x - 1) / gridDim.x : 0;
 }
-__device__ __forceinline__ UnitCoord unit_at(const GemmJob& j, int64_t i) {
+__device__ __forceinline__ UnitCoord unit_at(const GemmJob& j, const GemmJob& j2, int64_t i) {
   if (j.kind == 2) {
     int b, nt, lo, hi;
     kind2_range(j, &b, &nt, &lo, &hi);
@@ -110,9 +115,16 @@ __device__ __forceinline__ UnitCoord unit_at(const GemmJob& j, int64_t i) {
     c.nt = nt;
     c.mt = lo + (int)i;
     c.split = 0;
+    c.second = 0;
     return c;
   }
-  return unit_coord(j, blockIdx.x + i * gridDim.x);
+  const int64_t g = blockIdx.x + i * gridDim.x;
+  if (j.kind == 1 && g >= j.units) {
+    UnitCoord c = unit_coord(j2, g - j.units);
+    c.second = 1;
+    return c;
+  }
+  return unit_coord(j, g);
 }
 
 // Number of 64-wide K stages of a unit.
@@ -127,8 +139,9 @@ __device__ __forceinline__ int unit_kstages(const GemmJob& j, const UnitCoord& c
 template <class C>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                   const __grid_constant__ CUtensorMap tmY, const GemmJob job, float* __restrict__ partial,
-                   int* status) {
+                   const __grid_constant__ CUtensorMap tmY, const __grid_constant__ GemmJob job,
+                   const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB2,
+                   const __grid_constant__ GemmJob job2, float* __restrict__ partial, int* status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t* stg = smem;                      // kinds 0, 2: two 16 KB output staging chunks
@@ -137,7 +150,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   GemmBars* bars = (GemmBars*)(ring + C::NSTAGE * C::STAGE);
   int* abort_flag = &bars->abort_flag;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int64_t nmine = unit_count(job);  // units of this CTA
+  const int64_t nmine = unit_count(job, job2);  // units of this CTA
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::NSTAGE; ++i) {
@@ -171,9 +184,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       ptx::tma_prefetch_desc(&tmA);
       ptx::tma_prefetch_desc(&tmB);
       if (C::KIND != 1) ptx::tma_prefetch_desc(&tmY);
+      if (C::KIND == 1 && job2.units > 0) {
+        ptx::tma_prefetch_desc(&tmA2);
+        ptx::tma_prefetch_desc(&tmB2);
+      }
       const uint64_t pol = ptx::policy_evict_normal();
       if (C::KIND == 2 && nmine > 0) {
-        const UnitCoord c0 = unit_at(job, 0);
+        const UnitCoord c0 = unit_at(job, job2, 0);
         ptx::mbar_arrive_expect_tx(&bars->wfull, C::W_BYTES);
         for (int kb = 0; kb < C::KBOX; ++kb)
           ptx::tma_load_2d(wreg + kb * (C::BN * 128), &tmB, &bars->wfull, kb * 64, c0.b * job.b_b + c0.nt * C::BN,
@@ -182,8 +199,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       uint32_t it = 0;
       bool ok = true;
       for (int64_t i = 0; i < nmine && ok; ++i) {
-        const UnitCoord c = unit_at(job, i);
-        const int nk = unit_kstages(job, c);
+        const UnitCoord c = unit_at(job, job2, i);
+        const GemmJob& jb = c.second ? job2 : job;
+        const CUtensorMap* mapA = c.second ? &tmA2 : &tmA;
+        const CUtensorMap* mapB = c.second ? &tmB2 : &tmB;
+        const int nk = unit_kstages(jb, c);
         for (int kb = 0; kb < nk; ++kb, ++it) {
           const int st = it % C::NSTAGE;
           if (!wait_or_abort(&bars->empty[st], ((it / C::NSTAGE) & 1) ^ 1, abort_flag, status)) { ok = false; break; }
@@ -195,21 +215,21 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             ptx::tma_load_2d(sa, &tmA, &bars->full[st], ax, c.mt * C::BM, pol);
             if (C::KIND == 0) ptx::tma_load_2d(sb, &tmB, &bars->full[st], kb * 64, c.b * job.b_b + c.nt * C::BN, pol);
           } else {
-            const int row = (int)((int64_t)c.split * job.split_rows + (int64_t)kb * 64);
-            const int ax = c.b * job.a_b + c.mt * C::BM;
-            if (job.ab3d) {
+            const int row = (int)((int64_t)c.split * jb.split_rows + (int64_t)kb * 64);
+            const int ax = c.b * jb.a_b + c.mt * C::BM;
+            if (jb.ab3d) {
               // one op per operand: TMA throughput per SM grows with the bytes per op (8 KB boxes
               // cap it near 50 GB/s, 16-32 KB ones reach 90-115 GB/s from L2)
-              ptx::tma_load_3d(sa, &tmA, &bars->full[st], 0, row, ax / 64, pol);
-              ptx::tma_load_3d(sb, &tmB, &bars->full[st], 0, row,
-                               gcol(c.b, job.b_b, c.nt * (C::BN / 64), job.b_grp, job.b_gs) / 64, pol);
+              ptx::tma_load_3d(sa, mapA, &bars->full[st], 0, row, ax / 64, pol);
+              ptx::tma_load_3d(sb, mapB, &bars->full[st], 0, row,
+                               gcol(c.b, jb.b_b, c.nt * (C::BN / 64), jb.b_grp, jb.b_gs) / 64, pol);
             } else {
-              ptx::tma_load_2d(sa, &tmA, &bars->full[st], ax, row, pol);
-              ptx::tma_load_2d(sa + 8192, &tmA, &bars->full[st], ax + 64, row, pol);
+              ptx::tma_load_2d(sa, mapA, &bars->full[st], ax, row, pol);
+              ptx::tma_load_2d(sa + 8192, mapA, &bars->full[st], ax + 64, row, pol);
 #pragma unroll
               for (int h = 0; h < C::BN / 64; ++h)
-                ptx::tma_load_2d(sb + h * 8192, &tmB, &bars->full[st],
-                                 gcol(c.b, job.b_b, c.nt * (C::BN / 64) + h, job.b_grp, job.b_gs), row, pol);
+                ptx::tma_load_2d(sb + h * 8192, mapB, &bars->full[st],
+                                 gcol(c.b, jb.b_b, c.nt * (C::BN / 64) + h, jb.b_grp, jb.b_gs), row, pol);
             }
           }
         }
@@ -234,8 +254,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     bool ok = true;
     if (C::KIND == 2 && nmine > 0) ok = warp_wait_or_abort(lane, &bars->wfull, 0, abort_flag, status);
     for (int64_t i = 0; i < nmine && ok; ++i, ++n) {
-      const UnitCoord c = unit_at(job, i);
-      const int nk = unit_kstages(job, c);
+      const UnitCoord c = unit_at(job, job2, i);
+      const int nk = unit_kstages(c.second ? job2 : job, c);
       const int slot = n & 1;
       if (!warp_wait_or_abort(lane, &bars->acc_empty[slot], ((n >> 1) & 1) ^ 1, abort_flag, status)) { ok = false; break; }
       ptx::tc_fence_after();
@@ -269,7 +289,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     uint32_t n = 0, chunk_n = 0;
     bool ok = true;
     for (int64_t i = 0; i < nmine && ok; ++i, ++n) {
-      const UnitCoord c = unit_at(job, i);
+      const UnitCoord c = unit_at(job, job2, i);
+      const GemmJob& jb = c.second ? job2 : job;
       const int slot = n & 1;
       if (!wait_or_abort(&bars->acc_full[slot], (n >> 1) & 1, abort_flag, status)) { ok = false; break; }
       ptx::tc_fence_after();
@@ -310,18 +331,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         // its values go to the columns of that block, in logical column order (any column
         // permutation is applied when the partials are summed).  32-bit index math, one
         // division per unit, float4 stores.
-        const int bla = (int)job.blk_a, blb = (int)job.blk_b;
-        const int ma = c.b * job.a_b + c.mt * C::BM + r;
-        const int nb0 = c.b * job.b_lb + c.nt * C::BN;
+        const int bla = (int)jb.blk_a, blb = (int)jb.blk_b;
+        const int ma = c.b * jb.a_b + c.mt * C::BM + r;
+        const int nb0 = c.b * jb.b_lb + c.nt * C::BN;
         const int blk = ma / bla;
-        const bool row_ok = ma < (int)job.a_cols;
+        const bool row_ok = ma < (int)jb.a_cols;
         const int t_lo = max(0, blk * blb - nb0);
-        const int t_hi = min(C::BN, min((blk + 1) * blb, (int)job.b_cols) - nb0);
+        const int t_hi = min(C::BN, min((blk + 1) * blb, (int)jb.b_cols) - nb0);
         // the warp's column range: from its first row's block to its last row's block
-        const int ma0 = c.b * job.a_b + c.mt * C::BM + quad * 32;
+        const int ma0 = c.b * jb.a_b + c.mt * C::BM + quad * 32;
         const int w_lo = max(0, (ma0 / bla) * blb - nb0) & ~15;
         const int w_hi = min(C::BN, ((ma0 + 31) / bla + 1) * blb - nb0);
-        float* prow = partial + (int64_t)c.split * job.p_stride + job.p_off + (int64_t)blk * bla * blb +
+        float* prow = partial + (int64_t)c.split * jb.p_stride + jb.p_off + (int64_t)blk * bla * blb +
                       (int64_t)(ma - blk * bla) * blb + (nb0 - blk * blb);  // + tile column
         for (int c0 = w_lo; c0 < w_hi; c0 += 16) {
           uint32_t t16[16];
@@ -353,8 +374,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
 template <int BN, int KIND, int KBOX = 0>
 static cudaError_t launch_gemm_cfg(const CUtensorMap& mA, const CUtensorMap& mB, const CUtensorMap& mY,
-                                   const GemmJob& job, float* partial, int* status, cudaStream_t st,
-                                   bool pdl) {
+                                   const GemmJob& job, const CUtensorMap& mA2, const CUtensorMap& mB2,
+                                   const GemmJob& job2, float* partial, int* status, cudaStream_t st, bool pdl) {
   using C = GemmCfg<BN, KIND, KBOX>;
   cudaError_t e = ensure_smem_attr((const void*)tc_gemm_kernel<C>, C::SMEM_BYTES);
   if (e != cudaSuccess) return e;
@@ -367,11 +388,20 @@ static cudaError_t launch_gemm_cfg(const CUtensorMap& mA, const CUtensorMap& mB,
     if (cpw > job.mtiles) cpw = job.mtiles;
     grid = nwg * cpw;
   } else {
+    const int64_t units = job.units + (KIND == 1 ? job2.units : 0);
     grid = num_sms();
-    if (grid > job.units) grid = job.units;
+    if (grid > units) grid = units;
   }
   return launch_kernel(tc_gemm_kernel<C>, dim3((unsigned)grid), dim3(kGemmThreads), C::SMEM_BYTES, st, pdl,
-                       mA, mB, mY, job, partial, status);
+                       mA, mB, mY, job, mA2, mB2, job2, partial, status);
+}
+
+// One-job launch of the block-diagonal stage kinds (the second job is empty).
+template <int BN, int KIND, int KBOX = 0>
+static cudaError_t launch_stage_cfg(const CUtensorMap& mA, const CUtensorMap& mB, const CUtensorMap& mY,
+                                    const GemmJob& job, int* status, cudaStream_t st, bool pdl) {
+  const GemmJob none = {};
+  return launch_gemm_cfg<BN, KIND, KBOX>(mA, mB, mY, job, mA, mB, none, nullptr, status, st, pdl);
 }
 
 cudaError_t gemm_bd(const void* A, int64_t rows, int64_t a_cols, const void* W, int64_t w_rows, int K,
@@ -392,22 +422,67 @@ cudaError_t gemm_bd(const void* A, int64_t rows, int64_t a_cols, const void* W, 
   job.kind = 0;
   if (stationary) {
     job.kind = 2;
-    if (BN == 256 && kbox == 4) return launch_gemm_cfg<256, 2, 4>(mA, mB, mY, job, nullptr, status, st, pdl);
-    if (BN == 256 && kbox == 2) return launch_gemm_cfg<256, 2, 2>(mA, mB, mY, job, nullptr, status, st, pdl);
-    if (BN == 128 && kbox == 8) return launch_gemm_cfg<128, 2, 8>(mA, mB, mY, job, nullptr, status, st, pdl);
-    if (BN == 128 && kbox == 4) return launch_gemm_cfg<128, 2, 4>(mA, mB, mY, job, nullptr, status, st, pdl);
-    if (BN == 128 && kbox == 2) return launch_gemm_cfg<128, 2, 2>(mA, mB, mY, job, nullptr, status, st, pdl);
-    if (BN == 64 && kbox == 16) return launch_gemm_cfg<64, 2, 16>(mA, mB, mY, job, nullptr, status, st, pdl);
-    if (BN == 64 && kbox == 4) return launch_gemm_cfg<64, 2, 4>(mA, mB, mY, job, nullptr, status, st, pdl);
-    if (BN == 64 && kbox == 3) return launch_gemm_cfg<64, 2, 3>(mA, mB, mY, job, nullptr, status, st, pdl);
-    if (BN == 64 && kbox == 2) return launch_gemm_cfg<64, 2, 2>(mA, mB, mY, job, nullptr, status, st, pdl);
-    if (BN == 64 && kbox == 1) return launch_gemm_cfg<64, 2, 1>(mA, mB, mY, job, nullptr, status, st, pdl);
+    if (BN == 256 && kbox == 4) return launch_stage_cfg<256, 2, 4>(mA, mB, mY, job, status, st, pdl);
+    if (BN == 256 && kbox == 2) return launch_stage_cfg<256, 2, 2>(mA, mB, mY, job, status, st, pdl);
+    if (BN == 128 && kbox == 8) return launch_stage_cfg<128, 2, 8>(mA, mB, mY, job, status, st, pdl);
+    if (BN == 128 && kbox == 4) return launch_stage_cfg<128, 2, 4>(mA, mB, mY, job, status, st, pdl);
+    if (BN == 128 && kbox == 2) return launch_stage_cfg<128, 2, 2>(mA, mB, mY, job, status, st, pdl);
+    if (BN == 64 && kbox == 16) return launch_stage_cfg<64, 2, 16>(mA, mB, mY, job, status, st, pdl);
+    if (BN == 64 && kbox == 4) return launch_stage_cfg<64, 2, 4>(mA, mB, mY, job, status, st, pdl);
+    if (BN == 64 && kbox == 3) return launch_stage_cfg<64, 2, 3>(mA, mB, mY, job, status, st, pdl);
+    if (BN == 64 && kbox == 2) return launch_stage_cfg<64, 2, 2>(mA, mB, mY, job, status, st, pdl);
+    if (BN == 64 && kbox == 1) return launch_stage_cfg<64, 2, 1>(mA, mB, mY, job, status, st, pdl);
     job.kind = 0;  // no resident configuration for this tile: stream the weights
   }
   switch (BN) {
-    case 64: return launch_gemm_cfg<64, 0>(mA, mB, mY, job, nullptr, status, st, pdl);
-    case 128: return launch_gemm_cfg<128, 0>(mA, mB, mY, job, nullptr, status, st, pdl);
-    case 256: return launch_gemm_cfg<256, 0>(mA, mB, mY, job, nullptr, status, st, pdl);
+    case 64: return launch_stage_cfg<64, 0>(mA, mB, mY, job, status, st, pdl);
+    case 128: return launch_stage_cfg<128, 0>(mA, mB, mY, job, status, st, pdl);
+    case 256: return launch_stage_cfg<256, 0>(mA, mB, mY, job, status, st, pdl);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+// Operand maps of one weight-gradient job; sets job.ab3d, kind, rows, widths and units.
+static bool wgrad_maps(const void* A1, int64_t a_cols, const void* A2, int64_t b_cols, int64_t rows, int BN,
+                       GemmJob* job, CUtensorMap* mA, CUtensorMap* mB) {
+  // Multi-chunk boxes need every unit's operand columns to start on a 64-column chunk and a
+  // stage's BN/64 B chunks to be contiguous (one gathered group, or no gather).
+  const int nbc = BN / 64;
+  const bool b_contig = job->b_grp >= (1 << 29) || (job->b_grp % nbc == 0 && job->b_gs % 64 == 0);
+  job->ab3d = (a_cols % 64 == 0 && b_cols % 64 == 0 && job->a_b % 64 == 0 && job->b_b % 64 == 0 && b_contig) ? 1 : 0;
+  if (job->ab3d) {
+    const uint64_t da[3] = {64, (uint64_t)rows, (uint64_t)a_cols / 64}, sa_[2] = {(uint64_t)a_cols * 2, 128};
+    const uint64_t db[3] = {64, (uint64_t)rows, (uint64_t)b_cols / 64}, sb_[2] = {(uint64_t)b_cols * 2, 128};
+    const uint32_t ba[3] = {64, 64, 2}, bb[3] = {64, 64, (uint32_t)nbc};
+    if (!make_map_3d(mA, A1, da, sa_, ba, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map_3d(mB, A2, db, sb_, bb, CU_TENSOR_MAP_SWIZZLE_128B))
+      return false;
+  } else if (!make_map_2d(mA, A1, (uint64_t)a_cols, (uint64_t)rows, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
+             !make_map_2d(mB, A2, (uint64_t)b_cols, (uint64_t)rows, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B)) {
+    return false;
+  }
+  job->kind = 1;
+  job->rows = rows;
+  job->a_cols = a_cols;
+  job->b_cols = b_cols;
+  job->units = (int64_t)job->mtiles * job->ntiles * job->nb * job->nsplit;
+  return true;
+}
+
+template <int BN>
+static cudaError_t launch_wgrad_cfg(const CUtensorMap& mA, const CUtensorMap& mB, const GemmJob& job,
+                                    const CUtensorMap& mA2, const CUtensorMap& mB2, const GemmJob& job2,
+                                    float* partial, int* status, cudaStream_t st, bool pdl) {
+  return launch_gemm_cfg<BN, 1>(mA, mB, mA, job, mA2, mB2, job2, partial, status, st, pdl);
+}
+
+static cudaError_t launch_wgrad(int BN, const CUtensorMap& mA, const CUtensorMap& mB, const GemmJob& job,
+                                const CUtensorMap& mA2, const CUtensorMap& mB2, const GemmJob& job2,
+                                float* partial, int* status, cudaStream_t st, bool pdl) {
+  switch (BN) {
+    case 64: return launch_wgrad_cfg<64>(mA, mB, job, mA2, mB2, job2, partial, status, st, pdl);
+    case 128: return launch_wgrad_cfg<128>(mA, mB, job, mA2, mB2, job2, partial, status, st, pdl);
+    case 256: return launch_wgrad_cfg<256>(mA, mB, job, mA2, mB2, job2, partial, status, st, pdl);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -415,33 +490,18 @@ cudaError_t gemm_bd(const void* A, int64_t rows, int64_t a_cols, const void* W, 
 cudaError_t gemm_wgrad(const void* A1, int64_t a_cols, const void* A2, int64_t b_cols, int64_t rows, int BN,
                        GemmJob job, float* partial, int* status, cudaStream_t st, bool pdl) {
   CUtensorMap mA, mB;
-  // Multi-chunk boxes need every unit's operand columns to start on a 64-column chunk and a
-  // stage's BN/64 B chunks to be contiguous (one gathered group, or no gather).
-  const int nbc = BN / 64;
-  const bool b_contig = job.b_grp >= (1 << 29) || (job.b_grp % nbc == 0 && job.b_gs % 64 == 0);
-  job.ab3d = (a_cols % 64 == 0 && b_cols % 64 == 0 && job.a_b % 64 == 0 && job.b_b % 64 == 0 && b_contig) ? 1 : 0;
-  if (job.ab3d) {
-    const uint64_t da[3] = {64, (uint64_t)rows, (uint64_t)a_cols / 64}, sa_[2] = {(uint64_t)a_cols * 2, 128};
-    const uint64_t db[3] = {64, (uint64_t)rows, (uint64_t)b_cols / 64}, sb_[2] = {(uint64_t)b_cols * 2, 128};
-    const uint32_t ba[3] = {64, 64, 2}, bb[3] = {64, 64, (uint32_t)nbc};
-    if (!make_map_3d(&mA, A1, da, sa_, ba, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_map_3d(&mB, A2, db, sb_, bb, CU_TENSOR_MAP_SWIZZLE_128B))
-      return cudaErrorInvalidValue;
-  } else if (!make_map_2d(&mA, A1, (uint64_t)a_cols, (uint64_t)rows, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
-             !make_map_2d(&mB, A2, (uint64_t)b_cols, (uint64_t)rows, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B)) {
+  if (!wgrad_maps(A1, a_cols, A2, b_cols, rows, BN, &job, &mA, &mB)) return cudaErrorInvalidValue;
+  const GemmJob none = {};
+  return launch_wgrad(BN, mA, mB, job, mA, mB, none, partial, status, st, pdl);
+}
+
+cudaError_t gemm_wgrad2(const WgradOperands& o1, GemmJob job1, const WgradOperands& o2, GemmJob job2,
+                        int64_t rows, int BN, float* partial, int* status, cudaStream_t st, bool pdl) {
+  CUtensorMap mA, mB, mA2, mB2;
+  if (!wgrad_maps(o1.A1, o1.a_cols, o1.A2, o1.b_cols, rows, BN, &job1, &mA, &mB) ||
+      !wgrad_maps(o2.A1, o2.a_cols, o2.A2, o2.b_cols, rows, BN, &job2, &mA2, &mB2))
     return cudaErrorInvalidValue;
-  }
-  job.kind = 1;
-  job.rows = rows;
-  job.a_cols = a_cols;
-  job.b_cols = b_cols;
-  job.units = (int64_t)job.mtiles * job.ntiles * job.nb * job.nsplit;
-  switch (BN) {
-    case 64: return launch_gemm_cfg<64, 1>(mA, mB, mA, job, partial, status, st, pdl);
-    case 128: return launch_gemm_cfg<128, 1>(mA, mB, mA, job, partial, status, st, pdl);
-    case 256: return launch_gemm_cfg<256, 1>(mA, mB, mA, job, partial, status, st, pdl);
-    default: return cudaErrorInvalidValue;
-  }
+  return launch_wgrad(BN, mA, mB, job1, mA2, mB2, job2, partial, status, st, pdl);
 }
 
 }  // namespace monarch

@@ -50,6 +50,15 @@ cudaError_t gemm_bd(const void* A, int64_t rows, int64_t a_cols, const void* W, 
 // p_stride, p_off.
 cudaError_t gemm_wgrad(const void* A1, int64_t a_cols, const void* A2, int64_t b_cols, int64_t rows, int BN,
                        GemmJob job, float* partial, int* status, cudaStream_t st, bool pdl);
+// Two kind-1 jobs with the same BN in one launch (the second job's units follow the first's).
+struct WgradOperands {
+  const void* A1;
+  int64_t a_cols;
+  const void* A2;
+  int64_t b_cols;
+};
+cudaError_t gemm_wgrad2(const WgradOperands& o1, GemmJob job1, const WgradOperands& o2, GemmJob job2,
+                        int64_t rows, int BN, float* partial, int* status, cudaStream_t st, bool pdl);
 
 // Row split of the weight-gradient GEMMs (see bwd_gemm.cu).
 struct WgradSplit {
@@ -60,6 +69,19 @@ WgradSplit wgrad_split(int64_t rows, int64_t units_per_split);
 cudaError_t wgrad_tc(const void* A1, int64_t a_cols, int64_t blk_a, const void* A2, int64_t b_cols, int64_t blk_b,
                      int64_t nblocks, int b_base, int b_grp, int b_gs, int64_t rows, WgradSplit sp, float* partial,
                      int64_t p_stride, int64_t p_off, int* status, cudaStream_t st);
+// One weight-gradient product of wgrad_tc, for the two-product launch.
+struct WgradArgs {
+  const void* A1;
+  int64_t a_cols, blk_a;
+  const void* A2;
+  int64_t b_cols, blk_b, nblocks;
+  int b_base, b_grp, b_gs;
+  WgradSplit sp;
+  int64_t p_stride, p_off;  // partial[split*p_stride + p_off + ...]
+};
+// dR and dL partials (or any two products) in one launch when their N tiles agree, else two.
+cudaError_t wgrad_tc2(const WgradArgs& w1, const WgradArgs& w2, int64_t rows, float* partial, int* status,
+                      cudaStream_t st);
 
 // Rt[k][i][p] = R[k][p][i] and Lt[j][c][o] = L[j][o][cmap(c)] (bf16), one launch;
 // cmap(c) = (c % G)*nb1 + c / G when G > 0, else c.
@@ -79,8 +101,10 @@ __global__ void reduce_partials_kernel(const float* __restrict__ partial, __nv_b
 
 bool packed_bwd_supported(const Shape& s);
 size_t packed_bwd_workspace(const Shape& s);
+// saved: the middle vector Z from the training forward (used when the streaming stages serve the
+// shape), or nullptr to recompute it.
 cudaError_t packed_bwd(const void* dY, const void* X, const void* R, const void* L, void* dX, void* dR, void* dL,
-                       void* ws, const Shape& s, int* status, cudaStream_t st);
+                       void* ws, const Shape& s, int* status, cudaStream_t st, const void* saved = nullptr);
 
 size_t gemm_fwd_workspace(const Shape& s);
 cudaError_t gemm_fwd(const void* X, const void* R, const void* L, void* Y, void* ws, const Shape& s, int* status,

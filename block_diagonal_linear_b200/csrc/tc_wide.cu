@@ -15,6 +15,9 @@
 //      come through a two-stage ring.
 //   4. Each round's run is staged in one of two shared-memory buffers and written with
 //      TMA tensor stores while the next round computes and drains into the other.
+// With SAVE, the middle tile Z (the L stage's input vector, bf16) is also written to global
+// memory with TMA stores as soon as the drain has built it (the training forward keeps it for
+// the backward).
 // bm (rows per unit, a multiple of 8) is chosen on the host so the units spread evenly
 // over the SMs; MMAs always cover 64 rows, and rows >= bm of a tile are never stored.
 // Roles: warp 0 TMA producer (X), warp 1 MMA issuer + TMEM owner, warps 2..9 drain,
@@ -87,11 +90,11 @@ __device__ __forceinline__ void tmem_ld4(uint32_t taddr, uint32_t (&r)[4]) {
                : "r"(taddr));
 }
 
-template <class C>
+template <class C, int SAVE>
 __global__ void __launch_bounds__(kWideThreads, 1)
     tc_wide_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmY,
-                   const __nv_bfloat16* __restrict__ R, const __nv_bfloat16* __restrict__ L,
-                   int64_t rows, int bm, int* status) {
+                   const __grid_constant__ CUtensorMap tmZ, const __nv_bfloat16* __restrict__ R,
+                   const __nv_bfloat16* __restrict__ L, int64_t rows, int bm, int* status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t* zbuf = smem;                    // X tile, then Z tile
@@ -134,6 +137,7 @@ __global__ void __launch_bounds__(kWideThreads, 1)
     if (lane == 0) {
       ptx::tma_prefetch_desc(&tmX);
       ptx::tma_prefetch_desc(&tmY);
+      if (SAVE) ptx::tma_prefetch_desc(&tmZ);
       const uint64_t pol_x = ptx::policy_evict_first();
       const uint32_t xbytes = (uint32_t)bm * 128u;
       uint32_t unit_n = 0;
@@ -288,6 +292,16 @@ __global__ void __launch_bounds__(kWideThreads, 1)
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(&bars->z_full);
       const int row0 = (int)(u * bm);
+      if (SAVE && leader) {
+        // every drain warp has written and fenced its part of Z: store the tile (rows >= bm
+        // of a tile are not part of the box)
+        if (!wait_or_abort(&bars->z_full, unit_n & 1, abort_flag, status)) {
+          ok = false;
+        } else {
+          for (int a = 0; a < C::ZATOMS; ++a) ptx::tma_store_2d(&tmZ, zbuf + a * C::ATOM, a * 64, row0);
+          ptx::bulk_commit_group();
+        }
+      }
       // ---- L-stage rounds -> staged output runs
       for (int r2 = 0; r2 < C::NR2 && ok; ++r2, ++g2) {
         const int slot = g2 & 1;
@@ -339,6 +353,9 @@ __global__ void __launch_bounds__(kWideThreads, 1)
         }
       }
       if (!ok) break;
+      // with SAVE, the next unit's X may overwrite Z only once the Z stores (the group before
+      // the last round's) have read it
+      if (SAVE && leader) ptx::bulk_wait_read_allbut1();
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(&bars->tmem_free);
       if (leader) {
@@ -368,22 +385,25 @@ static int balanced_bm(int64_t rows, int nsm) {
   return (int)bm;
 }
 
-template <class C>
-static cudaError_t launch_wide(const void* X, const void* R, const void* L, void* Y, int64_t rows,
+template <class C, int SAVE>
+static cudaError_t launch_wide(const void* X, const void* R, const void* L, void* Y, void* Z, int64_t rows,
                                int* status, cudaStream_t st) {
   if (rows == 0) return cudaSuccess;
   const int nsm = num_sms();
   const int bm = balanced_bm(rows, nsm);
-  CUtensorMap mX, mY;
+  CUtensorMap mX, mY, mZ;
   if (!make_map_2d(&mX, X, C::N_IN, (uint64_t)rows, 64, (uint32_t)bm, CU_TENSOR_MAP_SWIZZLE_128B) ||
       !make_map_2d(&mY, Y, C::N_OUT, (uint64_t)rows, 64, (uint32_t)bm, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
-  cudaError_t e = ensure_smem_attr((const void*)tc_wide_kernel<C>, C::SMEM_BYTES);
+  if (SAVE && !make_map_2d(&mZ, Z, C::N_MID, (uint64_t)rows, 64, (uint32_t)bm, CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  if (!SAVE) mZ = mY;  // unused
+  cudaError_t e = ensure_smem_attr((const void*)tc_wide_kernel<C, SAVE>, C::SMEM_BYTES);
   if (e != cudaSuccess) return e;
   const int64_t nunits = (rows + bm - 1) / bm;
   const int64_t grid = nunits < nsm ? nunits : nsm;
-  return launch_kernel(tc_wide_kernel<C>, dim3((unsigned)grid), dim3(kWideThreads), C::SMEM_BYTES, st, false,
-                       mX, mY, (const __nv_bfloat16*)R, (const __nv_bfloat16*)L, rows, bm, status);
+  return launch_kernel(tc_wide_kernel<C, SAVE>, dim3((unsigned)grid), dim3(kWideThreads), C::SMEM_BYTES, st,
+                       false, mX, mY, mZ, (const __nv_bfloat16*)R, (const __nv_bfloat16*)L, rows, bm, status);
 }
 
 using WideR768 = WideCfg<16, 48, 48, 48, 16, 64>;  // 768 -> 3072
@@ -398,7 +418,13 @@ bool tc_wide_supported(const Shape& s) { return wide_shape_is<WideR768>(s); }
 
 cudaError_t tc_wide_fwd(const void* X, const void* R, const void* L, void* Y, const Shape& s,
                         int* status, cudaStream_t st) {
-  if (wide_shape_is<WideR768>(s)) return launch_wide<WideR768>(X, R, L, Y, s.rows, status, st);
+  if (wide_shape_is<WideR768>(s)) return launch_wide<WideR768, 0>(X, R, L, Y, nullptr, s.rows, status, st);
+  return cudaErrorNotSupported;
+}
+
+cudaError_t tc_wide_fwd_save(const void* X, const void* R, const void* L, void* Y, void* Z, const Shape& s,
+                             int* status, cudaStream_t st) {
+  if (wide_shape_is<WideR768>(s)) return launch_wide<WideR768, 1>(X, R, L, Y, Z, s.rows, status, st);
   return cudaErrorNotSupported;
 }
 

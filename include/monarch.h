@@ -124,9 +124,10 @@ MONARCH_API int monarch_fwd_ws(const void* X, const void* R, const void* L, cons
  *
  * monarch_fwd_train computes Y = X * M^T exactly as monarch_fwd_ws does (same kernels, same
  * results) and leaves the middle vector of these rows in `saved`, in the layout the backward's
- * own recompute would produce: for the fused small-block forward (monarch_fwd_path 2) and the
- * streaming-stage forward (monarch_fwd_ws_path 6) the permuted middle vector Z (rows x n_mid
- * bf16, Z[r][j*in2 + q]); for the two-pass GEMM forward (monarch_fwd_ws_path 5) that
+ * own recompute would produce: for the fused small-block forward (monarch_fwd_path 2), the
+ * wide-output forward (monarch_fwd_path 3) when the backward runs the streaming stages (e.g.
+ * 768 -> 3072), and the streaming-stage forward (monarch_fwd_ws_path 6) the permuted middle
+ * vector Z (rows x n_mid bf16, Z[r][j*in2 + q]); for the two-pass GEMM forward (monarch_fwd_ws_path 5) that
  * forward's whole workspace (the reordered L, then U = blockdiag(R) X).  This is what an
  * autograd framework saves for the backward of a product of factors; it trades a write and a
  * read of rows x n_mid bf16 for the backward's recompute pass (a read of X, a write of the

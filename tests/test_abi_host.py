@@ -92,7 +92,7 @@ def test_training_pair_sizes_and_checks_before_device_work():
     assert bdl.saved_bytes(n1024, 100, "bf16") == 100 * 1024 * 2  # Z of the fused forward
     assert bdl.saved_bytes(n4096, 100, "bf16") == 100 * 4096 * 2  # Z of the streaming stages
     assert bdl.saved_bytes(nblk4, 100, "bf16") == bdl.fwd_workspace_bytes(nblk4, 100, "bf16")  # L reordered, U
-    assert bdl.saved_bytes(r768, 100, "bf16") == 0                # the backward recomputes
+    assert bdl.saved_bytes(r768, 100, "bf16") == 100 * 768 * 2   # Z of the wide-output forward
     assert bdl.saved_bytes(n1024, 100, "f32") == 0
     lib = bdl.lib()
     d = bdl.make_dims(n1024, 1000, "bf16")

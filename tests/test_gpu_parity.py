@@ -177,6 +177,27 @@ def test_tc_forward_tile_edges(name, rows):
         check(to_f64(Y), ref, "bf16", "Y")
 
 
+@pytest.mark.parametrize("name,rows", [("n1024_bf16", r) for r in (1, 129, 257)]
+                         + [("r768x3072_bf16", r) for r in (1, 63, 65, 191, 9473)]
+                         + [("n4096_bf16", r) for r in (1, 129, 1000)])
+def test_training_pair_tile_edges(name, rows):
+    """Ragged row counts: the training forward's kept middle vector (partial last tiles of the Z
+    stores) gives the backward the same results as recomputing it, bit for bit."""
+    w = W[name]
+    shape = synthetic.shape_of(w)
+    inp = synthetic.make_inputs(w, seed=31, rows=rows)
+    d = dev_inputs(inp)
+    Y1 = bdl.fwd_ws(d["X"], d["R"], d["L"], shape)
+    Y2, saved = bdl.fwd_train(d["X"], d["R"], d["L"], shape)
+    assert saved is not None
+    g1 = bdl.bwd(d["dY"], d["X"], d["R"], d["L"], shape)
+    g2 = bdl.bwd_saved(d["dY"], d["X"], d["R"], d["L"], shape, saved)
+    assert bdl.last_device_status() == 0
+    assert torch.equal(Y1, Y2)
+    for a, b, what in zip(g1, g2, ("dX", "dR", "dL")):
+        assert torch.equal(a, b), what
+
+
 def test_bwd_deterministic():
     w = W["n1024_bf16"]
     inp = synthetic.make_inputs(w, seed=9, rows=2000)
@@ -252,7 +273,7 @@ def test_stage_forward_tile_edges(name, rows):
     check(to_f64(Y), ref, "bf16", "Y")
 
 
-@pytest.mark.parametrize("name", ["n1024_bf16", "n4096_bf16", "nblk4_1024x4096_bf16"])
+@pytest.mark.parametrize("name", ["n1024_bf16", "r768x3072_bf16", "n4096_bf16", "nblk4_1024x4096_bf16"])
 def test_training_pair_matches_forward_and_backward_bitwise(name):
     """Full workload size: the training forward's Y equals monarch_fwd_ws's and the saved backward's
     dX, dR, dL equal monarch_bwd's bit for bit (the saved middle vector is the recomputed one)."""
