@@ -25,11 +25,13 @@ cudaError_t tc_rows_dual(const void* dV, const void* Lt, const void* Rt, void* d
                          const Shape& s, int* status, cudaStream_t st);
 
 // ------------------------------------------------------------------ small kernels
-// dV[r][j*out2 + o] = dY[r][o*nb2 + j]: per row an (out2 x nb2) -> (nb2 x out2)
-// transpose.  One warp per row: the row is read with 16-byte coalesced loads, staged in
-// shared memory with an odd word pitch (nb2 + 2 elements, so the column reads of the
+// dV[r][j*out2 + o] = dY[r][o*nb2 + j]: per row an (out2 x nb2) -> (nb2 x out2) element
+// transpose.  Each warp takes two rows at a time: all of both rows' 16-byte loads are issued
+// before any is used (rows of up to 1024 elements: four chunks a lane each), the rows are
+// staged in shared memory with an odd word pitch (nb2 + 2 elements, so the column reads of the
 // transpose hit 32 different banks), and written back with 16-byte coalesced stores.
 constexpr int kGatherWarps = 8;
+constexpr int kGatherChunks = 4;  // 16-byte chunks a lane loads per row (n_out <= 1024)
 __global__ void __launch_bounds__(kGatherWarps * 32)
     gather_dv_kernel(const __nv_bfloat16* __restrict__ dY, __nv_bfloat16* __restrict__ dV, Shape s) {
   extern __shared__ __align__(16) uint32_t shw[];
@@ -38,27 +40,44 @@ __global__ void __launch_bounds__(kGatherWarps * 32)
   const int n = (int)s.n_out(), nb2 = s.nb2, out2 = s.out2;
   const int pitch = nb2 + 2;          // elements per staged grid row (o)
   const int wpitch = pitch / 2;       // 32-bit words per staged grid row
+  const int nch = n / 8;              // 16-byte chunks per row (<= 32 * kGatherChunks)
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  uint32_t* buf = shw + warp * (out2 * wpitch);
-  const uint16_t* hb = (const uint16_t*)buf;
-  for (int64_t r = (int64_t)blockIdx.x * kGatherWarps + warp; r < s.rows;
-       r += (int64_t)gridDim.x * kGatherWarps) {
-    const __nv_bfloat16* src = dY + r * n;
-    for (int c = lane; c < n / 8; c += 32) {  // chunk c: o = (8c) / nb2, j0 = (8c) % nb2
-      const uint4 v = *(const uint4*)(src + c * 8);
-      const int o = (c * 8) / nb2, j0 = (c * 8) % nb2;
-      uint32_t* d = buf + o * wpitch + j0 / 2;
-      d[0] = v.x; d[1] = v.y; d[2] = v.z; d[3] = v.w;
-    }
-    __syncwarp();
-    __nv_bfloat16* dst = dV + r * n;
-    for (int c = lane; c < n / 8; c += 32) {  // output chunk: j = (8c) / out2, o0 = (8c) % out2
-      const int j = (c * 8) / out2, o0 = (c * 8) % out2;
-      uint32_t w[4];
+  uint32_t* buf = shw + warp * (2 * out2 * wpitch);
+  const int64_t stride = (int64_t)gridDim.x * kGatherWarps;
+  for (int64_t r0 = (int64_t)blockIdx.x * kGatherWarps + warp; r0 < s.rows; r0 += 2 * stride) {
+    const int64_t rr[2] = {r0, r0 + stride};
+    uint4 v[2][kGatherChunks];
 #pragma unroll
-      for (int e = 0; e < 4; ++e)
-        w[e] = (uint32_t)hb[(o0 + 2 * e) * pitch + j] | ((uint32_t)hb[(o0 + 2 * e + 1) * pitch + j] << 16);
-      *(uint4*)(dst + c * 8) = make_uint4(w[0], w[1], w[2], w[3]);
+    for (int h = 0; h < 2; ++h)
+#pragma unroll
+      for (int i = 0; i < kGatherChunks; ++i) {
+        const int c = lane + 32 * i;
+        if (rr[h] < s.rows && c < nch) v[h][i] = *(const uint4*)(dY + rr[h] * n + c * 8);
+      }
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+#pragma unroll
+      for (int i = 0; i < kGatherChunks; ++i) {
+        const int c = lane + 32 * i;  // chunk c: o = (8c) / nb2, j0 = (8c) % nb2
+        if (rr[h] < s.rows && c < nch) {
+          uint32_t* d = buf + h * (out2 * wpitch) + ((c * 8) / nb2) * wpitch + ((c * 8) % nb2) / 2;
+          d[0] = v[h][i].x; d[1] = v[h][i].y; d[2] = v[h][i].z; d[3] = v[h][i].w;
+        }
+      }
+    __syncwarp();
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      if (rr[h] >= s.rows) continue;
+      const uint16_t* hb = (const uint16_t*)(buf + h * (out2 * wpitch));
+      __nv_bfloat16* dst = dV + rr[h] * n;
+      for (int c = lane; c < nch; c += 32) {  // output chunk: j = (8c) / out2, o0 = (8c) % out2
+        const int j = (c * 8) / out2, o0 = (c * 8) % out2;
+        uint32_t w[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          w[e] = (uint32_t)hb[(o0 + 2 * e) * pitch + j] | ((uint32_t)hb[(o0 + 2 * e + 1) * pitch + j] << 16);
+        *(uint4*)(dst + c * 8) = make_uint4(w[0], w[1], w[2], w[3]);
+      }
     }
     __syncwarp();
   }
@@ -168,8 +187,9 @@ cudaError_t fast_bwd(const void* dY, const void* X, const void* R, const void* L
     }
     if ((e = bdgemm64(dU, Rt, dX, s.nb1, s.rows, status, st, true)) != cudaSuccess) return e;
   } else if (s.rows > 0) {
-    const size_t gsm = (size_t)kGatherWarps * (size_t)s.out2 * (size_t)(s.nb2 + 2) * 2;
-    if ((e = launch_kernel(gather_dv_kernel, dim3(2 * 148), dim3(kGatherWarps * 32), gsm, st, true,
+    const size_t gsm = (size_t)kGatherWarps * 2 * (size_t)s.out2 * (size_t)(s.nb2 + 2) * 2;
+    if (s.n_out() > 32 * kGatherChunks * 8) return cudaErrorInvalidValue;
+    if ((e = launch_kernel(gather_dv_kernel, dim3(4 * 148), dim3(kGatherWarps * 32), gsm, st, true,
                            (const __nv_bfloat16*)dY, dV, s)) != cudaSuccess)
       return e;
     if (saved == nullptr && (e = tc_rows_middle(X, R, Z, s, status, st)) != cudaSuccess) return e;
