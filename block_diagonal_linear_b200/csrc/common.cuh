@@ -154,7 +154,7 @@ cudaError_t tc_split_fwd(const void* X, const void* R, const void* L, void* Y, c
 cudaError_t bdgemm64(const void* X, const void* W, void* Y, int nb, int64_t rows, int* status,
                      cudaStream_t st, bool pdl);
 // dst[r][b*A + a] = src[r][a*B + b] (bf16; dst may equal src; A, B multiples of 8).
-cudaError_t permute_rows(const void* src, void* dst, int64_t rows, int A, int B, cudaStream_t st);
+cudaError_t permute_rows(const void* src, void* dst, int64_t rows, int A, int B, cudaStream_t st, bool pdl = true);
 // dst[r][b*A + a] += src[r][a*B + b] (bf16, fp32 add rounded once; dst distinct from src).
 cudaError_t permute_rows_add(const void* src, void* dst, int64_t rows, int A, int B, cudaStream_t st);
 

@@ -281,7 +281,8 @@ static cudaError_t launch_bdgemm(const void* X, const void* W, void* Y, int nb, 
 }
 
 template <bool ACC>
-static cudaError_t launch_permute(const void* src, void* dst, int64_t rows, int A, int B, cudaStream_t st) {
+static cudaError_t launch_permute(const void* src, void* dst, int64_t rows, int A, int B, cudaStream_t st,
+                                  bool pdl = true) {
   if (rows == 0) return cudaSuccess;
   // one staged row per warp: as many warps (up to 8) as shared memory holds rows
   const size_t row_smem = (size_t)A * (size_t)(B + 2) * 2;
@@ -291,12 +292,12 @@ static cudaError_t launch_permute(const void* src, void* dst, int64_t rows, int 
   const size_t smem = (size_t)nwarps * row_smem;
   cudaError_t e = ensure_smem_attr((const void*)permute_rows_kernel<ACC>, (int)smem);
   if (e != cudaSuccess) return e;
-  return launch_kernel(permute_rows_kernel<ACC>, dim3(2 * 148), dim3(nwarps * 32), smem, st, true,
+  return launch_kernel(permute_rows_kernel<ACC>, dim3(2 * 148), dim3(nwarps * 32), smem, st, pdl,
                        (const __nv_bfloat16*)src, (__nv_bfloat16*)dst, rows, A, B);
 }
 
-cudaError_t permute_rows(const void* src, void* dst, int64_t rows, int A, int B, cudaStream_t st) {
-  return launch_permute<false>(src, dst, rows, A, B, st);
+cudaError_t permute_rows(const void* src, void* dst, int64_t rows, int A, int B, cudaStream_t st, bool pdl) {
+  return launch_permute<false>(src, dst, rows, A, B, st, pdl);
 }
 
 cudaError_t permute_rows_add(const void* src, void* dst, int64_t rows, int A, int B, cudaStream_t st) {
@@ -322,10 +323,12 @@ cudaError_t tc_split_fwd(const void* X, const void* R, const void* L, void* Y, c
   if (s.rows == 0) return cudaSuccess;
   __nv_bfloat16* y = (__nv_bfloat16*)Y;
   cudaError_t e;
+  // Plain stream order here: with programmatic launch this four-pass chain measured 240 us
+  // against 216 us without (16384 rows), unlike the backward chains it speeds up.
   if ((e = launch_bdgemm<Bd64>(X, R, Y, s.nb1, s.rows, status, st, false)) != cudaSuccess) return e;
-  if ((e = permute_rows(y, y, s.rows, s.nb1, s.out1, st)) != cudaSuccess) return e;
-  if ((e = launch_bdgemm<Bd64>(Y, L, Y, s.nb2, s.rows, status, st, true)) != cudaSuccess) return e;
-  if (s.out_transpose) return permute_rows(y, y, s.rows, s.nb2, s.out2, st);
+  if ((e = permute_rows(y, y, s.rows, s.nb1, s.out1, st, false)) != cudaSuccess) return e;
+  if ((e = launch_bdgemm<Bd64>(Y, L, Y, s.nb2, s.rows, status, st, false)) != cudaSuccess) return e;
+  if (s.out_transpose) return permute_rows(y, y, s.rows, s.nb2, s.out2, st, false);
   return cudaSuccess;
 }
 
