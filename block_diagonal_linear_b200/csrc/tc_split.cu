@@ -219,10 +219,12 @@ __global__ void __launch_bounds__(kBdThreads, 1)
 
 // dst[r][b*A + a] = src[r][a*B + b]: per row an (A x B) -> (B x A) transpose.  One warp per
 // row: the whole row is read with 16-byte loads into shared memory (odd word pitch, so the
-// column reads hit 32 banks) before any of it is written, so src may equal dst.
+// column reads hit 32 banks) before any of it is written, so src may equal dst.  With CH > 0
+// (rows of at most CH * 256 elements) a lane issues all of its CH loads before storing any, so
+// a warp keeps the whole row in flight; CH = 0 is the plain loop for longer rows.
 // With ACC, dst[r][b*A + a] = round(dst[r][b*A + a] + src[r][a*B + b]) (src and dst distinct).
 constexpr int kPermWarps = 8;
-template <bool ACC>
+template <bool ACC, int CH>
 __global__ void __launch_bounds__(kPermWarps * 32)
     permute_rows_kernel(const __nv_bfloat16* src, __nv_bfloat16* dst, int64_t rows, int A, int B) {
   extern __shared__ __align__(16) uint32_t shw[];
@@ -235,10 +237,27 @@ __global__ void __launch_bounds__(kPermWarps * 32)
   const int nwarps = blockDim.x / 32;  // one staged row per warp
   for (int64_t r = (int64_t)blockIdx.x * nwarps + warp; r < rows; r += (int64_t)gridDim.x * nwarps) {
     const __nv_bfloat16* s = src + r * n;
-    for (int c = lane; c < n / 8; c += 32) {  // source chunk: a = 8c / B, b0 = 8c % B
-      const uint4 v = *(const uint4*)(s + c * 8);
-      uint32_t* d = buf + ((c * 8) / B) * wpitch + ((c * 8) % B) / 2;
-      d[0] = v.x; d[1] = v.y; d[2] = v.z; d[3] = v.w;
+    if (CH > 0) {
+      uint4 v[CH > 0 ? CH : 1];
+#pragma unroll
+      for (int i = 0; i < CH; ++i) {
+        const int c = lane + 32 * i;
+        if (c < n / 8) v[i] = *(const uint4*)(s + c * 8);
+      }
+#pragma unroll
+      for (int i = 0; i < CH; ++i) {
+        const int c = lane + 32 * i;  // source chunk: a = 8c / B, b0 = 8c % B
+        if (c < n / 8) {
+          uint32_t* d = buf + ((c * 8) / B) * wpitch + ((c * 8) % B) / 2;
+          d[0] = v[i].x; d[1] = v[i].y; d[2] = v[i].z; d[3] = v[i].w;
+        }
+      }
+    } else {
+      for (int c = lane; c < n / 8; c += 32) {  // source chunk: a = 8c / B, b0 = 8c % B
+        const uint4 v = *(const uint4*)(s + c * 8);
+        uint32_t* d = buf + ((c * 8) / B) * wpitch + ((c * 8) % B) / 2;
+        d[0] = v.x; d[1] = v.y; d[2] = v.z; d[3] = v.w;
+      }
     }
     __syncwarp();
     __nv_bfloat16* d = dst + r * n;
@@ -290,9 +309,13 @@ static cudaError_t launch_permute(const void* src, void* dst, int64_t rows, int 
   if (row_smem > cap) return cudaErrorInvalidValue;
   const int nwarps = (int)std::min<size_t>(kPermWarps, cap / row_smem);
   const size_t smem = (size_t)nwarps * row_smem;
-  cudaError_t e = ensure_smem_attr((const void*)permute_rows_kernel<ACC>, (int)smem);
+  const int64_t nch = (int64_t)A * B / 8;  // 16-byte chunks per row
+  auto kern = nch <= 32 * 4 ? permute_rows_kernel<ACC, 4>
+              : nch <= 32 * 8 ? permute_rows_kernel<ACC, 8>
+              : nch <= 32 * 16 ? permute_rows_kernel<ACC, 16> : permute_rows_kernel<ACC, 0>;
+  cudaError_t e = ensure_smem_attr((const void*)kern, (int)smem);
   if (e != cudaSuccess) return e;
-  return launch_kernel(permute_rows_kernel<ACC>, dim3(2 * 148), dim3(nwarps * 32), smem, st, pdl,
+  return launch_kernel(kern, dim3(2 * 148), dim3(nwarps * 32), smem, st, pdl,
                        (const __nv_bfloat16*)src, (__nv_bfloat16*)dst, rows, A, B);
 }
 
