@@ -517,6 +517,26 @@ __global__ void pack_weights_kernel(const __nv_bfloat16* __restrict__ R, const _
   }
 }
 
+// The factors the streaming-stage form of the packed backward needs, in one launch:
+// Wx as in pack_weights_kernel (the packed dX stage) and Lt[j][c][o] = L[j][o][c] (the L^T stage).
+__global__ void pack_staged_kernel(const __nv_bfloat16* __restrict__ R, const __nv_bfloat16* __restrict__ L,
+                                   __nv_bfloat16* __restrict__ Wx, __nv_bfloat16* __restrict__ Lt, Shape s, int gx) {
+  ptx::griddep_wait();
+  ptx::griddep_launch_dependents();
+  const int64_t nx = (int64_t)s.nb1 * s.in1 * gx * s.out1, nL = s.n_L();
+  const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (e < nx) {
+    const int64_t kw = (int64_t)gx * s.out1, n = e / kw, k = e % kw;
+    const int64_t g = n / ((int64_t)gx * s.in1), nn = n % ((int64_t)gx * s.in1);
+    const int kk = (int)(nn / s.in1), i = (int)(nn % s.in1), kq = (int)(k / s.out1), p = (int)(k % s.out1);
+    Wx[e] = kk == kq ? R[((g * gx + kk) * s.out1 + p) * s.in1 + i] : __float2bfloat16_rn(0.f);
+  } else if (e < nx + nL) {
+    const int64_t f = e - nx, per = (int64_t)s.in2 * s.out2, j = f / per, rem = f % per;
+    const int c = (int)(rem / s.out2), o = (int)(rem % s.out2);
+    Lt[f] = L[(j * s.out2 + o) * s.in2 + c];
+  }
+}
+
 // Wp[grp][jj*nw + n][jj'*kw + k] = W[grp*g + jj][n][k] if jj == jj' (else 0), from W (nb, nw, kw);
 // with trans, W is read as (nb, kw, nw) and transposed: Wp[...][jj*nw + n][jj*kw + k] = W[b][k][n].
 __global__ void pack_bd_kernel(const __nv_bfloat16* __restrict__ W, __nv_bfloat16* __restrict__ Wp, int nb,
@@ -600,18 +620,21 @@ cudaError_t packed_bwd(const void* dY, const void* X, const void* R, const void*
   const int64_t nR = s.n_R(), nL = s.n_L(), nP = nR + nL;
   const int64_t nz = (int64_t)s.nb2 * s.in2 * pk.gz * s.out2, nx = (int64_t)s.nb1 * s.in1 * pk.gx * s.out1;
   cudaError_t e;
-  if ((e = launch_kernel(pack_weights_kernel, dim3((unsigned)((nz + 2 * nx + 255) / 256)), dim3(256), 0, st, true,
-                         (const __nv_bfloat16*)R, (const __nv_bfloat16*)L, Wz, Wx, Wu, s, pk.gz, pk.gx)) !=
-      cudaSuccess)
-    return e;
   const bool staged = tc_stage_supported(s);
+  if (staged) {
+    // the streaming stages take the plain L^T (into the otherwise unused packed L^T region); only
+    // the dX stage is packed
+    if (s.rows > 0 &&
+        (e = launch_kernel(pack_staged_kernel, dim3((unsigned)((nx + nL + 255) / 256)), dim3(256), 0, st, true,
+                           (const __nv_bfloat16*)R, (const __nv_bfloat16*)L, Wx, Wz, s, pk.gx)) != cudaSuccess)
+      return e;
+  } else if ((e = launch_kernel(pack_weights_kernel, dim3((unsigned)((nz + 2 * nx + 255) / 256)), dim3(256), 0, st,
+                                true, (const __nv_bfloat16*)R, (const __nv_bfloat16*)L, Wz, Wx, Wu, s, pk.gz,
+                                pk.gx)) != cudaSuccess) {
+    return e;
+  }
   if (saved != nullptr && staged) Z = (__nv_bfloat16*)saved;  // kept by the training forward
   const bool need_z = saved == nullptr || !staged;
-  if (staged && s.rows > 0) {
-    // the streaming stages take the plain factors: L^T into the (then unused) packed L^T
-    // region, R^T into the packed-R region (the transpose helper writes both)
-    if ((e = factor_transposes(R, Wu, L, Wz, s, 0, st, false)) != cudaSuccess) return e;
-  }
   if (s.rows > 0) {
     if (s.out_transpose && (e = permute_rows(dY, dV, s.rows, s.out2, s.nb2, st)) != cudaSuccess) return e;
     if (staged) {
