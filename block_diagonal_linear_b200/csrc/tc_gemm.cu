@@ -443,6 +443,12 @@ cudaError_t gemm_bd(const void* A, int64_t rows, int64_t a_cols, const void* W, 
 }
 
 // Operand maps of one weight-gradient job; sets job.ab3d, kind, rows, widths and units.
+// CTA-pair kernel (tc_wgrad2.cu); the caller builds 3-D operand maps whose B box is two 64-column
+// chunks.
+cudaError_t launch_wgrad_pair(const CUtensorMap& mA, const CUtensorMap& mB, GemmJob job, const CUtensorMap& mA2,
+                              const CUtensorMap& mB2, GemmJob job2, float* partial, int* status, cudaStream_t st,
+                              bool pdl);
+
 static bool wgrad_maps(const void* A1, int64_t a_cols, const void* A2, int64_t b_cols, int64_t rows, int BN,
                        GemmJob* job, CUtensorMap* mA, CUtensorMap* mB) {
   // Multi-chunk boxes need every unit's operand columns to start on a 64-column chunk and a
@@ -495,9 +501,38 @@ cudaError_t gemm_wgrad(const void* A1, int64_t a_cols, const void* A2, int64_t b
   return launch_wgrad(BN, mA, mB, job, mA, mB, none, partial, status, st, pdl);
 }
 
+// Operand maps of a CTA-pair job: A as (64 columns, rows, 64-column chunks) with two-chunk boxes;
+// B likewise when a pair of its chunks is contiguous (ab3d = 1), else (columns, rows) with
+// one-chunk boxes (ab3d = 0).  Sets kind, rows, widths; units are set by the pair launch.
+static bool pair_maps(const WgradOperands& o, int64_t rows, GemmJob* job, CUtensorMap* mA, CUtensorMap* mB) {
+  if (o.a_cols % 64 || job->a_b % 64) return false;
+  const uint64_t da[3] = {64, (uint64_t)rows, (uint64_t)o.a_cols / 64}, sa_[2] = {(uint64_t)o.a_cols * 2, 128};
+  const uint32_t box2[3] = {64, 64, 2};
+  if (!make_map_3d(mA, o.A1, da, sa_, box2, CU_TENSOR_MAP_SWIZZLE_128B)) return false;
+  const bool b_pairs = job->b_grp >= (1 << 29) || (job->b_grp % 2 == 0 && job->b_gs % 64 == 0);
+  job->ab3d = (o.b_cols % 64 == 0 && job->b_b % 64 == 0 && b_pairs) ? 1 : 0;
+  if (job->ab3d) {
+    const uint64_t db[3] = {64, (uint64_t)rows, (uint64_t)o.b_cols / 64}, sb_[2] = {(uint64_t)o.b_cols * 2, 128};
+    if (!make_map_3d(mB, o.A2, db, sb_, box2, CU_TENSOR_MAP_SWIZZLE_128B)) return false;
+  } else if (!make_map_2d(mB, o.A2, (uint64_t)o.b_cols, (uint64_t)rows, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B)) {
+    return false;
+  }
+  job->kind = 1;
+  job->rows = rows;
+  job->a_cols = o.a_cols;
+  job->b_cols = o.b_cols;
+  return true;
+}
+
 cudaError_t gemm_wgrad2(const WgradOperands& o1, GemmJob job1, const WgradOperands& o2, GemmJob job2,
                         int64_t rows, int BN, float* partial, int* status, cudaStream_t st, bool pdl) {
   CUtensorMap mA, mB, mA2, mB2;
+  if (wgrad_pair_ok(job1, BN) && wgrad_pair_ok(job2, BN)) {
+    // M tiles of 256 on CTA pairs: each CTA loads 128 columns of A and two 64-column chunks of B
+    GemmJob p1 = job1, p2 = job2;
+    if (pair_maps(o1, rows, &p1, &mA, &mB) && pair_maps(o2, rows, &p2, &mA2, &mB2))
+      return launch_wgrad_pair(mA, mB, p1, mA2, mB2, p2, partial, status, st, pdl);
+  }
   if (!wgrad_maps(o1.A1, o1.a_cols, o1.A2, o1.b_cols, rows, BN, &job1, &mA, &mB) ||
       !wgrad_maps(o2.A1, o2.a_cols, o2.A2, o2.b_cols, rows, BN, &job2, &mA2, &mB2))
     return cudaErrorInvalidValue;
