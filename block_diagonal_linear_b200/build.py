@@ -12,7 +12,7 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libmonarch.so")
-SOURCES = ["api.cu", "generic.cu", "tc_fwd.cu", "tc_rows.cu", "tc_wide.cu", "tc_split.cu", "tc_stage.cu", "tc_gemm.cu", "tc_wgrad2.cu",
+SOURCES = ["api.cu", "generic.cu", "tc_fwd.cu", "tc_rows.cu", "tc_wide.cu", "tc_split.cu", "tc_stage.cu", "tc_gemm.cu", "tc_pair.cu",
            "bwd_fast.cu", "bwd_gemm.cu", "linear.cu", "project.cu", "dyad.cu", "lattice.cu", "noalloc.cu"]
 HEADERS = ["common.cuh", "ptx.cuh", "tc_common.cuh", "tc_gemm.cuh"]
 

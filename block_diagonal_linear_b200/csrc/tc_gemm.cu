@@ -31,6 +31,14 @@
 
 namespace monarch {
 
+// CTA-pair kernels (tc_pair.cu).  launch_wgrad_pair: the caller builds 3-D operand maps whose B
+// box is two 64-column chunks.  gemm_bd_pair: a kind-0 job with BN = 256 (maps built inside).
+cudaError_t launch_wgrad_pair(const CUtensorMap& mA, const CUtensorMap& mB, GemmJob job, const CUtensorMap& mA2,
+                              const CUtensorMap& mB2, GemmJob job2, float* partial, int* status, cudaStream_t st,
+                              bool pdl);
+cudaError_t gemm_bd_pair(const void* A, int64_t rows, int64_t a_cols, const void* W, int64_t w_rows, int K, void* Y,
+                         int64_t y_cols, GemmJob job, int* status, cudaStream_t st, bool pdl);
+
 constexpr int kGemmThreads = 192;
 constexpr int kGemmEpiWarps = 4;
 
@@ -407,6 +415,15 @@ static cudaError_t launch_stage_cfg(const CUtensorMap& mA, const CUtensorMap& mB
 cudaError_t gemm_bd(const void* A, int64_t rows, int64_t a_cols, const void* W, int64_t w_rows, int K,
                     void* Y, int64_t y_cols, int BN, GemmJob job, int* status, cudaStream_t st, bool pdl) {
   if (rows == 0) return cudaSuccess;
+  {
+    // streamed 256-wide weight tiles (no resident configuration) with enough 256-row units to
+    // fill the SM pairs: run on CTA pairs, each SM loading half of every weight stage
+    const int64_t mt128 = (rows + 127) / 128, nwg = (int64_t)job.nb * job.ntiles;
+    const bool stationary = mt128 >= 2 * ((num_sms() / nwg) > 0 ? (num_sms() / nwg) : 1);
+    const bool resident = stationary && BN == 256 && (job.kboxes == 4 || job.kboxes == 2);
+    if (BN == 256 && !resident && (rows + 255) / 256 * nwg >= num_sms() / 2)
+      return gemm_bd_pair(A, rows, a_cols, W, w_rows, K, Y, y_cols, job, status, st, pdl);
+  }
   CUtensorMap mA, mB, mY;
   if (!make_map_2d(&mA, A, (uint64_t)a_cols, (uint64_t)rows, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
       !make_map_2d(&mB, W, (uint64_t)K, (uint64_t)w_rows, 64, (uint32_t)BN, CU_TENSOR_MAP_SWIZZLE_128B) ||
@@ -443,11 +460,6 @@ cudaError_t gemm_bd(const void* A, int64_t rows, int64_t a_cols, const void* W, 
 }
 
 // Operand maps of one weight-gradient job; sets job.ab3d, kind, rows, widths and units.
-// CTA-pair kernel (tc_wgrad2.cu); the caller builds 3-D operand maps whose B box is two 64-column
-// chunks.
-cudaError_t launch_wgrad_pair(const CUtensorMap& mA, const CUtensorMap& mB, GemmJob job, const CUtensorMap& mA2,
-                              const CUtensorMap& mB2, GemmJob job2, float* partial, int* status, cudaStream_t st,
-                              bool pdl);
 
 static bool wgrad_maps(const void* A1, int64_t a_cols, const void* A2, int64_t b_cols, int64_t rows, int BN,
                        GemmJob* job, CUtensorMap* mA, CUtensorMap* mB) {

@@ -59,7 +59,7 @@ struct WgradOperands {
 };
 cudaError_t gemm_wgrad2(const WgradOperands& o1, GemmJob job1, const WgradOperands& o2, GemmJob job2,
                         int64_t rows, int BN, float* partial, int* status, cudaStream_t st, bool pdl);
-// CTA-pair form of a two-job kind-1 launch (tc_wgrad2.cu): BN = 256, M side of each group a
+// CTA-pair form of a two-job kind-1 launch (tc_pair.cu): BN = 256, M side of each group a
 // multiple of 256, one N tile (launch_wgrad_pair, declared where tensor maps are known).
 bool wgrad_pair_ok(const GemmJob& j, int BN);
 

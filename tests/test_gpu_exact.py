@@ -32,6 +32,8 @@ CASES = [
     ("r768x3072_wide", synthetic.shape_of(W["r768x3072_bf16"]), "bf16", 300, 3, 3),
     ("n4096_split", synthetic.shape_of(W["n4096_bf16"]), "bf16", 300, 4, 1),
     ("nblk4_group", synthetic.shape_of(W["nblk4_1024x4096_bf16"]), "bf16", 300, 1, 2),
+    # enough rows for the CTA-pair kernels (weight gradient and the streamed-weight dU stage)
+    ("nblk4_pairs", synthetic.shape_of(W["nblk4_1024x4096_bf16"]), "bf16", 5003, 1, 2),
     # G = in2 / nb1 = 128: two 64-column groups per R block in the gathers
     ("nblk2_gemm", dict(nb1=2, in1=128, out1=256, nb2=2, in2=256, out2=384, out_transpose=0), "bf16", 300, 0, 2),
     ("odd_generic_bf16", ODD, "bf16", 203, 0, 0),
@@ -86,6 +88,12 @@ def test_backward_exact(case):
     _, shape, dtype, rows, _, bpath = case
     assert bdl.bwd_path(shape, dtype) == bpath
     inp = synthetic.make_sparse_sign_inputs(dict(shape, rows=rows), seed=22)
+    if rows > 1000:
+        # the weight gradients sum over rows: keep every 25th row live (all tiles and row splits
+        # still run) so that those sums stay in the exact bf16 integer range
+        dead = np.arange(rows) % 25 != 0
+        inp["X"][dead] = 0.0
+        inp["dY"][dead] = 0.0
     _check_exact_range(inp)
     refs = oracle.backward(shape, inp["dY"], inp["X"], inp["R"], inp["L"])
     for r in refs:
