@@ -107,7 +107,7 @@ def test_backward_exact(case):
             what, len(bad), tuple(bad[0]), g[tuple(bad[0])], r[tuple(bad[0])])
 
 
-WS_PATHS = {"nblk4_group": 5, "nblk2_gemm": 5, "n4096_split": 6}
+WS_PATHS = {"nblk4_group": 5, "nblk4_pairs": 5, "nblk2_gemm": 5, "n4096_split": 6}
 
 
 @pytest.mark.parametrize("case", [c for c in CASES if c[0] in WS_PATHS], ids=_ids)
