@@ -71,7 +71,7 @@ enum {
   MONARCH_ERR_WORKSPACE = -5,   /* workspace NULL or smaller than required */
   MONARCH_ERR_CUDA = -6,        /* a CUDA runtime call or kernel launch failed */
   MONARCH_ERR_TIMEOUT = -7,     /* a bounded device wait gave up (device status) */
-  MONARCH_ERR_UNSUPPORTED = -8, /* shape too large for any kernel of this build */
+  MONARCH_ERR_UNSUPPORTED = -8, /* shape too large for any kernel of this library */
   MONARCH_ERR_SCRATCH = -9,     /* monarch_bwd_noalloc: problem needs more than its fixed scratch */
   MONARCH_ERR_ALIAS = -10       /* an output (or the workspace) overlaps an input or another output */
 };
