@@ -114,7 +114,7 @@ bool fast_bwd_supported(const Shape& s) { return is_fast_square(s) || is_split_s
 
 // Weight-gradient units per row split: 128-column groups of dR and of dL.
 static WgradSplit wg_split(const Shape& s) {
-  return wgrad_split(s.rows, s.n_mid() / 128 + s.n_out() / 128);
+  return wgrad_split_wave(s.rows, s.n_mid() / 128 + s.n_out() / 128);
 }
 
 static size_t al256(size_t b) { return (b + 255) & ~size_t(255); }

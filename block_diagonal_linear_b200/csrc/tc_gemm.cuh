@@ -69,6 +69,7 @@ struct WgradSplit {
   int64_t rows_per_split;
 };
 WgradSplit wgrad_split(int64_t rows, int64_t units_per_split);
+WgradSplit wgrad_split_wave(int64_t rows, int64_t units_per_split);
 cudaError_t wgrad_tc(const void* A1, int64_t a_cols, int64_t blk_a, const void* A2, int64_t b_cols, int64_t blk_b,
                      int64_t nblocks, int b_base, int b_grp, int b_gs, int64_t rows, WgradSplit sp, float* partial,
                      int64_t p_stride, int64_t p_off, int* status, cudaStream_t st);
