@@ -577,7 +577,7 @@ static PackedWs packed_layout(const Shape& s) {
   const PackInfo pk = pack_info(s);
   PackedWs w;
   const size_t rows = (size_t)s.rows;
-  w.sp = wgrad_split(s.rows, wgrad_units(s.nb1, s.out1, s.in1) + wgrad_units(s.nb2, s.out2, s.in2));
+  w.sp = wgrad_split_wave(s.rows, wgrad_units(s.nb1, s.out1, s.in1) + wgrad_units(s.nb2, s.out2, s.in2));
   w.wz = 0;
   w.wx = w.wz + al256((size_t)s.nb2 * s.in2 * pk.gz * s.out2 * 2);
   w.wu = w.wx + al256((size_t)s.nb1 * s.in1 * pk.gx * s.out1 * 2);
