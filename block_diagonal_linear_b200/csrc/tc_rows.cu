@@ -1,7 +1,7 @@
-// Fused Monarch forward for small blocks (out1, out2 <= 32): one 64-row tile of
-// X per unit and the whole middle vector on chip, on the tcgen05 tensor cores.
+// Fused Monarch forward for small blocks (out1, out2 <= 32): one row tile of X (at most 64 rows)
+// per unit and the whole middle vector on chip, on the tcgen05 tensor cores.
 //
-// Per unit (64 rows):
+// Per unit (bm <= 64 rows; the MMAs always cover 64, rows >= bm of a tile are never stored):
 //   1. R stage: X tile (TMA, 128B swizzle, 64-column boxes) x R[k]^T, M = 64 MMAs.
 //      A round covers 16 blocks k: blocks k0..k0+7 accumulate at TMEM lane offset 0
 //      and k0+8..k0+15 at lane offset 16 (the two halves of the M = 64 data-path
@@ -100,7 +100,7 @@ __global__ void __launch_bounds__(kRowsThreads, 1)
     tc_rows_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmY,
                    const __grid_constant__ CUtensorMap tmZ,
                    const __nv_bfloat16* __restrict__ R, const __nv_bfloat16* __restrict__ L,
-                   int64_t rows, int* status) {
+                   int64_t rows, int bm, int* status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t* zbuf = smem;  // Z tile, later the output staging tile
@@ -109,7 +109,7 @@ __global__ void __launch_bounds__(kRowsThreads, 1)
   int* abort_flag = &bars->abort_flag;
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int64_t nunits = (rows + C::BM - 1) / C::BM;
+  const int64_t nunits = (rows + bm - 1) / bm;  // units of bm <= 64 rows (MMAs always cover 64)
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::NSTAGE; ++i) {
@@ -152,17 +152,17 @@ __global__ void __launch_bounds__(kRowsThreads, 1)
       uint32_t it = 0;
       bool ok = true;
       for (int64_t u = blockIdx.x; u < nunits && ok; u += gridDim.x) {
-        const int row0 = (int)(u * C::BM);
+        const int row0 = (int)(u * bm);
         for (int b = 0; b < C::NXB; ++b, ++it) {
           const int st = it % C::NSTAGE;
           if (!wait_or_abort(&bars->empty[st], ((it / C::NSTAGE) & 1) ^ 1, abort_flag, status)) { ok = false; break; }
-          ptx::mbar_arrive_expect_tx(&bars->full[st], C::XBOX_BYTES);
+          ptx::mbar_arrive_expect_tx(&bars->full[st], (uint32_t)bm * 128u);  // a box of bm rows
           ptx::tma_load_2d(ring + st * C::STAGE_BYTES, &tmX, &bars->full[st], b * 64, row0, pol_x);
         }
         // this unit's X is on its way: pull the next unit's X tile into L2 now, so that HBM
         // streams it during this unit's L stage and stores instead of after them
         if (ok && u + gridDim.x < nunits)
-          for (int b = 0; b < C::NXB; ++b) ptx::tma_prefetch_l2_2d(&tmX, b * 64, (int)((u + gridDim.x) * C::BM));
+          for (int b = 0; b < C::NXB; ++b) ptx::tma_prefetch_l2_2d(&tmX, b * 64, (int)((u + gridDim.x) * bm));
         for (int sp = 0; sp < C::NSTAGE2 && ok; ++sp, ++it) {
           const int st = it % C::NSTAGE;
           if (!wait_or_abort(&bars->empty[st], ((it / C::NSTAGE) & 1) ^ 1, abort_flag, status)) { ok = false; break; }
@@ -344,7 +344,7 @@ __global__ void __launch_bounds__(kRowsThreads, 1)
           if (!wait_or_abort(&bars->staged, unit_n & 1, abort_flag, status)) {
             ok = false;
           } else {
-            const int row0 = (int)(u * C::BM);
+            const int row0 = (int)(u * bm);
             for (int a = 0; a < C::ZATOMS; ++a) ptx::tma_store_2d(&tmZ, zbuf + a * C::ATOM_BYTES, a * 64, row0);
             ptx::bulk_commit_group();
           }
@@ -358,7 +358,7 @@ __global__ void __launch_bounds__(kRowsThreads, 1)
         if (leader) {
           // `staged` completes twice per unit in this mode: phase 2n (middle tile), 2n+1 (Y)
           if (wait_or_abort(&bars->staged, 0u, abort_flag, status)) {
-            const int row0 = (int)(u * C::BM);
+            const int row0 = (int)(u * bm);
             for (int a = 0; a < C::ZATOMS; ++a) ptx::tma_store_2d(&tmZ, zbuf + a * C::ATOM_BYTES, a * 64, row0);
             ptx::bulk_commit_group();
             ptx::bulk_wait_read_all();
@@ -417,7 +417,7 @@ __global__ void __launch_bounds__(kRowsThreads, 1)
         if (!wait_or_abort(&bars->staged, C::MODE == 1 ? 1u : (unit_n & 1), abort_flag, status)) {
           ok = false;
         } else {
-          const int row0 = (int)(u * C::BM);
+          const int row0 = (int)(u * bm);
           for (int a = 0; a < C::OATOMS; ++a) ptx::tma_store_2d(&tmY, zbuf + a * C::ATOM_BYTES, a * 64, row0);
           ptx::bulk_commit_group();
         }
@@ -435,28 +435,43 @@ __global__ void __launch_bounds__(kRowsThreads, 1)
 // Run one row-tile kernel.  X: (rows, N_IN) input; W1 (nb1, out1, in1) and W2
 // (nb2, out2, in2) the stage weights in the forward layout; Y (rows, N_OUT) output
 // (MODE 0/1); Zout (rows, N_MID) middle tile (MODE 1/2).
+// Rows per unit: a multiple of 8, at most 64, chosen so the units fill the SMs in as few equal
+// waves as possible (16384 rows on 148 SMs: 56-row units, two a CTA, against 64-row units of which
+// 40 CTAs get one and 108 get two).  A unit's time is its dependency chain, so the slowest CTA
+// sets the kernel's.
+static int rows_unit_bm(int64_t rows, int nsm) {
+  const int64_t per_wave = (int64_t)64 * nsm;
+  const int64_t waves = (rows + per_wave - 1) / per_wave;
+  const int64_t per_unit = (rows + waves * nsm - 1) / (waves * nsm);
+  int64_t bm = (per_unit + 7) / 8 * 8;
+  if (bm > 64) bm = 64;
+  if (bm < 8) bm = 8;
+  return (int)bm;
+}
+
 template <class C>
 static cudaError_t launch_rows(const void* X, const void* W1, const void* W2, void* Y, void* Zout,
                                int64_t rows, int* status, cudaStream_t st, bool pdl = false) {
   if (rows == 0) return cudaSuccess;
+  const int bm = rows_unit_bm(rows, num_sms());
   CUtensorMap mX, mY, mZ;
-  if (!make_map_2d(&mX, X, C::N_IN, (uint64_t)rows, 64, C::BM, CU_TENSOR_MAP_SWIZZLE_128B))
+  if (!make_map_2d(&mX, X, C::N_IN, (uint64_t)rows, 64, (uint32_t)bm, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
   mY = mX;
   mZ = mX;
   if (C::MODE != 2 &&
-      !make_map_2d(&mY, Y, C::N_OUT, (uint64_t)rows, 64, C::BM, CU_TENSOR_MAP_SWIZZLE_128B))
+      !make_map_2d(&mY, Y, C::N_OUT, (uint64_t)rows, 64, (uint32_t)bm, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
   if (C::MODE != 0 &&
-      !make_map_2d(&mZ, Zout, C::N_MID, (uint64_t)rows, 64, C::BM, CU_TENSOR_MAP_SWIZZLE_128B))
+      !make_map_2d(&mZ, Zout, C::N_MID, (uint64_t)rows, 64, (uint32_t)bm, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
   cudaError_t e = ensure_smem_attr((const void*)tc_rows_kernel<C>, C::SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  const int64_t nunits = (rows + C::BM - 1) / C::BM;
+  const int64_t nunits = (rows + bm - 1) / bm;
   int64_t grid = num_sms();
   if (grid > nunits) grid = nunits;
   return launch_kernel(tc_rows_kernel<C>, dim3((unsigned)grid), dim3(kRowsThreads), C::SMEM_BYTES, st,
-                       pdl, mX, mY, mZ, (const __nv_bfloat16*)W1, (const __nv_bfloat16*)W2, rows, status);
+                       pdl, mX, mY, mZ, (const __nv_bfloat16*)W1, (const __nv_bfloat16*)W2, rows, bm, status);
 }
 
 using RowsSq16 = RowsCfg<16, 16, 16, 16, 16, 16, 1>;  // n = 256 = 16^2
