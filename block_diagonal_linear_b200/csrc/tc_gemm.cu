@@ -415,6 +415,11 @@ static cudaError_t launch_stage_cfg(const CUtensorMap& mA, const CUtensorMap& mB
 cudaError_t gemm_bd(const void* A, int64_t rows, int64_t a_cols, const void* W, int64_t w_rows, int K,
                     void* Y, int64_t y_cols, int BN, GemmJob job, int* status, cudaStream_t st, bool pdl) {
   if (rows == 0) return cudaSuccess;
+  // few rows (e.g. 1000): narrower N tiles, so that the units cover more of the SMs
+  while (BN > 64 && (rows + 127) / 128 * job.nb * job.ntiles < num_sms() / 2) {
+    BN /= 2;
+    job.ntiles *= 2;
+  }
   {
     // streamed 256-wide weight tiles (no resident configuration) with enough 256-row units to
     // fill the SM pairs: run on CTA pairs, each SM loading half of every weight stage
