@@ -3,13 +3,15 @@
 // a 1e-5 normwise tolerance), shapes that have no tcgen05 instantiation, and
 // the backward until a fused tensor-core backward covers the shape.
 //
-// Forward (one CTA = up to kMaxRows rows, whole row in shared memory):
+// Forward (one CTA = up to kMaxRows rows, whole row in shared memory; few rows spread over
+// more CTAs so that small problems still use many SMs):
 //   xs <- X rows;  zs[r][p*nb1+k] = sum_i R[k][p][i] xs[r][k*in1+i]
 //   (the permutation P is the store index); y[out_index(j,o)] = sum_q L[j][o][q] zs[r][j*in2+q].
 // Backward: a row kernel recomputes Z, forms dZ = L^T dV and dX = R^T dU, and
 // spills Z and dZ (fp32) to the workspace; a weight-gradient kernel reduces
 // dR and dL over row splits; a final kernel sums the splits in fixed order.
 #include "common.cuh"
+#include "tc_common.cuh"
 
 namespace monarch {
 
@@ -23,9 +25,39 @@ static int gen_rows_per_cta(int64_t floats_per_row) {
   return (int)r;
 }
 
+// Rows per CTA for a launch over `rows` rows: the shared-memory limit, but no more than one
+// wave of CTAs needs (every row of a CTA is computed the same way, so this changes no result).
+static int gen_rows_for(int64_t rows, int64_t floats_per_row) {
+  const int cap = gen_rows_per_cta(floats_per_row);
+  const int64_t wave = (rows + num_sms() - 1) / num_sms();
+  return (int)(wave < 1 ? 1 : (wave < cap ? wave : cap));
+}
+
 bool generic_fwd_supported(const Shape& s) { return gen_rows_per_cta(s.n_in() + s.n_mid()) >= 1; }
 bool generic_bwd_supported(const Shape& s) {
   return gen_rows_per_cta(s.n_in() + s.n_out() + 2 * s.n_mid()) >= 1;
+}
+
+// acc[r] = fma(w[t*ws], act[r*rs + t*ts], acc[r]) for t = 0, 1, ..., n-1 in that order (r < nr).
+// The weights are loaded four at a time before their FMAs, so their load latencies overlap
+// instead of following one another.
+template <typename T>
+__device__ __forceinline__ void fma_rows(float (&acc)[kMaxRows], const T* __restrict__ w, int64_t ws,
+                                         const float* act, int64_t rs, int64_t ts, int n, int nr) {
+  for (int t0 = 0; t0 < n; t0 += 4) {
+    float wv[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) wv[u] = t0 + u < n ? ld_as_f32(w + (int64_t)(t0 + u) * ws) : 0.f;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      if (t0 + u < n) {
+        const float* a = act + (int64_t)(t0 + u) * ts;
+#pragma unroll
+        for (int r = 0; r < kMaxRows; ++r)
+          if (r < nr) acc[r] = fmaf(wv[u], a[r * rs], acc[r]);
+      }
+    }
+  }
 }
 
 // zs[r][p*nb1 + k] = sum_i R[k][p][i] * xs[r][k*in1 + i] for r < nr  (steps a1..a3)
@@ -38,14 +70,7 @@ __device__ void gen_stage_R(const T* __restrict__ R, const float* xs, float* zs,
     float acc[kMaxRows];
 #pragma unroll
     for (int r = 0; r < kMaxRows; ++r) acc[r] = 0.f;
-    const T* Rkp = R + idx * s.in1;
-    const float* xk = xs + (int64_t)k * s.in1;
-    for (int i = 0; i < s.in1; ++i) {
-      const float w = ld_as_f32(Rkp + i);
-#pragma unroll
-      for (int r = 0; r < kMaxRows; ++r)
-        if (r < nr) acc[r] = fmaf(w, xk[r * n_in + i], acc[r]);
-    }
+    fma_rows(acc, R + idx * s.in1, 1, xs + (int64_t)k * s.in1, n_in, 1, s.in1, nr);
     const int64_t t = (int64_t)p * s.nb1 + k;
 #pragma unroll
     for (int r = 0; r < kMaxRows; ++r)
@@ -73,14 +98,7 @@ __global__ void __launch_bounds__(kGenThreads)
     float acc[kMaxRows];
 #pragma unroll
     for (int r = 0; r < kMaxRows; ++r) acc[r] = 0.f;
-    const T* Ljo = L + idx * s.in2;
-    const float* zj = zs + (int64_t)j * s.in2;
-    for (int q = 0; q < s.in2; ++q) {
-      const float w = ld_as_f32(Ljo + q);
-#pragma unroll
-      for (int r = 0; r < kMaxRows; ++r)
-        if (r < nr) acc[r] = fmaf(w, zj[r * n_mid + q], acc[r]);
-    }
+    fma_rows(acc, L + idx * s.in2, 1, zs + (int64_t)j * s.in2, n_mid, 1, s.in2, nr);
     const int64_t col = s.out_index(j, o);
 #pragma unroll
     for (int r = 0; r < kMaxRows; ++r)
@@ -116,14 +134,7 @@ __global__ void __launch_bounds__(kGenThreads)
     float acc[kMaxRows];
 #pragma unroll
     for (int r = 0; r < kMaxRows; ++r) acc[r] = 0.f;
-    const T* Ljq = L + (int64_t)j * s.out2 * s.in2 + q;
-    const float* dvj = dvs + (int64_t)j * s.out2;
-    for (int o = 0; o < s.out2; ++o) {
-      const float w = ld_as_f32(Ljq + (int64_t)o * s.in2);
-#pragma unroll
-      for (int r = 0; r < kMaxRows; ++r)
-        if (r < nr) acc[r] = fmaf(w, dvj[r * n_out + o], acc[r]);
-    }
+    fma_rows(acc, L + (int64_t)j * s.out2 * s.in2 + q, s.in2, dvs + (int64_t)j * s.out2, n_out, 1, s.out2, nr);
 #pragma unroll
     for (int r = 0; r < kMaxRows; ++r)
       if (r < nr) dzs[r * n_mid + idx] = acc[r];
@@ -135,14 +146,8 @@ __global__ void __launch_bounds__(kGenThreads)
     float acc[kMaxRows];
 #pragma unroll
     for (int r = 0; r < kMaxRows; ++r) acc[r] = 0.f;
-    const T* Rki = R + (int64_t)k * s.out1 * s.in1 + i;
-    for (int p = 0; p < s.out1; ++p) {
-      const float w = ld_as_f32(Rki + (int64_t)p * s.in1);
-      const int64_t t = (int64_t)p * s.nb1 + k;
-#pragma unroll
-      for (int r = 0; r < kMaxRows; ++r)
-        if (r < nr) acc[r] = fmaf(w, dzs[r * n_mid + t], acc[r]);
-    }
+    // dZflat index of p is p*nb1 + k
+    fma_rows(acc, R + (int64_t)k * s.out1 * s.in1 + i, s.in1, dzs + k, n_mid, s.nb1, s.out1, nr);
 #pragma unroll
     for (int r = 0; r < kMaxRows; ++r)
       if (r < nr) st_from_f32(dX + (r0 + r) * n_in + idx, acc[r]);
@@ -172,14 +177,36 @@ __global__ void __launch_bounds__(kGenThreads)
     const int64_t rem = e % ((int64_t)s.out1 * s.in1);
     const int p = (int)(rem / s.in1), i = (int)(rem % s.in1);
     const int64_t t = (int64_t)p * s.nb1 + k, c = (int64_t)k * s.in1 + i;
-    for (int64_t r = ra; r < rb; ++r) acc = fmaf(wsdZ[r * n_mid + t], ld_as_f32(X + r * n_in + c), acc);
+    int64_t r = ra;
+    for (; r + 4 <= rb; r += 4) {
+      float a[4], b[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        a[u] = wsdZ[(r + u) * n_mid + t];
+        b[u] = ld_as_f32(X + (r + u) * n_in + c);
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) acc = fmaf(a[u], b[u], acc);
+    }
+    for (; r < rb; ++r) acc = fmaf(wsdZ[r * n_mid + t], ld_as_f32(X + r * n_in + c), acc);
   } else {
     const int64_t e2 = e - nR;
     const int j = (int)(e2 / ((int64_t)s.out2 * s.in2));
     const int64_t rem = e2 % ((int64_t)s.out2 * s.in2);
     const int o = (int)(rem / s.in2), q = (int)(rem % s.in2);
     const int64_t col = s.out_index(j, o), t = (int64_t)j * s.in2 + q;
-    for (int64_t r = ra; r < rb; ++r) acc = fmaf(ld_as_f32(dY + r * n_out + col), wsZ[r * n_mid + t], acc);
+    int64_t r = ra;
+    for (; r + 4 <= rb; r += 4) {
+      float a[4], b[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        a[u] = ld_as_f32(dY + (r + u) * n_out + col);
+        b[u] = wsZ[(r + u) * n_mid + t];
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) acc = fmaf(a[u], b[u], acc);
+    }
+    for (; r < rb; ++r) acc = fmaf(ld_as_f32(dY + r * n_out + col), wsZ[r * n_mid + t], acc);
   }
   partial[(int64_t)sp * nP + e] = acc;
 }
@@ -192,7 +219,15 @@ __global__ void __launch_bounds__(kGenThreads)
   const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (e >= nP) return;
   float acc = 0.f;
-  for (int sp = 0; sp < nsplit; ++sp) acc += partial[(int64_t)sp * nP + e];
+  int sp = 0;
+  for (; sp + 8 <= nsplit; sp += 8) {
+    float v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) v[u] = partial[(int64_t)(sp + u) * nP + e];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) acc += v[u];
+  }
+  for (; sp < nsplit; ++sp) acc += partial[(int64_t)sp * nP + e];
   if (e < nR)
     st_from_f32(dR + e, acc);
   else
@@ -232,8 +267,8 @@ __global__ void __launch_bounds__(kGenThreads)
 template <typename T>
 static cudaError_t launch_fwd(const void* X, const void* R, const void* L, void* Y, const Shape& s,
                               cudaStream_t st) {
-  const int rpc = gen_rows_per_cta(s.n_in() + s.n_mid());
-  if (rpc < 1) return cudaErrorNotSupported;
+  if (gen_rows_per_cta(s.n_in() + s.n_mid()) < 1) return cudaErrorNotSupported;
+  const int rpc = gen_rows_for(s.rows, s.n_in() + s.n_mid());
   const size_t smem = sizeof(float) * (size_t)rpc * (size_t)(s.n_in() + s.n_mid());
   cudaError_t e = ensure_smem_attr((const void*)gen_fwd_kernel<T>, (int)smem);
   if (e != cudaSuccess) return e;
@@ -253,8 +288,8 @@ static int gen_nsplit(const Shape& s) {
   const int64_t nP = s.n_R() + s.n_L();
   int64_t n = (int64_t(1) << 21) / (nP > 0 ? nP : 1);
   if (n > 64) n = 64;
+  if (n > s.rows / 8) n = s.rows / 8;  // at least eight rows per split
   if (n < 1) n = 1;
-  if (n > s.rows) n = s.rows > 0 ? s.rows : 1;
   return (int)n;
 }
 
@@ -270,8 +305,8 @@ size_t generic_bwd_workspace(const Shape& s) {
 template <typename T>
 static cudaError_t launch_bwd(const void* dY, const void* X, const void* R, const void* L, void* dX,
                               void* dR, void* dL, void* ws, const Shape& s, cudaStream_t st) {
-  const int rpc = gen_rows_per_cta(s.n_in() + s.n_out() + 2 * s.n_mid());
-  if (rpc < 1) return cudaErrorNotSupported;
+  if (gen_rows_per_cta(s.n_in() + s.n_out() + 2 * s.n_mid()) < 1) return cudaErrorNotSupported;
+  const int rpc = gen_rows_for(s.rows, s.n_in() + s.n_out() + 2 * s.n_mid());
   const size_t zbytes = align256(sizeof(float) * (size_t)s.rows * (size_t)s.n_mid());
   float* wsZ = (float*)ws;
   float* wsdZ = (float*)((char*)ws + zbytes);
