@@ -9,7 +9,9 @@
 //   (the permutation P is the store index); y[out_index(j,o)] = sum_q L[j][o][q] zs[r][j*in2+q].
 // Backward: a row kernel recomputes Z, forms dZ = L^T dV and dX = R^T dU, and
 // spills Z and dZ (fp32) to the workspace; a weight-gradient kernel reduces
-// dR and dL over row splits; a final kernel sums the splits in fixed order.
+// dR and dL over row splits; a final kernel sums the splits in fixed order.  The two
+// later kernels are launched as programmatic dependents of the one before, so their
+// launches overlap it; each waits for its predecessor before reading.
 #include "common.cuh"
 #include "tc_common.cuh"
 
@@ -111,6 +113,7 @@ __global__ void __launch_bounds__(kGenThreads)
     gen_bwd_rows_kernel(const T* __restrict__ dY, const T* __restrict__ X, const T* __restrict__ R,
                         const T* __restrict__ L, T* __restrict__ dX, float* __restrict__ wsZ,
                         float* __restrict__ wsdZ, Shape s, int rpc) {
+  ptx::griddep_launch_dependents();  // the weight-gradient grid waits for this one to complete
   extern __shared__ float sm[];
   const int64_t n_in = s.n_in(), n_mid = s.n_mid(), n_out = s.n_out();
   float* xs = sm;
@@ -165,6 +168,8 @@ __global__ void __launch_bounds__(kGenThreads)
     gen_bwd_wgrad_kernel(const T* __restrict__ dY, const T* __restrict__ X,
                          const float* __restrict__ wsZ, const float* __restrict__ wsdZ,
                          float* __restrict__ partial, Shape s, int nsplit) {
+  ptx::griddep_wait();  // Z and dZ from the row kernel
+  ptx::griddep_launch_dependents();
   const int64_t nR = s.n_R(), nP = s.n_R() + s.n_L();
   const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (e >= nP) return;
@@ -215,6 +220,7 @@ template <typename T>
 __global__ void __launch_bounds__(kGenThreads)
     gen_bwd_reduce_kernel(const float* __restrict__ partial, T* __restrict__ dR,
                           T* __restrict__ dL, Shape s, int nsplit) {
+  ptx::griddep_wait();  // the partials
   const int64_t nR = s.n_R(), nP = s.n_R() + s.n_L();
   const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (e >= nP) return;
@@ -326,11 +332,11 @@ static cudaError_t launch_bwd(const void* dY, const void* X, const void* R, cons
       return e;
   }
   dim3 g((unsigned)((nP + kGenThreads - 1) / kGenThreads), (unsigned)nsplit);
-  if ((e = launch_kernel(gen_bwd_wgrad_kernel<T>, g, dim3(kGenThreads), 0, st, false, (const T*)dY,
+  if ((e = launch_kernel(gen_bwd_wgrad_kernel<T>, g, dim3(kGenThreads), 0, st, true, (const T*)dY,
                          (const T*)X, (const float*)wsZ, (const float*)wsdZ, partial, s, nsplit)) != cudaSuccess)
     return e;
   return launch_kernel(gen_bwd_reduce_kernel<T>, dim3((unsigned)((nP + kGenThreads - 1) / kGenThreads)),
-                       dim3(kGenThreads), 0, st, false, (const float*)partial, (T*)dR, (T*)dL, s, nsplit);
+                       dim3(kGenThreads), 0, st, true, (const float*)partial, (T*)dR, (T*)dL, s, nsplit);
 }
 
 cudaError_t generic_bwd(const void* dY, const void* X, const void* R, const void* L, void* dX,
